@@ -1,0 +1,540 @@
+"""SparsePR per-call sparse attention: a plain fp64 CPU oracle.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import or call this
+module: only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg use it.  It shares no code with the CUDA library (no kernels, headers, tables or
+helpers) and imports nothing from the product package.
+
+Sources.  [P] = "Partition the Support, Reconstruct the Residual: Training-Free Sparse
+Attention for Video Generation and World Models" (the paper text; its display
+equations were lost in extraction, so several formulas are re-derived from the
+sentences around them).  [R] = the paper.rainbus.top review of the same paper, which
+restates the pipeline with concrete values (w_p = |G_a^Q|/m_a, lambda = 0.1, r = 16,
+the subspace Psi_r, dense output on probe rows).  Section labels of [P] are inferred
+from its content: S2 problem setup, S4.1 Response-Coupled Partitioning (RCP), S4.2
+Probe-Fitted Residual Reconstruction (PFRR), S4.3 routing budget, App. A.1 hard-drop
+derivation, App. A.2 probe selection (Algorithm A.1), App. A.3 estimator statistics,
+App. B.1 key metric, App. B.2 query metric and RMS normalisation, App. B.3 routing,
+App. C implementation, App. D ablations.
+
+Readings where the pages are silent (each is listed in the design doc):
+  S1  evenly spaced sample rows are floor(s*N_q/M_s), s = 0..M_s-1 (all rows if M_s >= N_q)
+  S2  M_K = (1/M_s) Q_s^T Q_s, the unique symmetric matrix with
+      dk M_K dk^T = mean_s (q_s . dk)^2
+  S3  eigenvalues normalised to unit mean over the retained r; negatives clamped to 0
+  S5  k-means assignment ties go to the lowest centre index
+  S6  an empty cluster keeps its previous centre
+  S7  k-means stops after max_iter assignment steps or when an assignment changes no label
+  S8  k-means init: C rows drawn with replacement by SplitMix64 (counter-based)
+  S9  phi_Q = z / max(rms(z), 1e-6)
+  S11 routing score (the SVG-EAR value-error score is not on the pages):
+      l_ab = tau qbar_a.kbar_b + ln|G_b|, pi_ab = softmax_b l_ab,
+      ohat_a = sum_b pi_ab vbar_b, score_ab = pi_ab * ||vbar_b - ohat_a||_2
+  S12 score ties ranked by ascending KV group id
+  S14 group-major order keeps ascending original index inside a group
+  S16 probe distance d_i is the squared distance to the group centre in phi_Q space
+  S20 r = 0 means no subspace projection (P = I)
+  S21 singular values <= 1e-10 * sigma_max are dropped before taking the leading r
+
+Parity status: every function here is pinned by tests in ``tests/test_oracle_*.py``
+except ``route_scores``, whose formula is a reading (S11) of a score the pages only
+name: its parity against the SVG-EAR definition is UNPINNED (its stated properties and
+a hand-worked value are pinned).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+import numpy as np
+
+RMS_EPS = 1e-6            # [P] App. B.2: floor of the RMS denominator
+STD_EPS = 1e-6            # [P] App. D.3: sqrt(weighted variance + 1e-6)
+SV_REL_TOL = 1e-10        # [P] App. D.5: relative singular-value tolerance
+
+# ----------------------------------------------------------------------------------
+# S8: SplitMix64 (Steele, Lea & Flood, "Fast Splittable Pseudorandom Number
+# Generators", OOPSLA 2014), used in counter form: output n of a generator whose
+# state starts at `key` is mix(key + n * GAMMA), n = 1, 2, ...
+_M64 = (1 << 64) - 1
+_GAMMA = 0x9E3779B97F4A7C15
+
+
+def _mix64(z: int) -> int:
+    z &= _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def kmeans_init_indices(seed: int, head: int, stage: int, C: int, N: int) -> np.ndarray:
+    """Initial centre rows: C draws with replacement from [0, N) ([P] App. C: "initial
+    k means centers are sampled uniformly with replacement from feature rows").
+
+    stage 0 = key clustering, 1 = query clustering.  The stream key is output number
+    (2*head + stage + 1) of SplitMix64 seeded with `seed`; draw c uses output c+1 of
+    the generator keyed by it, mapped to an index by the high 32 bits:
+    idx = (hi32 * N) >> 32.
+    """
+    key = _mix64(seed + (2 * head + stage + 1) * _GAMMA)
+    out = np.empty(C, dtype=np.int64)
+    for c in range(C):
+        z = _mix64(key + (c + 1) * _GAMMA)
+        out[c] = ((z >> 32) * N) >> 32
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# RCP: key side ([P] S4.1 "Key-response coordinates", App. B.1)
+
+def sample_rows(N_q: int, M_s: int) -> np.ndarray:
+    """S1: M_s query rows at deterministic evenly spaced token positions."""
+    if M_s >= N_q:
+        return np.arange(N_q, dtype=np.int64)
+    return (np.arange(M_s, dtype=np.int64) * N_q) // M_s
+
+
+def key_metric(Q: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """S2: key response metric M_K = (1/M_s) Q_s^T Q_s ([P] S4.1, App. B.1)."""
+    Qs = Q[rows]
+    return (Qs.T @ Qs) / Qs.shape[0]
+
+
+def eigen_factor(Msym: np.ndarray, r: int):
+    """Eigenvalue-weighted factor F (d x r) of a symmetric PSD metric.
+
+    [P] S4.1 / App. B.1: keep the leading r eigenvectors, normalise their eigenvalues
+    to unit mean (S3: mean over the r kept), and scale each eigenvector by the square
+    root of its normalised eigenvalue.  Returns (F, kept eigenvalues, eigenvectors).
+    """
+    w, U = np.linalg.eigh(Msym)
+    order = np.argsort(-w, kind="stable")[:r]
+    lam = np.maximum(w[order], 0.0)
+    mean = lam.mean()
+    if not mean > 0.0:
+        raise ValueError("metric has no positive eigenvalue among the leading r")
+    Ur = U[:, order]
+    return Ur * np.sqrt(lam / mean)[None, :], lam, Ur
+
+
+# ----------------------------------------------------------------------------------
+# k-means ([P] S4.1, App. C: Lloyd iterations, fresh centres, at most 25 iterations)
+
+@dataclass
+class KMeansResult:
+    labels: np.ndarray          # int64 [N], in [0, C)
+    centres: np.ndarray         # fp64 [C, r], means of the final labels (S6 for empties)
+    iterations: int             # assignment steps taken
+    objective: float            # sum_i ||x_i - c_label(i)||^2 at the final centres
+    history: List[float] = field(default_factory=list)  # objective after each update
+
+
+def _assign(X: np.ndarray, centres: np.ndarray) -> np.ndarray:
+    # squared Euclidean distances; np.argmin returns the lowest index on ties (S5)
+    d2 = (X * X).sum(1)[:, None] - 2.0 * (X @ centres.T) + (centres * centres).sum(1)[None, :]
+    return np.argmin(d2, axis=1)
+
+
+def _update(X: np.ndarray, labels: np.ndarray, centres: np.ndarray) -> np.ndarray:
+    C = centres.shape[0]
+    counts = np.bincount(labels, minlength=C)
+    sums = np.zeros_like(centres)
+    np.add.at(sums, labels, X)
+    new = centres.copy()
+    nz = counts > 0
+    new[nz] = sums[nz] / counts[nz][:, None]          # S6: empty clusters keep theirs
+    return new
+
+
+def objective(X: np.ndarray, labels: np.ndarray, centres: np.ndarray) -> float:
+    diff = X - centres[labels]
+    return float((diff * diff).sum())
+
+
+def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int) -> KMeansResult:
+    """Lloyd's algorithm: assign to the nearest centre, move centres to member means.
+
+    S7: stop after `max_iter` assignment steps or as soon as an assignment step leaves
+    every label unchanged.  The returned centres are the means of the returned labels.
+    """
+    centres = X[init_idx].copy()
+    labels = None
+    it = 0
+    history = []
+    for _ in range(max_iter):
+        new = _assign(X, centres)
+        it += 1
+        if labels is not None and np.array_equal(new, labels):
+            break
+        labels = new
+        centres = _update(X, labels, centres)
+        history.append(objective(X, labels, centres))
+    return KMeansResult(labels, centres, it, objective(X, labels, centres), history)
+
+
+# ----------------------------------------------------------------------------------
+# RCP: query side ([P] S4.1 "Query-response coordinates", App. B.2)
+
+@dataclass
+class Groups:
+    """Non-empty groups of a labelling, renumbered 0..C'-1 in ascending label order."""
+    compact: np.ndarray      # int64 [N] compact group id of each row
+    sizes: np.ndarray        # int64 [C'] member counts
+    labels_used: np.ndarray  # int64 [C'] original label of each compact id
+
+
+def compact_groups(labels: np.ndarray, C: int) -> Groups:
+    counts = np.bincount(labels, minlength=C)
+    used = np.flatnonzero(counts > 0)
+    remap = -np.ones(C, dtype=np.int64)
+    remap[used] = np.arange(used.size)
+    return Groups(remap[labels], counts[used], used)
+
+
+def group_means(X: np.ndarray, g: Groups) -> np.ndarray:
+    sums = np.zeros((g.sizes.size, X.shape[1]))
+    np.add.at(sums, g.compact, X)
+    return sums / g.sizes[:, None]
+
+
+def centred_key_centroids(kbar: np.ndarray) -> np.ndarray:
+    """[P] S4.1 / App. B.2: subtract the uniform mean of the non-empty group centroids."""
+    return kbar - kbar.mean(axis=0, keepdims=True)
+
+
+def query_metric(Ktil: np.ndarray) -> np.ndarray:
+    """M_Q = (1/C_k') K~^T K~: each non-empty KV group weighs equally ([P] App. B.2)."""
+    return (Ktil.T @ Ktil) / Ktil.shape[0]
+
+
+def query_coords(Q: np.ndarray, F_Q: np.ndarray) -> np.ndarray:
+    """phi_Q(q) = z / max(rms(z), eps), z = q F_Q; no gain, no bias ([P] S4.1, App. B.2)."""
+    z = Q @ F_Q
+    rms = np.sqrt((z * z).mean(axis=1))
+    return z / np.maximum(rms, RMS_EPS)[:, None]
+
+
+# ----------------------------------------------------------------------------------
+# Routing ([P] App. B.3, S4.3)
+
+def route_scores(qbar: np.ndarray, kbar: np.ndarray, vbar: np.ndarray,
+                 size_b: np.ndarray, d: int) -> np.ndarray:
+    """S11 (reading; the SVG-EAR formula is not on the pages; parity unpinned against it).
+
+    Centroid estimate of how much dropping KV group b moves query group a's output:
+    the estimated attention mass of b times the distance of b's value centroid from
+    the estimated output, following the hard-drop identity of [P] App. A.1.
+    """
+    tau = 1.0 / math.sqrt(d)
+    logits = tau * (qbar @ kbar.T) + np.log(size_b.astype(np.float64))[None, :]
+    logits -= logits.max(axis=1, keepdims=True)
+    pi = np.exp(logits)
+    pi /= pi.sum(axis=1, keepdims=True)
+    ohat = pi @ vbar
+    S = np.empty_like(pi)
+    for a in range(pi.shape[0]):
+        S[a] = pi[a] * np.sqrt(((vbar - ohat[a][None, :]) ** 2).sum(axis=1))
+    return S
+
+
+def route_budget(rho_target: float, M: int, N_q: int, N_k: int) -> float:
+    """[P] S4.3: the router reserves the probe cost, rho*_route = rho* - M/N_q; the common
+    per-query key-token budget is rho*_route * N_k."""
+    return (rho_target - float(M) / float(N_q)) * float(N_k)
+
+
+def select_cells(S: np.ndarray, size_b: np.ndarray, beta: float) -> List[np.ndarray]:
+    """[P] App. B.3: rank non-empty KV groups by decreasing score (S12: ties by id) and keep
+    the shortest prefix whose key-token count reaches beta (all groups if none does).
+    Each query group's selected ids are returned in ascending order."""
+    C_k = S.shape[1]
+    ids = np.arange(C_k)
+    sel = []
+    for a in range(S.shape[0]):
+        order = np.lexsort((ids, -S[a]))
+        csum = np.cumsum(size_b[order]).astype(np.float64)
+        hit = np.flatnonzero(csum >= beta)
+        k = (hit[0] + 1) if hit.size else C_k
+        sel.append(np.sort(order[:k]))
+    return sel
+
+
+def executed_pairs(size_a: np.ndarray, size_b: np.ndarray, sel: List[np.ndarray]) -> int:
+    """Routed query-key interactions: each selected cell costs |G_a^Q| |G_b^KV| ([P] S2)."""
+    return int(sum(int(size_a[a]) * int(size_b[s].sum()) for a, s in enumerate(sel)))
+
+
+# ----------------------------------------------------------------------------------
+# Group-major permutation ([R] step 3: Q, K, V rearranged group-major, output restored)
+
+def group_major_permutation(compact: np.ndarray, n_groups: int):
+    """S14: stable order by group id; returns (perm, offsets) with perm[pos] = row."""
+    perm = np.argsort(compact, kind="stable")
+    sizes = np.bincount(compact, minlength=n_groups)
+    offsets = np.concatenate([[0], np.cumsum(sizes)])
+    return perm, offsets
+
+
+# ----------------------------------------------------------------------------------
+# Attention ([P] S2: dense attention and renormalised hard drop)
+
+def attention_rows(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """softmax(tau q K^T) V for rows q, with tau = 1/sqrt(d) ([P] S4.1: the common 1/sqrt(d)
+    scale).  Renormalised hard drop is this same formula over the retained keys only."""
+    tau = 1.0 / math.sqrt(q.shape[1])
+    logits = tau * (q @ K.T)
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    return (p @ V) / p.sum(axis=1, keepdims=True)
+
+
+def sparse_attention(Q, K, V, gq: Groups, gk: Groups, sel: List[np.ndarray],
+                     rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """O^sp for `rows` (default all): row i in query group a attends, with softmax
+    renormalised over them, to the keys of the KV groups selected for a ([P] S2)."""
+    rows = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
+    out = np.empty((rows.size, V.shape[1]))
+    members_k = [np.flatnonzero(gk.compact == b) for b in range(gk.sizes.size)]
+    ga = gq.compact[rows]
+    for a in np.unique(ga):
+        pos = np.flatnonzero(ga == a)
+        keys = np.concatenate([members_k[b] for b in sel[a]])
+        out[pos] = attention_rows(Q[rows[pos]], K[keys], V[keys])
+    return out
+
+
+def dense_attention(Q, K, V, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    rows = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
+    out = np.empty((rows.size, V.shape[1]))
+    for s in range(0, rows.size, 512):
+        out[s:s + 512] = attention_rows(Q[rows[s:s + 512]], K, V)
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# PFRR ([P] S4.2, App. A.2-A.3, App. D; [R] step 4)
+
+def probe_distances(phiQ: np.ndarray, cQ_compact: np.ndarray, gq: Groups) -> np.ndarray:
+    """S16: d_i = ||phi_Q(q_i) - c_a||^2 for i in G_a, c_a the group's phi_Q centre."""
+    diff = phiQ - cQ_compact[gq.compact]
+    return (diff * diff).sum(axis=1)
+
+
+def select_probes(dist: np.ndarray, gq: Groups, M: int):
+    """Algorithm A.1 ([P] App. A.2): stratified radial round robin.
+
+    Rows inside a group by increasing d_i (ties by row index); non-empty groups by
+    decreasing size (ties by group index); each pass takes the next row of every group
+    that still has one; stop after M distinct probes.  Returns (probes in selection
+    order, m_a = number of probes per compact group).
+    """
+    n_groups = gq.sizes.size
+    if M > gq.compact.size:
+        raise ValueError("more probes than query rows")
+    ranked = []
+    for a in range(n_groups):
+        mem = np.flatnonzero(gq.compact == a)
+        ranked.append(mem[np.lexsort((mem, dist[mem]))])
+    order = np.lexsort((np.arange(n_groups), -gq.sizes))
+    probes = []
+    t = 0
+    while len(probes) < M:
+        for a in order:
+            if t < ranked[a].size:
+                probes.append(int(ranked[a][t]))
+                if len(probes) == M:
+                    break
+        t += 1
+    probes = np.array(probes, dtype=np.int64)
+    m_a = np.bincount(gq.compact[probes], minlength=n_groups)
+    return probes, m_a
+
+
+@dataclass
+class Fit:
+    mu_x: np.ndarray
+    mu_R: np.ndarray
+    s: np.ndarray
+    B: np.ndarray          # d x d weighted ridge coefficients on standardised features
+    P: np.ndarray          # d x d projector Psi_r Psi_r^T (identity when r == 0)
+    r_eff: int
+    sigma: np.ndarray      # singular values of Omega^{1/2} R_bar
+
+
+def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int) -> Fit:
+    """Coverage-weighted ridge fit of the residual on the sparse output.
+
+    [P] App. A.3: weights normalised to unit sum give mu_x, mu_R and the elementwise
+    scale s = sqrt(weighted variance + 1e-6) ([P] App. D.3); x_bar = (x - mu_x) / s,
+    R_bar = R - mu_R.  Weights normalised to unit mean (omega) weigh the ridge objective
+    sum_p omega_p ||R_bar_p - x_bar_p B||^2 + lambda ||B||_F^2 ([P] S4.2), whose
+    minimiser is (X^T Omega X + lambda I)^-1 X^T Omega R.  [P] App. D.2 / [R] step 4: the
+    centred prediction is projected on the leading r right singular vectors of
+    Omega^{1/2} R_bar.
+    """
+    M, d = x.shape
+    wt = w / w.sum()
+    mu_x = wt @ x
+    mu_R = wt @ R
+    s = np.sqrt(wt @ ((x - mu_x) ** 2) + STD_EPS)
+    xb = (x - mu_x) / s
+    Rb = R - mu_R
+    omega = M * w / w.sum()
+    lhs = xb.T @ (omega[:, None] * xb) + lam * np.eye(d)
+    rhs = xb.T @ (omega[:, None] * Rb)
+    B = np.linalg.solve(lhs, rhs)
+    Y = np.sqrt(omega)[:, None] * Rb
+    _, sig, Vt = np.linalg.svd(Y, full_matrices=False)
+    if r == 0:
+        return Fit(mu_x, mu_R, s, B, np.eye(d), d, sig)
+    keep = int((sig > SV_REL_TOL * sig[0]).sum()) if sig[0] > 0 else 0
+    r_eff = min(r, keep)
+    Psi = Vt[:r_eff].T
+    return Fit(mu_x, mu_R, s, B, Psi @ Psi.T, r_eff, sig)
+
+
+def correct_rows(xs: np.ndarray, fit: Fit) -> np.ndarray:
+    """Unprobed rows: O_hat = O^sp + mu_R + ((O^sp - mu_x) / s) B P ([R] step 5; [P] App. D.2)."""
+    return xs + fit.mu_R[None, :] + (((xs - fit.mu_x) / fit.s) @ fit.B) @ fit.P
+
+
+# ----------------------------------------------------------------------------------
+# The whole call for one head
+
+@dataclass
+class Params:
+    d: int
+    M_s: int
+    r_K: int
+    r_Q: int
+    C_q: int
+    C_k: int
+    M: int
+    r: int
+    lam: float
+    rho: float
+    kmeans_max_iter: int = 25
+    seed: int = 0
+
+    @classmethod
+    def from_dict(cls, p: Dict) -> "Params":
+        return cls(d=p["d"], M_s=p["M_s"], r_K=p["r_K"], r_Q=p["r_Q"], C_q=p["C_q"],
+                   C_k=p["C_k"], M=p["M"], r=p["r"], lam=p["lam"],
+                   rho=p["target_density"], kmeans_max_iter=p["kmeans_max_iter"],
+                   seed=p["seed"])
+
+
+@dataclass
+class Partition:
+    """Response-Coupled Partitioning of one head ([P] S4.1)."""
+    sample: np.ndarray
+    M_K: np.ndarray
+    F_K: np.ndarray
+    lam_K: np.ndarray
+    phiK: np.ndarray
+    km_K: KMeansResult
+    gk: Groups
+    kbar: np.ndarray
+    vbar: np.ndarray
+    Ktil: np.ndarray
+    M_Q: np.ndarray
+    F_Q: np.ndarray
+    lam_Q: np.ndarray
+    phiQ: np.ndarray
+    km_Q: KMeansResult
+    gq: Groups
+    qbar: np.ndarray
+
+
+def partition(Q, K, V, p: Params, head: int) -> Partition:
+    N_q, N_k = Q.shape[0], K.shape[0]
+    rows = sample_rows(N_q, p.M_s)
+    M_K = key_metric(Q, rows)
+    F_K, lam_K, _ = eigen_factor(M_K, p.r_K)
+    phiK = K @ F_K
+    km_K = kmeans(phiK, kmeans_init_indices(p.seed, head, 0, p.C_k, N_k), p.kmeans_max_iter)
+    gk = compact_groups(km_K.labels, p.C_k)
+    kbar = group_means(K, gk)
+    vbar = group_means(V, gk)
+    Ktil = centred_key_centroids(kbar)
+    M_Q = query_metric(Ktil)
+    F_Q, lam_Q, _ = eigen_factor(M_Q, p.r_Q)
+    phiQ = query_coords(Q, F_Q)
+    km_Q = kmeans(phiQ, kmeans_init_indices(p.seed, head, 1, p.C_q, N_q), p.kmeans_max_iter)
+    gq = compact_groups(km_Q.labels, p.C_q)
+    qbar = group_means(Q, gq)
+    return Partition(rows, M_K, F_K, lam_K, phiK, km_K, gk, kbar, vbar, Ktil, M_Q, F_Q,
+                     lam_Q, phiQ, km_Q, gq, qbar)
+
+
+@dataclass
+class CallResult:
+    part: Partition
+    scores: np.ndarray
+    beta: float
+    sel: List[np.ndarray]
+    pairs_route: int
+    pairs_exec: int
+    rho_route: float
+    rho_exec: float
+    permQ: np.ndarray
+    offQ: np.ndarray
+    permK: np.ndarray
+    offK: np.ndarray
+    probes: np.ndarray
+    m_a: np.ndarray
+    probe_dist: np.ndarray
+    weights: np.ndarray
+    x_probe: np.ndarray
+    dense_probe: np.ndarray
+    fit: Fit
+    rows: np.ndarray         # rows of `out`, `osp`
+    osp: np.ndarray          # sparse output on `rows`
+    out: np.ndarray          # corrected output on `rows`
+
+
+def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] = None,
+                  part: Optional[Partition] = None) -> CallResult:
+    """One SparsePR attention call for one head, in the pages' order.
+
+    `rows` limits the rows whose sparse and corrected outputs are formed (the fit only
+    needs the probe rows); `part` reuses a partition computed earlier for this head.
+    """
+    N_q, N_k = Q.shape[0], K.shape[0]
+    part = partition(Q, K, V, p, head) if part is None else part
+    gq, gk = part.gq, part.gk
+    S = route_scores(part.qbar, part.kbar, part.vbar, gk.sizes, p.d)
+    beta = route_budget(p.rho, p.M, N_q, N_k)
+    sel = select_cells(S, gk.sizes, beta)
+    pairs = executed_pairs(gq.sizes, gk.sizes, sel)
+    pairs_exec = pairs + p.M * N_k                       # [P] S4.3: probes add M/N_q
+    permQ, offQ = group_major_permutation(gq.compact, gq.sizes.size)
+    permK, offK = group_major_permutation(gk.compact, gk.sizes.size)
+    cQ = part.km_Q.centres[gq.labels_used]
+    dist = probe_distances(part.phiQ, cQ, gq)
+    probes, m_a = select_probes(dist, gq, p.M)
+    a_of = gq.compact[probes]
+    w = gq.sizes[a_of].astype(np.float64) / m_a[a_of]  # [R] step 4: w_p = |G_a^Q| / m_a
+    x_probe = sparse_attention(Q, K, V, gq, gk, sel, probes)
+    dense_probe = dense_attention(Q, K, V, probes)
+    fit = fit_residual(x_probe, dense_probe - x_probe, w, p.lam, p.r)
+    rows = np.arange(N_q) if rows is None else np.asarray(rows)
+    osp = sparse_attention(Q, K, V, gq, gk, sel, rows)
+    out = correct_rows(osp, fit)
+    is_probe = np.zeros(N_q, dtype=bool)
+    is_probe[probes] = True
+    where = np.flatnonzero(is_probe[rows])
+    if where.size:                                       # [R] step 5: probes keep dense output
+        lookup = {int(pr): k for k, pr in enumerate(probes)}
+        out[where] = dense_probe[[lookup[int(i)] for i in rows[where]]]
+    return CallResult(part, S, beta, sel, pairs, pairs_exec, pairs / (N_q * N_k),
+                      pairs_exec / (N_q * N_k), permQ, offQ, permK, offK, probes, m_a,
+                      dist, w, x_probe, dense_probe, fit, rows, osp, out)
+
+
+def cell_csr(sel: List[np.ndarray]):
+    """Selected cells as (row pointer, KV group ids) with ids ascending per query group."""
+    ptr = np.concatenate([[0], np.cumsum([s.size for s in sel])]).astype(np.int64)
+    ids = np.concatenate(sel).astype(np.int64) if sel else np.zeros(0, np.int64)
+    return ptr, ids

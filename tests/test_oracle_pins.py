@@ -1,0 +1,479 @@
+"""Pins of the fp64 oracle against what the SparsePR pages and the mathematics fix.
+
+Every check here uses something other than the oracle's own formula: hand-worked
+values (tests/golden/), closed forms, library routines on special cases, identities the
+paper states, and brute force on tiny inputs.  CPU only.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import GOLDEN
+from oracle import sparsepr_oracle as O
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- sampling / RNG
+def test_sample_rows_evenly_spaced():
+    assert O.sample_rows(10, 4).tolist() == [0, 2, 5, 7]          # floor(s*10/4)
+    assert O.sample_rows(1024, 64).tolist() == list(range(0, 1024, 16))
+    assert O.sample_rows(5, 8).tolist() == [0, 1, 2, 3, 4]        # all rows if fewer
+
+
+def test_splitmix64_published_vector():
+    g = _golden("splitmix64_seed1234567.json")
+    x = g["seed"]
+    outs = []
+    for _ in range(5):
+        x = (x + O._GAMMA) & O._M64
+        outs.append(O._mix64(x))
+    assert outs == [int(v) for v in g["outputs"]]
+
+
+def test_kmeans_init_indices_range_and_uniformity():
+    idx = O.kmeans_init_indices(0, 3, 1, 20000, 1000)
+    assert idx.min() >= 0 and idx.max() < 1000
+    counts = np.bincount(idx, minlength=1000)
+    chi2 = ((counts - 20.0) ** 2 / 20.0).sum()
+    assert 850 < chi2 < 1150          # 999 dof: mean 999, sd ~45
+    # streams of different heads / stages differ
+    assert not np.array_equal(O.kmeans_init_indices(0, 0, 0, 64, 1000),
+                              O.kmeans_init_indices(0, 0, 1, 64, 1000))
+
+
+# ---------------------------------------------------------------- key metric / factor
+def test_key_metric_is_average_squared_response_difference():
+    rng = _rng(1)
+    Q = rng.standard_normal((50, 6))
+    rows = O.sample_rows(50, 7)
+    MK = O.key_metric(Q, rows)
+    for _ in range(5):
+        dk = rng.standard_normal(6)
+        brute = sum(float(np.dot(Q[i], dk)) ** 2 for i in rows) / len(rows)
+        assert abs(dk @ MK @ dk - brute) <= 1e-12 * brute
+
+
+def test_eigen_factor_diagonal_closed_form():
+    M = np.diag([4.0, 1.0, 9.0])
+    F, lam, _ = O.eigen_factor(M, 2)
+    assert np.allclose(lam, [9.0, 4.0])
+    expect = np.zeros((3, 2))
+    expect[2, 0] = math.sqrt(9.0 / 6.5)
+    expect[0, 1] = math.sqrt(4.0 / 6.5)
+    assert np.allclose(np.abs(F), expect, atol=1e-14)
+
+
+def test_eigen_factor_full_rank_reproduces_metric_up_to_scale():
+    rng = _rng(2)
+    A = rng.standard_normal((40, 8))
+    M = A.T @ A / 40
+    F, lam, U = O.eigen_factor(M, 8)
+    scale = lam.mean()
+    for _ in range(5):
+        x, y = rng.standard_normal(8), rng.standard_normal(8)
+        lhs = np.sum(((x - y) @ F) ** 2)
+        rhs = (x - y) @ M @ (x - y) / scale
+        assert abs(lhs - rhs) <= 1e-12 * rhs
+    # F F^T = U_r diag(lam_hat) U_r^T and eigen-residuals vanish
+    assert np.allclose(F @ F.T, U @ np.diag(lam / scale) @ U.T, atol=1e-13)
+    assert np.abs(M @ U - U * lam[None, :]).max() < 1e-12
+
+
+def test_eigen_factor_rejects_zero_metric():
+    with pytest.raises(ValueError):
+        O.eigen_factor(np.zeros((4, 4)), 2)
+
+
+# ---------------------------------------------------------------- k-means
+def test_kmeans_hand_worked():
+    g = _golden("kmeans_1d.json")
+    X = np.array(g["points"])
+    res = O.kmeans(X, np.array(g["init_idx"]), g["max_iter"])
+    assert res.labels.tolist() == g["labels"]
+    assert np.allclose(res.centres, g["centres"], atol=0)
+    assert res.iterations == g["iterations"]
+    assert res.objective == g["objective"]
+    one = O.kmeans(X, np.array(g["init_idx"]), 1)
+    assert one.labels.tolist() == g["labels_max_iter_1"]
+    assert np.allclose(one.centres, g["centres_max_iter_1"], rtol=1e-15)
+
+
+def test_kmeans_matches_sklearn_lloyd():
+    from sklearn.cluster import KMeans
+    rng = _rng(3)
+    centres = rng.standard_normal((6, 4)) * 6
+    X = np.concatenate([c + rng.standard_normal((40, 4)) for c in centres])
+    init = np.array([0, 41, 85, 130, 170, 201])
+    res = O.kmeans(X, init, 50)
+    km = KMeans(n_clusters=6, init=X[init], n_init=1, algorithm="lloyd", max_iter=50, tol=0.0)
+    km.fit(X)
+    assert res.iterations < 50
+    assert np.array_equal(res.labels, km.labels_)
+    assert np.allclose(res.centres, km.cluster_centers_, atol=1e-12)
+
+
+def test_kmeans_brute_force_fixed_point_tiny():
+    rng = _rng(4)
+    for trial in range(30):
+        N, C = rng.integers(3, 9), rng.integers(1, 4)
+        X = rng.standard_normal((N, 2))
+        init = rng.integers(0, N, C)
+        res = O.kmeans(X, init, 100)
+        # objective never increases
+        assert all(b <= a + 1e-12 for a, b in zip(res.history, res.history[1:]))
+        if res.iterations < 100:
+            # Lloyd fixed point: each point's label is its nearest centre (lowest on ties)
+            for i in range(N):
+                dists = [sum((X[i][k] - res.centres[c][k]) ** 2 for k in range(2)) for c in range(C)]
+                best = min(dists)
+                assert res.labels[i] == dists.index(best)
+            # each non-empty centre is its members' mean
+            for c in range(C):
+                mem = [i for i in range(N) if res.labels[i] == c]
+                if mem:
+                    assert np.allclose(res.centres[c], X[mem].mean(axis=0), atol=1e-14)
+
+
+def test_kmeans_empty_cluster_keeps_centre():
+    # Duplicate init: centre 1 loses every tie (lowest index wins), stays empty after step
+    # 1 and keeps its value 0.0 (S6); step 2 it is nearer to point 0 than centre 0 (now
+    # 0.05), regains it, and step 3 changes nothing.
+    X = np.array([[0.0], [0.1], [5.0]])
+    one = O.kmeans(X, np.array([0, 0, 2]), 1)
+    assert one.labels.tolist() == [0, 0, 2]
+    assert one.centres[:, 0].tolist() == [0.05, 0.0, 5.0]
+    res = O.kmeans(X, np.array([0, 0, 2]), 10)
+    assert res.labels.tolist() == [1, 0, 2]
+    assert res.centres[:, 0].tolist() == [0.1, 0.0, 5.0]
+    assert res.iterations == 3
+
+
+# ---------------------------------------------------------------- query side
+def test_groups_and_centring():
+    g = O.compact_groups(np.array([3, 3, 0, 5]), 6)
+    assert g.compact.tolist() == [1, 1, 0, 2]
+    assert g.sizes.tolist() == [1, 2, 1]
+    assert g.labels_used.tolist() == [0, 3, 5]
+    rng = _rng(5)
+    kbar = rng.standard_normal((7, 5))
+    Kt = O.centred_key_centroids(kbar)
+    assert np.abs(Kt.sum(axis=0)).max() < 1e-14
+    q = rng.standard_normal(5)
+    sm = lambda z: np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+    assert np.allclose(sm(kbar @ q), sm(Kt @ q), atol=1e-15)   # [P] App. B.2
+
+
+def test_query_metric_is_average_squared_centred_logit_difference():
+    rng = _rng(6)
+    Kt = O.centred_key_centroids(rng.standard_normal((9, 4)))
+    MQ = O.query_metric(Kt)
+    for _ in range(5):
+        dq = rng.standard_normal(4)
+        brute = sum(float(np.dot(Kt[b], dq)) ** 2 for b in range(9)) / 9
+        assert abs(dq @ MQ @ dq - brute) <= 1e-12 * brute
+
+
+def test_query_coords_rms_normalisation():
+    rng = _rng(7)
+    Q = rng.standard_normal((20, 6))
+    F = rng.standard_normal((6, 4))
+    phi = O.query_coords(Q, F)
+    assert np.allclose((phi ** 2).mean(axis=1), 1.0, atol=1e-14)
+    assert np.allclose(O.query_coords(3.5 * Q, F), phi, atol=1e-14)   # scale invariant
+    Q[0] = 0.0
+    assert np.all(O.query_coords(Q, F)[0] == 0.0)                   # floor, no NaN
+    tiny = O.query_coords(np.full((1, 6), 1e-9), np.eye(6)[:, :4])
+    assert np.allclose(tiny, 1e-9 / 1e-6)                           # max(rms, eps)
+
+
+# ---------------------------------------------------------------- routing
+def test_route_score_hand_worked():
+    g = _golden("route_score_example.json")
+    for c in g["cases"]:
+        S = O.route_scores(np.array(c["qbar"]), np.array(c["kbar"]), np.array(c["vbar"]),
+                           np.array(c["sizes"]), 1)
+        assert np.allclose(S, c["scores"], atol=1e-15)
+
+
+def test_route_score_singletons_match_hard_drop_of_one_key():
+    # With one key per group and the query at its centroid, pi is the exact attention and
+    # the score equals (1 - pi_b) * || O_dense - O_sp(without b) || (App. A.1 identity).
+    rng = _rng(8)
+    d = 4
+    q = rng.standard_normal((1, d))
+    K = rng.standard_normal((6, d))
+    V = rng.standard_normal((6, d))
+    S = O.route_scores(q, K, V, np.ones(6, dtype=np.int64), d)[0]
+    dense = O.attention_rows(q, K, V)[0]
+    z = np.exp(q @ K.T / math.sqrt(d))[0]
+    pi = z / z.sum()
+    for b in range(6):
+        keep = [j for j in range(6) if j != b]
+        osp = O.attention_rows(q, K[keep], V[keep])[0]
+        assert abs(S[b] - (1 - pi[b]) * np.linalg.norm(dense - osp)) < 1e-12
+
+
+def test_select_cells_hand_worked():
+    g = _golden("cell_selection_example.json")
+    for c in g["cases"]:
+        sel = O.select_cells(np.array(g["scores"]), np.array(g["sizes"]), c["beta"])
+        assert sel[0].tolist() == c["selected"]
+
+
+def test_select_cells_prefix_minimal_and_full_budget():
+    rng = _rng(9)
+    S = rng.random((12, 15))
+    sizes = rng.integers(1, 30, 15)
+    beta = 0.3 * sizes.sum()
+    for a, sel in enumerate(O.select_cells(S, sizes, beta)):
+        assert sizes[sel].sum() >= beta
+        worst = sel[np.argmin(S[a, sel])]
+        assert sizes[sel].sum() - sizes[worst] < beta         # shortest prefix
+        others = np.setdiff1d(np.arange(15), sel)
+        if others.size:
+            assert S[a, sel].min() >= S[a, others].max()
+    for sel in O.select_cells(S, sizes, float(sizes.sum())):
+        assert sel.tolist() == list(range(15))
+
+
+# ---------------------------------------------------------------- permutation
+def test_group_major_permutation():
+    perm, off = O.group_major_permutation(np.array([2, 0, 1, 0, 2, 1]), 3)
+    assert perm.tolist() == [1, 3, 2, 5, 0, 4]
+    assert off.tolist() == [0, 2, 4, 6]
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(6)
+    assert np.array_equal(perm[inv], np.arange(6))
+
+
+# ---------------------------------------------------------------- attention
+def test_dense_attention_matches_torch_sdpa():
+    rng = _rng(10)
+    Q, K, V = (rng.standard_normal((33, 16)) for _ in range(3))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+    assert np.abs(O.dense_attention(Q, K, V) - ref).max() < 1e-13
+
+
+def test_attention_small_closed_forms():
+    rng = _rng(11)
+    q = rng.standard_normal((1, 4))
+    k = rng.standard_normal((1, 4))
+    v = rng.standard_normal((1, 4))
+    assert np.allclose(O.attention_rows(q, k, v), v, atol=1e-15)          # one key
+    K2, V2 = rng.standard_normal((2, 4)), rng.standard_normal((2, 4))
+    delta = float(q[0] @ (K2[0] - K2[1])) / 2.0                           # tau = 1/2
+    p0 = 1.0 / (1.0 + math.exp(-delta))
+    assert np.allclose(O.attention_rows(q, K2, V2)[0], p0 * V2[0] + (1 - p0) * V2[1], atol=1e-14)
+    K5 = rng.standard_normal((5, 4))
+    probs = O.attention_rows(q, K5, np.eye(5))[0]                         # one-hot V
+    z = np.exp(K5 @ q[0] / 2.0)
+    assert np.allclose(probs, z / z.sum(), atol=1e-15)
+
+
+def _tiny_problem(seed=12, N=96, d=8, C=6):
+    rng = _rng(seed)
+    Q, K, V = (rng.standard_normal((N, d)) * 1.5 for _ in range(3))
+    gq = O.compact_groups(rng.integers(0, C, N), C)
+    gk = O.compact_groups(rng.integers(0, C, N), C)
+    return Q, K, V, gq, gk
+
+
+def test_hard_drop_residual_identity():
+    # [P] App. A.1: O_dense - O_sp = p_U (O_U - O_sp), p_U the omitted dense mass.
+    Q, K, V, gq, gk = _tiny_problem()
+    rng = _rng(13)
+    n = gk.sizes.size
+    sel = [np.sort(rng.choice(n, size=rng.integers(1, n), replace=False)) for _ in range(gq.sizes.size)]
+    osp = O.sparse_attention(Q, K, V, gq, gk, sel)
+    dense = O.dense_attention(Q, K, V)
+    comp = [np.setdiff1d(np.arange(n), s) for s in sel]
+    d = Q.shape[1]
+    for i in range(Q.shape[0]):
+        a = gq.compact[i]
+        if comp[a].size == 0:
+            assert np.allclose(osp[i], dense[i], atol=1e-14)
+            continue
+        U = np.flatnonzero(np.isin(gk.compact, comp[a]))
+        z = np.exp(Q[i] @ K.T / math.sqrt(d))
+        pU = z[U].sum() / z.sum()
+        oU = (z[U] @ V[U]) / z[U].sum()
+        lhs = dense[i] - osp[i]
+        rhs = pU * (oU - osp[i])
+        assert np.abs(lhs - rhs).max() <= 1e-12 * max(1.0, np.abs(lhs).max())
+
+
+def test_all_cells_selected_is_dense():
+    Q, K, V, gq, gk = _tiny_problem(seed=14)
+    sel = [np.arange(gk.sizes.size) for _ in range(gq.sizes.size)]
+    assert np.abs(O.sparse_attention(Q, K, V, gq, gk, sel) - O.dense_attention(Q, K, V)).max() < 1e-13
+
+
+# ---------------------------------------------------------------- probes
+def test_probe_selection_hand_worked():
+    g = _golden("probe_selection_example.json")
+    gq = O.compact_groups(np.array(g["labels"]), 3)
+    for c in g["cases"]:
+        probes, m_a = O.select_probes(np.array(g["dist"]), gq, c["M"])
+        assert probes.tolist() == c["probes"]
+        assert m_a.tolist() == c["m_a"]
+
+
+def test_probe_selection_many_groups_takes_nearest_of_largest():
+    # [P] App. A.2: with at least M non-empty groups, the row nearest the centroid of
+    # each of the M largest groups.
+    rng = _rng(15)
+    lab = rng.integers(0, 40, 2000)
+    gq = O.compact_groups(lab, 40)
+    dist = rng.random(2000)
+    probes, m_a = O.select_probes(dist, gq, 16)
+    largest = sorted(range(gq.sizes.size), key=lambda a: (-gq.sizes[a], a))[:16]
+    expect = []
+    for a in largest:
+        mem = [i for i in range(2000) if gq.compact[i] == a]
+        expect.append(min(mem, key=lambda i: (dist[i], i)))
+    assert probes.tolist() == expect
+    assert m_a.sum() == 16 and len(set(probes.tolist())) == 16
+
+
+# ---------------------------------------------------------------- fit / correction
+def _fit_inputs(seed=16, M=40, d=6):
+    rng = _rng(seed)
+    x = rng.standard_normal((M, d)) * rng.random(d) * 3
+    R = rng.standard_normal((M, d))
+    w = rng.integers(1, 9, M).astype(np.float64)
+    return x, R, w
+
+
+def test_ridge_matches_augmented_least_squares_and_dual():
+    x, R, w = _fit_inputs()
+    lam = 0.1
+    f = O.fit_residual(x, R, w, lam, 0)
+    M, d = x.shape
+    # brute force from the definition: minimise sum omega ||Rb - xb B||^2 + lam ||B||^2
+    wt = w / w.sum()
+    mu_x = sum(wt[p] * x[p] for p in range(M))
+    mu_R = sum(wt[p] * R[p] for p in range(M))
+    var = sum(wt[p] * (x[p] - mu_x) ** 2 for p in range(M))
+    s = np.sqrt(var + 1e-6)
+    xb = (x - mu_x) / s
+    Rb = R - mu_R
+    om = w * M / w.sum()
+    assert abs(om.mean() - 1.0) < 1e-15 and abs(wt.sum() - 1.0) < 1e-15
+    A = np.vstack([np.sqrt(om)[:, None] * xb, math.sqrt(lam) * np.eye(d)])
+    Y = np.vstack([np.sqrt(om)[:, None] * Rb, np.zeros((d, d))])
+    B_ls = np.linalg.lstsq(A, Y, rcond=None)[0]
+    assert np.abs(f.B - B_ls).max() < 1e-10
+    Xo = np.sqrt(om)[:, None] * xb
+    B_dual = Xo.T @ np.linalg.inv(Xo @ Xo.T + lam * np.eye(M)) @ (np.sqrt(om)[:, None] * Rb)
+    assert np.abs(f.B - B_dual).max() < 1e-10
+    assert np.allclose(f.mu_x, mu_x) and np.allclose(f.mu_R, mu_R) and np.allclose(f.s, s)
+
+
+def test_ridge_large_lambda_is_mean_only():
+    x, R, w = _fit_inputs(seed=17)
+    f = O.fit_residual(x, R, w, 1e12, 0)
+    assert np.abs(f.B).max() < 1e-9
+    xs = np.random.default_rng(1).standard_normal((5, x.shape[1]))
+    assert np.allclose(O.correct_rows(xs, f), xs + f.mu_R, atol=1e-9)
+
+
+def test_planted_affine_residual_is_recovered():
+    # If the residual is exactly affine in the sparse output, a near-unregularised fit
+    # with r = d recovers it, so corrected outputs are exact on unseen rows.
+    rng = _rng(18)
+    M, d = 60, 5
+    Bt = rng.standard_normal((d, d))          # non-symmetric: a transposed B fails
+    bt = rng.standard_normal(d)
+    x = rng.standard_normal((M, d)) * 2 + 1
+    R = bt + x @ Bt
+    w = rng.integers(1, 5, M).astype(np.float64)
+    f = O.fit_residual(x, R, w, 1e-12, d)
+    xs = rng.standard_normal((7, d))
+    truth = xs + bt + xs @ Bt
+    assert np.abs(O.correct_rows(xs, f) - truth).max() < 1e-8
+
+
+def test_subspace_projector_properties():
+    x, R, w = _fit_inputs(seed=19, M=30, d=10)
+    f = O.fit_residual(x, R, w, 0.1, 4)
+    P = f.P
+    assert f.r_eff == 4
+    assert np.abs(P @ P - P).max() < 1e-13 and np.abs(P - P.T).max() < 1e-14
+    assert abs(np.trace(P) - 4) < 1e-12
+    # with r >= rank(Y), Y P = Y
+    full = O.fit_residual(x, R, w, 0.1, 10)
+    om = w * len(w) / w.sum()
+    Y = np.sqrt(om)[:, None] * (R - full.mu_R)
+    assert np.abs(Y @ full.P - Y).max() < 1e-12
+    # centring makes rank(Y) <= M - 1: a rank-deficient case keeps only real directions
+    x2, R2, w2 = _fit_inputs(seed=20, M=4, d=10)
+    f2 = O.fit_residual(x2, R2, w2, 0.1, 16)
+    assert f2.r_eff == 3
+
+
+# ---------------------------------------------------------------- whole call
+def _small_workload_params(**kw):
+    base = dict(d=8, M_s=32, r_K=4, r_Q=4, C_q=8, C_k=8, M=8, r=3, lam=0.1, rho=0.3,
+                kmeans_max_iter=25, seed=0)
+    base.update(kw)
+    return O.Params(**base)
+
+
+def _clustered(seed, N=240, d=8, C=8):
+    rng = _rng(seed)
+    mu = rng.standard_normal((C, d)) * 2
+    cid = rng.integers(0, C, N)
+    Q = mu[cid] + 0.4 * rng.standard_normal((N, d))
+    K = mu[cid] + 0.4 * rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    return Q, K, V
+
+
+def test_full_call_at_full_density_is_dense():
+    Q, K, V = _clustered(21)
+    res = O.sparsepr_call(Q, K, V, _small_workload_params(rho=1.0))
+    dense = O.dense_attention(Q, K, V)
+    assert res.rho_route == 1.0
+    assert np.abs(res.out - dense).max() < 1e-12
+    assert np.abs(res.fit.mu_R).max() < 1e-13
+
+
+def test_full_call_probe_rows_exact_and_density_identity():
+    Q, K, V = _clustered(22)
+    p = _small_workload_params()
+    res = O.sparsepr_call(Q, K, V, p)
+    dense = O.dense_attention(Q, K, V, res.probes)
+    assert np.array_equal(res.out[res.probes], res.dense_probe)
+    assert np.abs(res.dense_probe - dense).max() < 1e-14
+    N = Q.shape[0]
+    assert res.pairs_exec == res.pairs_route + p.M * N                  # integer identity
+    assert abs(res.rho_exec - (res.rho_route + p.M / N)) < 1e-15
+    assert res.rho_exec >= p.rho                                       # prefix reaches budget
+    assert sorted(res.probes.tolist()) == sorted(set(res.probes.tolist()))
+    assert res.m_a.sum() == p.M
+
+
+def test_full_call_correction_reduces_error():
+    # PFRR's purpose ([P] S4.2, Table 2): the fitted correction moves unprobed rows toward
+    # the dense output.  A flipped residual sign or a dropped mean term fails this.
+    for seed in (23, 24, 25):
+        Q, K, V = _clustered(seed, N=600)
+        p = _small_workload_params(rho=0.3, M=64, r=8, lam=0.1)
+        res = O.sparsepr_call(Q, K, V, p)
+        dense = O.dense_attention(Q, K, V)
+        unprobed = np.setdiff1d(np.arange(Q.shape[0]), res.probes)
+        err = lambda A: np.linalg.norm(A[unprobed] - dense[unprobed]) / np.linalg.norm(dense[unprobed])
+        assert err(res.out) < 0.9 * err(res.osp)
