@@ -1,0 +1,344 @@
+"""Benchmark of one SparsePR attention call (plan + attend + probe_fit + correct) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid|wan|hunyuan|tiny]
+                    [--impl ours|reference]
+
+A step is one whole call over all heads of the workload with inputs resident in HBM.
+The headline value is executed-pair TFLOP/s of the call, 4 d (routed + probe pairs) /
+call time (paper S2/S4.3 count executed pairs; probes included), with ms per call, the
+stage breakdown, and this library's own dense attention on the same inputs beside it.
+Multi-GPU: one process per GPU, every rank runs the workload on its own heads (weak
+scaling, no collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def launches_per_call(w, iters_k_run, iters_q_run) -> int:
+    """Kernel launches of one call, in the order the library enqueues them.
+
+    plan:   key metric 1, eigen 1, key projection 1, k-means keys (init 1 + max_iter x
+            (assign 1 + update 4)), finalize 4 + groups 1, centroids 1, query metric 1,
+            eigen 1, query projection 1, k-means queries (same), finalize 5, centroids 1,
+            route 2, gather 3, probes 3.   attend: 1.  probe_fit: 2 + fit 1.  correct: 2.
+    Every k-means iteration is launched (converged heads return at once).
+    """
+    km = 1 + w.kmeans_max_iter * 5
+    plan = 3 + km + 5 + 1 + 3 + km + 5 + 1 + 2 + 3 + 3
+    return plan + 1 + 3 + 2
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while a region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(w, head=0):
+    """Time the fp64 CPU oracle on one head of the workload (a bounded sample)."""
+    import numpy as np
+    from free_block_sparse_plan_b200 import workloads as W
+    from oracle import sparsepr_oracle as O
+    q, k, v = W.make_head(w, head)
+    p = O.Params.from_dict(w.params())
+    t0 = time.perf_counter()
+    res = O.sparsepr_call(q, k, v, p, head=head)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.d * res.pairs_exec
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"head {head} of {w.H}: full fp64 call (partition, routing, all {w.N} rows "
+                      f"of sparse attention, probes, fit, correction) in {dt:.2f} s; "
+                      f"value = executed-pair FLOPs of that head / time",
+            "seconds_per_head": dt}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times, flops = [], []
+    from free_block_sparse_plan_b200 import workloads as W
+    from oracle import sparsepr_oracle as O
+    p = O.Params.from_dict(w.params())
+    for i in range(args.warmup + args.steps):
+        h = i % w.H
+        q, k, v = W.make_head(w, h)
+        t0 = time.perf_counter()
+        res = O.sparsepr_call(q, k, v, p, head=h)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(4.0 * w.d * res.pairs_exec)
+    value = sum(flops) / sum(times) / 1e12
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample": "one head per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one head of {w.H} per step (heads 0..), full fp64 call"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = ("executed-pair TFLOP/s of one SparsePR attention call (plan+attend+probe_fit+correct) "
+          "at rho_exec~22%; ms/call, % of BF16 peak and speedup over dense alongside")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run this many calls and exit (for an external profiler; no timing)")
+    args = ap.parse_args()
+
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.get(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from free_block_sparse_plan_b200 import native as N
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    # every rank takes its own heads: head index offset rank * H (weak scaling)
+    wr = w.with_(seed=w.seed + rank) if world > 1 else w
+    Q, K, V = W.make_inputs_torch(wr, device=dev)
+    params = N.params_from_dict(wr.params())
+    ws = torch.empty(N.sparsepr_workspace_size(params), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(Q)
+    dense_out = torch.empty_like(Q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(ev=None):
+        plan = N.Plan(params, Q, K, V, workspace=ws)
+        if ev: ev[1].record()
+        plan.attend()
+        if ev: ev[2].record()
+        plan.probe_fit()
+        if ev: ev[3].record()
+        plan.correct(out)
+        return plan
+
+    if args.profile_steps:
+        for _ in range(args.profile_steps):
+            call()
+        torch.cuda.synchronize()
+        return
+
+    for _ in range(args.warmup):
+        call()
+        N.dense_attention(Q, K, V, out=dense_out)
+    torch.cuda.synchronize()
+    plan = call()
+    st = plan.stats()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stage = np.zeros((args.steps, 4))
+    with Clocks(local) as clk:
+        barrier()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)                      # evict L2 between timed calls
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            ev[0].record()
+            call(ev)
+            ev[4].record()
+            ev[4].synchronize()
+            stage[i] = [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
+                        ev[2].elapsed_time(ev[3]), ev[3].elapsed_time(ev[4])]
+        barrier()
+        dense_ms = []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            N.dense_attention(Q, K, V, out=dense_out)
+            e1.record()
+            e1.synchronize()
+            dense_ms.append(e0.elapsed_time(e1))
+        barrier()
+    call_ms = stage.sum(axis=1)
+    ms = float(np.median(call_ms))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        tot = torch.tensor([float(st["pairs_exec"])], device=dev, dtype=torch.float64)
+        dist.all_reduce(tot)
+        pairs_exec_all = float(tot.item())
+    else:
+        pairs_exec_all = float(st["pairs_exec"])
+    flops_all = 4.0 * w.d * pairs_exec_all
+    value = flops_all / (ms * 1e-3) / 1e12
+    attend_ms = float(np.median(stage[:, 1]))
+    attend_tflops = 4.0 * w.d * st["pairs_route"] / (attend_ms * 1e-3) / 1e12
+    dense_med = float(np.median(dense_ms))
+
+    # end to end through the public call with host buffers: H2D inputs, call, D2H output
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+        e2e_ms = []
+        for i in range(args.warmup + args.steps):
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            dQ.copy_(hQ, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            N.forward(params, dQ, dK, dV, out=out, workspace=ws)
+            hOut.copy_(out, non_blocking=True)
+            e1.record()
+            e1.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(e0.elapsed_time(e1))
+        em = float(np.median(e2e_ms))
+        if world > 1:
+            t = torch.tensor([em], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            em = float(t.item())
+        nbytes_in = sum(t.numel() * t.element_size() for t in (hQ, hK, hV))
+        e2e = {"value": flops_all / (em * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": em, "h2d_bytes_per_step": nbytes_in,
+               "d2h_bytes_per_step": hOut.numel() * hOut.element_size()}
+
+    peaks, peak_kind = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "C_q": w.C_q, "C_k": w.C_k,
+                   "M": w.M, "r": w.r, "target_density": w.rho, "heads_per_gpu": w.H,
+                   "l2": "flushed between timed calls (256 MiB write)"},
+        "ms_per_call": ms,
+        "stages_ms": {"plan": float(np.median(stage[:, 0])), "attend": attend_ms,
+                      "probe_fit": float(np.median(stage[:, 2])),
+                      "correct": float(np.median(stage[:, 3]))},
+        "dense_ms": dense_med, "speedup_vs_dense": dense_med / ms,
+        "rho_route": st["rho_route"], "rho_exec": st["rho_exec"],
+        "kmeans_iters": [st["kmeans_iters_k_max"], st["kmeans_iters_q_max"]],
+        "roofline": {"kernel": "sparse attention (attend)", "bound": "tensor",
+                     "achieved": attend_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attend_tflops / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained"},
+        "pct_bf16_peak_call": value / peak,
+        "gpu_launches": launches_per_call(w, 0, 0) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_oracle_sample(w, 0)
+        cb.pop("seconds_per_head")
+        line["cpu_baseline"] = cb
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

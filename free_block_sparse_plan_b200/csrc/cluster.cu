@@ -1,0 +1,498 @@
+// Response-Coupled Partitioning on the GPU (paper S4.1, App. B.1-B.2, App. C):
+// key / query response coordinates, batched Lloyd k-means, and the groups it yields.
+//
+// k-means is batched over heads; every head stops on its own as soon as an assignment
+// step changes no label (or after kmeans_max_iter steps), tracked by device flags so
+// the host never synchronises.  Centre updates are deterministic: the labels are
+// stably counting-sorted (this order is also the group-major order the attention
+// uses) and each cluster's members are summed in that fixed order in fp64.
+#include "common.cuh"
+
+namespace spr {
+namespace {
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): output n of the generator whose state
+// starts at `key` is mix(key + n * gamma).
+__device__ __forceinline__ unsigned long long sm64_mix(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+constexpr unsigned long long kGamma = 0x9E3779B97F4A7C15ULL;
+
+struct KmView {         // one k-means instance (keys or queries) for all heads
+  const float* X;       // [H][N][r] features
+  float* cent;          // [H][C][r]
+  int* lab;             // [H][N]
+  int* hist;            // [H][C][nch]
+  int* perm;            // [H][N]
+  int* off;             // [H][C+1]
+  int* km;              // [H][4]: done, changed[0], changed[1], iterations
+  double* obj;          // [H][C]
+  int N, C, r, nch, stage;
+};
+
+KmView view(const Plan& p, bool query) {
+  const Buffers& b = p.b;
+  const Dims& m = p.dm;
+  if (query) return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, m.Nq, m.Cq, m.rQ, m.nchQ, 1};
+  return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, m.Nk, m.Ck, m.rK, m.nchK, 0};
+}
+
+// ---------------------------------------------------------------------------------
+// Response coordinates: phi = X F (keys), phi = RMSnorm(X F) (queries, floor 1e-6).
+template <int R, bool RMS>
+__global__ void __launch_bounds__(128) project_kernel(Dims m, const void* X, int N,
+                                                     const float* Fall, int r, float* out) {
+  extern __shared__ float sm[];
+  const int d = m.d, h = blockIdx.y;
+  float* F = sm;                       // [d][R] zero padded
+  float* T = sm + d * R;               // [128][d+1]
+  const float* Fh = Fall + (long long)h * d * r;
+  for (int e = threadIdx.x; e < d * R; e += blockDim.x) {
+    const int j = e / R, k = e % R;
+    F[e] = k < r ? Fh[j * r + k] : 0.0f;
+  }
+  const long long row0 = (long long)blockIdx.x * 128;
+  const long long base = ((long long)h * N) * d;
+  for (int e = threadIdx.x; e < 128 * d; e += blockDim.x) {
+    const int i = e / d, j = e % d;
+    const long long row = row0 + i;
+    T[i * (d + 1) + j] = row < N ? load_as_float(X, base + row * d + j, m.dtype) : 0.0f;
+  }
+  __syncthreads();
+  const long long row = row0 + threadIdx.x;
+  if (row >= N) return;
+  float acc[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) acc[k] = 0.0f;
+  const float* x = T + threadIdx.x * (d + 1);
+  for (int j = 0; j < d; ++j) {
+    const float xv = x[j];
+#pragma unroll
+    for (int k = 0; k < R; ++k) acc[k] = fmaf(xv, F[j * R + k], acc[k]);
+  }
+  float scale = 1.0f;
+  if (RMS) {
+    float ss = 0.0f;
+#pragma unroll
+    for (int k = 0; k < R; ++k) ss = fmaf(acc[k], acc[k], ss);
+    const float rms = sqrtf(ss / (float)r);
+    scale = 1.0f / fmaxf(rms, 1e-6f);
+  }
+  float* o = out + ((long long)h * N + row) * r;
+#pragma unroll
+  for (int k = 0; k < R; ++k)
+    if (k < r) o[k] = RMS ? acc[k] * scale : acc[k];
+}
+
+template <bool RMS>
+sparsepr_status launch_project(const Plan& p, const void* X, int N, const float* F, int r,
+                               float* out, cudaStream_t st) {
+  const int d = p.dm.d;
+  dim3 grid(cdiv(N, 128), p.dm.H);
+  auto run = [&](auto kern, int R) -> sparsepr_status {
+    const size_t smem = (size_t)(d * R + 128 * (d + 1)) * sizeof(float);
+    SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    kern<<<grid, 128, smem, st>>>(p.dm, X, N, F, r, out);
+    SPR_LAUNCH_OK();
+    return SPARSEPR_OK;
+  };
+  if (r <= 8) return run(project_kernel<8, RMS>, 8);
+  if (r <= 16) return run(project_kernel<16, RMS>, 16);
+  if (r <= 32) return run(project_kernel<32, RMS>, 32);
+  if (r <= 48) return run(project_kernel<48, RMS>, 48);
+  return run(project_kernel<64, RMS>, 64);
+}
+
+// ---------------------------------------------------------------------------------
+// k-means initialisation: C rows drawn with replacement (paper App. C), SplitMix64
+// stream (2h + stage + 1) of `seed`, index = (hi32 * N) >> 32.
+__global__ void km_init_kernel(KmView v, unsigned long long seed) {
+  const int h = blockIdx.x;
+  const unsigned long long key = sm64_mix(seed + (unsigned long long)(2 * h + v.stage + 1) * kGamma);
+  for (int e = threadIdx.x; e < v.C * v.r; e += blockDim.x) {
+    const int c = e / v.r, k = e % v.r;
+    const unsigned long long z = sm64_mix(key + (unsigned long long)(c + 1) * kGamma);
+    const long long idx = (long long)(((z >> 32) * (unsigned long long)v.N) >> 32);
+    v.cent[((long long)h * v.C + c) * v.r + k] = v.X[((long long)h * v.N + idx) * v.r + k];
+  }
+}
+
+// Assignment: label = argmin_c ||x - c||^2 (direct sum of squared differences in fp32,
+// dimensions in ascending order; ties to the lowest index).
+template <int R>
+__global__ void __launch_bounds__(128) km_assign_kernel(KmView v, int it) {
+  constexpr int TILE = 64;
+  __shared__ float cs[TILE * R];
+  const int h = blockIdx.y;
+  int* km = v.km + 4 * h;
+  if (km[0]) return;
+  const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool valid = row < v.N;
+  float x[R];
+  const float* xp = v.X + ((long long)h * v.N + (valid ? row : 0)) * v.r;
+#pragma unroll
+  for (int k = 0; k < R; ++k) x[k] = (k < v.r) ? xp[k] : 0.0f;
+  float best = 3.402823466e38f;
+  int bi = 0;
+  const float* ch = v.cent + (long long)h * v.C * v.r;
+  for (int c0 = 0; c0 < v.C; c0 += TILE) {
+    const int nc = (v.C - c0) < TILE ? (v.C - c0) : TILE;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nc * R; e += blockDim.x) {
+      const int c = e / R, k = e % R;
+      cs[e] = k < v.r ? ch[(long long)(c0 + c) * v.r + k] : 0.0f;
+    }
+    __syncthreads();
+    for (int c = 0; c < nc; ++c) {
+      float dsum = 0.0f;
+#pragma unroll
+      for (int k = 0; k < R; ++k) {
+        const float t = x[k] - cs[c * R + k];
+        dsum = fmaf(t, t, dsum);
+      }
+      if (dsum < best) {
+        best = dsum;
+        bi = c0 + c;
+      }
+    }
+  }
+  if (valid) {
+    int* lp = v.lab + (long long)h * v.N + row;
+    if (*lp != bi) {
+      *lp = bi;
+      km[1 + (it & 1)] = 1;
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) km[3] += 1;
+}
+
+// Should the update of iteration `it` run?  force: always (final pass / given labels).
+__device__ __forceinline__ bool km_skip(const KmView& v, int h, int it, bool force) {
+  if (force) return false;
+  const int* km = v.km + 4 * h;
+  return km[0] || !km[1 + (it & 1)];
+}
+
+// Stable counting sort, pass 1: per-chunk label histograms hist[h][c][chunk].
+__global__ void __launch_bounds__(kSortChunk) cs_hist_kernel(KmView v, int it, bool force) {
+  __shared__ int hist[kMaxC];
+  const int h = blockIdx.y, ch = blockIdx.x;
+  if (km_skip(v, h, it, force)) return;
+  for (int c = threadIdx.x; c < v.C; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  const long long row = (long long)ch * kSortChunk + threadIdx.x;
+  if (row < v.N) atomicAdd(&hist[v.lab[(long long)h * v.N + row]], 1);
+  __syncthreads();
+  int* g = v.hist + (long long)h * v.C * v.nch;
+  for (int c = threadIdx.x; c < v.C; c += blockDim.x) g[(long long)c * v.nch + ch] = hist[c];
+}
+
+// Pass 2: exclusive scan of hist in (label, chunk) order; off[c] = start of label c.
+__global__ void __launch_bounds__(1024) cs_scan_kernel(KmView v, int it, bool force) {
+  __shared__ int sh[32];
+  const int h = blockIdx.x;
+  if (km_skip(v, h, it, force)) return;
+  int* g = v.hist + (long long)h * v.C * v.nch;
+  const long long len = (long long)v.C * v.nch;
+  const long long per = (len + blockDim.x - 1) / blockDim.x;
+  const long long s0 = threadIdx.x * per, s1 = (s0 + per < len) ? s0 + per : len;
+  int local = 0;
+  for (long long e = s0; e < s1; ++e) local += g[e];
+  int total;
+  int run = block_exclusive_scan(local, sh, &total);
+  for (long long e = s0; e < s1; ++e) {
+    const int c = g[e];
+    g[e] = run;
+    run += c;
+  }
+  __syncthreads();
+  int* off = v.off + (long long)h * (v.C + 1);
+  for (int c = threadIdx.x; c < v.C; c += blockDim.x) off[c] = g[(long long)c * v.nch];
+  if (threadIdx.x == 0) off[v.C] = v.N;
+}
+
+// Pass 3: stable scatter; rank inside the chunk among equal labels at lower rows.
+__global__ void __launch_bounds__(kSortChunk) cs_scatter_kernel(KmView v, int it, bool force) {
+  constexpr int W = kSortChunk / 32;
+  __shared__ int wc[W][kMaxC];
+  const int h = blockIdx.y, ch = blockIdx.x;
+  if (km_skip(v, h, it, force)) return;
+  for (int e = threadIdx.x; e < W * v.C; e += blockDim.x) wc[e / v.C][e % v.C] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long row = (long long)ch * kSortChunk + threadIdx.x;
+  const int lab = row < v.N ? v.lab[(long long)h * v.N + row] : -1;
+  const unsigned peers = __match_any_sync(0xffffffffu, lab);
+  const int lower = __popc(peers & ((1u << lane) - 1u));
+  if (lab >= 0 && lower == 0) wc[w][lab] = __popc(peers);
+  __syncthreads();
+  if (lab < 0) return;
+  int before = 0;
+  for (int k = 0; k < w; ++k) before += wc[k][lab];
+  const int* g = v.hist + (long long)h * v.C * v.nch;
+  const int pos = g[(long long)lab * v.nch + ch] + before + lower;
+  v.perm[(long long)h * v.N + pos] = (int)row;
+}
+
+// Pass 4: centre = mean of members (fp64 sums in group-major order); empty clusters keep
+// their centre.  Also the cluster's share of the objective at its new centre.
+constexpr int kMeanSub = 4;
+__global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int it, bool force) {
+  __shared__ double part[kMeanSub][kMaxR];
+  __shared__ double opart[kMeanSub * kMaxR / 32];
+  const int h = blockIdx.y, c = blockIdx.x;
+  int* km = v.km + 4 * h;
+  if (!force) {
+    if (km[0]) return;
+    if (!km[1 + (it & 1)]) {            // converged: this assignment changed nothing
+      if (c == 0 && threadIdx.x == 0) km[0] = 1;
+      return;
+    }
+    if (c == 0 && threadIdx.x == 0) km[1 + ((it + 1) & 1)] = 0;  // reset next slot
+  }
+  const int k = threadIdx.x % kMaxR, sub = threadIdx.x / kMaxR;
+  const int* off = v.off + (long long)h * (v.C + 1);
+  const int m0 = off[c], m1 = off[c + 1];
+  const int* perm = v.perm + (long long)h * v.N;
+  const float* X = v.X + (long long)h * v.N * v.r;
+  double acc = 0.0;
+  if (k < v.r)
+    for (int mm = m0 + sub; mm < m1; mm += kMeanSub) acc += (double)X[(long long)perm[mm] * v.r + k];
+  part[sub][k] = acc;
+  __syncthreads();
+  const int cnt = m1 - m0;
+  float* cent = v.cent + ((long long)h * v.C + c) * v.r;
+  double mean = 0.0;
+  if (k < v.r) {
+    double s = 0.0;
+    for (int q = 0; q < kMeanSub; ++q) s += part[q][k];
+    mean = cnt > 0 ? s / (double)cnt : (double)cent[k];
+  }
+  __syncthreads();
+  if (cnt > 0 && sub == 0 && k < v.r) cent[k] = (float)mean;
+  // objective share: sum over members of ||x - centre||^2
+  double o = 0.0;
+  if (k < v.r)
+    for (int mm = m0 + sub; mm < m1; mm += kMeanSub) {
+      const double t = (double)X[(long long)perm[mm] * v.r + k] - mean;
+      o += t * t;
+    }
+  o = warp_sum(o);
+  if ((threadIdx.x & 31) == 0) opart[threadIdx.x >> 5] = o;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int q = 0; q < kMeanSub * kMaxR / 32; ++q) s += opart[q];
+    v.obj[(long long)h * v.C + c] = s;
+  }
+}
+
+sparsepr_status run_update(const Plan& p, const KmView& v, int it, bool force, cudaStream_t st) {
+  const int H = p.dm.H;
+  cs_hist_kernel<<<dim3(v.nch, H), kSortChunk, 0, st>>>(v, it, force);
+  cs_scan_kernel<<<H, 1024, 0, st>>>(v, it, force);
+  cs_scatter_kernel<<<dim3(v.nch, H), kSortChunk, 0, st>>>(v, it, force);
+  cs_mean_kernel<<<dim3(v.C, H), kMeanSub * kMaxR, 0, st>>>(v, it, force);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+template <int R>
+void assign(const KmView& v, int H, int it, cudaStream_t st) {
+  km_assign_kernel<R><<<dim3(cdiv(v.N, 128), H), 128, 0, st>>>(v, it);
+}
+
+// ---------------------------------------------------------------------------------
+// Groups of the final labels: compact ids in ascending label order, sizes, counts and
+// the final objective (sum of per-cluster shares in label order).
+__global__ void __launch_bounds__(1024) groups_kernel(KmView v, int* comp, int* used, int* size,
+                                                      int* ngroups, double* objH) {
+  __shared__ int sh[32];
+  __shared__ double red[32];
+  const int h = blockIdx.x;
+  const int* off = v.off + (long long)h * (v.C + 1);
+  int* comph = comp + (long long)h * v.C;
+  int* usedh = used + (long long)h * v.C;
+  int* sizeh = size + (long long)h * v.C;
+  const int c = threadIdx.x;
+  const int cnt = c < v.C ? off[c + 1] - off[c] : 0;
+  int total;
+  const int idx = block_exclusive_scan(cnt > 0 ? 1 : 0, sh, &total);
+  if (c < v.C) {
+    comph[c] = cnt > 0 ? idx : -1;
+    if (cnt > 0) {
+      usedh[idx] = c;
+      sizeh[idx] = cnt;
+    }
+  }
+  __syncthreads();
+  for (int e = total + threadIdx.x; e < v.C; e += blockDim.x) {
+    usedh[e] = -1;
+    sizeh[e] = 0;
+  }
+  if (threadIdx.x == 0) ngroups[h] = total;
+  // objective in label order (one thread: C <= 1024 terms, deterministic)
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int q = 0; q < v.C; ++q) s += v.obj[(long long)h * v.C + q];
+    objH[2 * h + v.stage] = s;
+  }
+  (void)red;
+}
+
+// Group centroids in the original space (compact ids), fp64 sums in group-major order.
+constexpr int kCentSub = 4;
+__global__ void __launch_bounds__(kCentSub * kMaxD) centroid_kernel(Dims m, const void* X,
+                                                                   const void* X2, int N, int C,
+                                                                   const int* perm, const int* off,
+                                                                   const int* used, const int* ngroups,
+                                                                   double* out, double* out2) {
+  __shared__ double part[kCentSub][kMaxD];
+  __shared__ double part2[kCentSub][kMaxD];
+  const int h = blockIdx.y, a = blockIdx.x, d = m.d;
+  if (a >= ngroups[h]) return;
+  const int lab = used[(long long)h * C + a];
+  const int m0 = off[(long long)h * (C + 1) + lab], m1 = off[(long long)h * (C + 1) + lab + 1];
+  const int j = threadIdx.x % kMaxD, sub = threadIdx.x / kMaxD;
+  const int* ph = perm + (long long)h * N;
+  const long long base = (long long)h * N * d;
+  double acc = 0.0, acc2 = 0.0;
+  if (j < d) {
+    for (int mm = m0 + sub; mm < m1; mm += kCentSub) {
+      const long long src = base + (long long)ph[mm] * d + j;
+      acc += (double)load_as_float(X, src, m.dtype);
+      if (X2) acc2 += (double)load_as_float(X2, src, m.dtype);
+    }
+  }
+  part[sub][j] = acc;
+  part2[sub][j] = acc2;
+  __syncthreads();
+  if (sub == 0 && j < d) {
+    double s = 0.0, s2 = 0.0;
+    for (int q = 0; q < kCentSub; ++q) {
+      s += part[q][j];
+      s2 += part2[q][j];
+    }
+    const double cnt = (double)(m1 - m0);
+    out[((long long)h * C + a) * d + j] = s / cnt;
+    if (X2) out2[((long long)h * C + a) * d + j] = s2 / cnt;
+  }
+}
+
+// M_Q = (1/C_k') K~^T K~ with K~ = kbar - mean of the non-empty kbar (paper App. B.2).
+__global__ void __launch_bounds__(1024) query_metric_kernel(Dims m, const double* kbar,
+                                                            const int* ngroups, double* MQ) {
+  constexpr int ROWS = 16;
+  __shared__ double mu[kMaxD];
+  __shared__ double tile[ROWS * kMaxD];
+  const int h = blockIdx.x, d = m.d, n = ngroups[h];
+  const double* kb = kbar + (long long)h * m.Ck * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double s = 0.0;
+    for (int b = 0; b < n; ++b) s += kb[(long long)b * d + j];
+    mu[j] = s / (double)n;
+  }
+  double acc[16];
+  for (int k = 0; k < 16; ++k) acc[k] = 0.0;
+  for (int b0 = 0; b0 < n; b0 += ROWS) {
+    const int nb = (n - b0) < ROWS ? (n - b0) : ROWS;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nb * d; e += blockDim.x)
+      tile[e] = kb[(long long)b0 * d + e] - mu[e % d];
+    __syncthreads();
+    for (int k = 0; k < 16; ++k) {
+      const int e = threadIdx.x + k * blockDim.x;
+      if (e >= d * d) break;
+      const int i = e / d, j = e % d;
+      double a = acc[k];
+      for (int b = 0; b < nb; ++b) a += tile[b * d + i] * tile[b * d + j];
+      acc[k] = a;
+    }
+  }
+  for (int k = 0; k < 16; ++k) {
+    const int e = threadIdx.x + k * blockDim.x;
+    if (e >= d * d) break;
+    MQ[(long long)h * d * d + e] = acc[k] / (double)n;
+  }
+}
+
+// Injected labels outside [0, C) are clamped to 0 and flagged.
+__global__ void check_labels_kernel(int* lab, long long n, int C, int* err) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int v = lab[i];
+    if (v < 0 || v >= C) {
+      lab[i] = 0;
+      atomicOr(err, kErrLabels);
+    }
+  }
+}
+
+}  // namespace
+
+sparsepr_status launch_check_labels(const Plan& p, bool query, cudaStream_t st) {
+  const KmView v = view(p, query);
+  check_labels_kernel<<<148 * 4, 256, 0, st>>>(v.lab, (long long)p.dm.H * v.N, v.C, p.b.err);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st) {
+  return launch_project<false>(p, p.K, p.dm.Nk, p.b.FK, p.dm.rK, p.b.phiK, st);
+}
+
+sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st) {
+  return launch_project<true>(p, p.Q, p.dm.Nq, p.b.FQ, p.dm.rQ, p.b.phiQ, st);
+}
+
+sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
+  const KmView v = view(p, query);
+  const int H = p.dm.H;
+  SPR_CUDA_OK(cudaMemsetAsync(v.km, 0, sizeof(int) * 4 * H, st));
+  SPR_CUDA_OK(cudaMemsetAsync(v.lab, 0xFF, sizeof(int) * (size_t)H * v.N, st));  // labels = -1
+  km_init_kernel<<<H, 256, 0, st>>>(v, p.dm.seed);
+  SPR_LAUNCH_OK();
+  for (int it = 0; it < p.dm.max_iter; ++it) {
+    if (v.r <= 8) assign<8>(v, H, it, st);
+    else if (v.r <= 16) assign<16>(v, H, it, st);
+    else if (v.r <= 32) assign<32>(v, H, it, st);
+    else if (v.r <= 48) assign<48>(v, H, it, st);
+    else assign<64>(v, H, it, st);
+    SPR_LAUNCH_OK();
+    sparsepr_status s = run_update(p, v, it, false, st);
+    if (s != SPARSEPR_OK) return s;
+  }
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_finalize_groups(const Plan& p, bool query, cudaStream_t st) {
+  const KmView v = view(p, query);
+  sparsepr_status s = run_update(p, v, 0, true, st);
+  if (s != SPARSEPR_OK) return s;
+  const Buffers& b = p.b;
+  if (query) groups_kernel<<<p.dm.H, 1024, 0, st>>>(v, b.compQ, b.usedQ, b.sizeQ, b.nQ, b.objH);
+  else groups_kernel<<<p.dm.H, 1024, 0, st>>>(v, b.compK, b.usedK, b.sizeK, b.nK, b.objH);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_centroids(const Plan& p, bool query, cudaStream_t st) {
+  const Buffers& b = p.b;
+  const Dims& m = p.dm;
+  if (query)
+    centroid_kernel<<<dim3(m.Cq, m.H), kCentSub * kMaxD, 0, st>>>(m, p.Q, nullptr, m.Nq, m.Cq, b.permQ, b.offQ, b.usedQ, b.nQ, b.qbar, nullptr);
+  else
+    centroid_kernel<<<dim3(m.Ck, m.H), kCentSub * kMaxD, 0, st>>>(m, p.K, p.V, m.Nk, m.Ck, b.permK, b.offK, b.usedK, b.nK, b.kbar, b.vbar);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_query_metric(const Plan& p, cudaStream_t st) {
+  query_metric_kernel<<<p.dm.H, 1024, 0, st>>>(p.dm, p.b.kbar, p.b.nK, p.b.MQ);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+}  // namespace spr

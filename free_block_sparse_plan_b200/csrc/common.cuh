@@ -1,0 +1,200 @@
+// Shared definitions of the SparsePR CUDA library: problem description, workspace
+// pointers, launch helpers and small device utilities.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sparsepr.h"
+
+namespace spr {
+
+constexpr int kMaxD = 128;      // head dimension limit
+constexpr int kMaxC = 1024;     // requested group count limit
+constexpr int kMaxR = 64;       // response-coordinate rank limit
+constexpr int kMaxM = 128;      // probe count limit
+constexpr int kSortChunk = 256; // rows per block of the stable counting sort
+constexpr int kProbeSplit = 4096;  // keys per partial of the exact probe attention
+
+// Device error word bits.
+enum : int {
+  kErrEigK = 1,        // key metric has no positive eigenvalue among the leading r_K
+  kErrEigQ = 2,        // query metric has no positive eigenvalue among the leading r_Q
+  kErrNonFinite = 4,   // a non-finite value reached the fit
+  kErrProbe = 8,       // probe selection could not find M rows
+  kErrLabels = 16,     // an injected label was outside [0, C)
+};
+
+// Problem dimensions, passed by value to kernels.
+struct Dims {
+  int H, Nq, Nk, d, dtype;
+  int Ms, rK, rQ, Cq, Ck, M, r;
+  double lambda, rho;
+  int max_iter, engine;
+  unsigned long long seed;
+  int nchK, nchQ;      // counting-sort chunks per head
+  int nsplit;          // partial blocks of the exact probe attention
+  double beta;         // per-query key budget (rho - M/N_q) * N_k
+};
+
+// Device buffers carved from the caller's workspace (see carve_workspace).
+struct Buffers {
+  double *MK, *MQ, *lamK, *lamQ, *FK64, *FQ64;
+  float *FK, *FQ;
+  float *phiK, *phiQ;
+  float *centK, *centQ;
+  int *labK, *labQ;
+  int *histK, *histQ;
+  int *permK, *permQ, *invQ;
+  int *offK, *offQ;          // raw-label offsets [H][C+1]
+  int *kmK, *kmQ;            // per-head k-means state [H][4]: done, changed, iters, -
+  double *objK, *objQ;       // per-cluster objective partials [H][C]
+  double *objH;              // [H][2] final objectives
+  int *compK, *compQ;        // raw label -> compact id (-1 if empty) [H][C]
+  int *usedK, *usedQ;        // compact id -> raw label [H][C]
+  int *nK, *nQ;              // [H] non-empty group counts
+  int *sizeK, *sizeQ;        // compact sizes [H][C]
+  double *kbar, *vbar, *qbar;  // compact centroids [H][C][d]
+  double *scores;            // [H][Cq][Ck]
+  int *cellCnt, *cellIds;    // [H][Cq], [H][Cq][Ck]
+  long long *pairs;          // [H]
+  void *Qp, *Kp, *Vp;        // group-major copies [H][N][d]
+  float *dist;               // [H][Nq]
+  int *probeTop;             // [H][Cq][M]
+  int *probes, *probeA, *mA; // [H][M], [H][M], [H][Cq]
+  double *wP;                // [H][M]
+  float *Osp;                // [H][Nq][d] group-major
+  float *Opart, *MLpart;     // [H][M][nsplit][d], [H][M][nsplit][2]
+  float *Odense;             // [H][M][d]
+  double *fitA, *fitY, *fitZ;  // fit scratch
+  double *muX, *muR, *sX;    // [H][d]
+  double *Bm, *Pm;           // [H][d][d]
+  double *sig;               // [H][kMaxM]
+  int *reff;                 // [H]
+  float *Bp, *cvec;          // folded correction [H][d][d], [H][d]
+  int *err;                  // device error word
+};
+
+// Host-side plan handle.
+struct Plan {
+  Dims dm;
+  Buffers b;
+  const void *Q, *K, *V;
+  int stage;                 // 1 planned, 2 attended, 3 fitted
+};
+
+// ---------------------------------------------------------------------------------
+// Launch helpers (host)
+#define SPR_CUDA_OK(expr)                                  \
+  do {                                                     \
+    cudaError_t e_ = (expr);                               \
+    if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA;       \
+  } while (0)
+
+#define SPR_LAUNCH_OK()                                    \
+  do {                                                     \
+    cudaError_t e_ = cudaGetLastError();                   \
+    if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA;       \
+  } while (0)
+
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// ---------------------------------------------------------------------------------
+// Device utilities
+__device__ __forceinline__ float load_as_float(const void* p, long long i, int dtype) {
+  if (dtype == SPARSEPR_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+
+__device__ __forceinline__ void store_from_float(void* p, long long i, float v, int dtype) {
+  if (dtype == SPARSEPR_BF16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(p)[i] = v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum of doubles; `red` holds blockDim.x/32 doubles. All threads get the sum.
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int i = 0; i < nw; ++i) t += red[i];   // fixed order: deterministic
+  return t;
+}
+
+__device__ __forceinline__ long long block_sum_ll(long long v, long long* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  long long t = 0;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
+
+// Exclusive block scan of ints (blockDim.x <= 1024); `sh` holds 32 ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int x = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) sh[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = (lane < nw) ? sh[lane] : 0;
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < nw) sh[lane] = s;   // inclusive per-warp totals
+  }
+  __syncthreads();
+  int base = (w > 0) ? sh[w - 1] : 0;
+  if (total) *total = sh[nw - 1];
+  return base + x - v;
+}
+
+// ---------------------------------------------------------------------------------
+// Stage launchers (defined in the .cu files; all enqueue on `st`, return a status).
+sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st);
+sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st);
+sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st);
+sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_finalize_groups(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_check_labels(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_centroids(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_query_metric(const Plan& p, cudaStream_t st);
+sparsepr_status launch_route(const Plan& p, cudaStream_t st);
+sparsepr_status launch_permute(const Plan& p, cudaStream_t st);
+sparsepr_status launch_select_probes(const Plan& p, cudaStream_t st);
+sparsepr_status launch_sparse_attention(const Plan& p, cudaStream_t st);
+sparsepr_status launch_probe_attention(const Plan& p, cudaStream_t st);
+sparsepr_status launch_fit(const Plan& p, cudaStream_t st);
+sparsepr_status launch_correct(const Plan& p, void* Out, cudaStream_t st);
+sparsepr_status launch_sparse_attention_simt(const Plan& p, cudaStream_t st);
+sparsepr_status launch_dense_attention_simt(const Dims& dm, const void* Q, const void* K,
+                                            const void* V, void* Out, cudaStream_t st);
+sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void* K,
+                                       const void* V, void* Out, cudaStream_t st);
+
+}  // namespace spr

@@ -1,0 +1,402 @@
+// Small dense linear algebra of SparsePR, one CTA per head, fp64:
+//   key response metric M_K (paper S4.1, App. B.1), the query metric M_Q of the centred
+//   K/V centroids (App. B.2), their eigenvalue-weighted factors F_K / F_Q, and the
+//   probe fit: coverage-weighted statistics, weighted ridge B_lambda and the residual
+//   subspace Psi_r (paper S4.2, App. A.3, App. D.2; review page step 4).
+//
+// Eigenvectors and singular vectors come from one-sided (Hestenes) Jacobi: rotating
+// column pairs of a matrix G until all columns are mutually orthogonal.  For a
+// symmetric PSD metric M, the converged columns of M V are lambda_j v_j, so their norms
+// are the eigenvalues and their directions the eigenvectors (no rotation accumulation
+// needed).  For the residual subspace, orthogonalising the columns of Y^T (one column
+// per probe) leaves columns sigma_k u_k with u_k the right singular vectors of Y.
+#include <cmath>
+
+#include "common.cuh"
+
+namespace spr {
+namespace {
+
+constexpr int kLinThreads = 1024;
+
+// ---------------------------------------------------------------------------------
+// M_K = (1/M_s') sum_s q_s^T q_s over rows floor(s*N_q/M_s) (all rows if M_s >= N_q).
+__global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const void* Q, double* MK) {
+  extern __shared__ float rows[];   // [64][d]
+  const int h = blockIdx.x, d = m.d;
+  const int Ms = m.Ms < m.Nq ? m.Ms : m.Nq;
+  const long long qbase = (long long)h * m.Nq * d;
+  double acc[16];
+  for (int k = 0; k < 16; ++k) acc[k] = 0.0;
+  const int entries = d * d;
+  for (int s0 = 0; s0 < Ms; s0 += 64) {
+    const int ns = (Ms - s0) < 64 ? (Ms - s0) : 64;
+    __syncthreads();
+    for (int e = threadIdx.x; e < ns * d; e += blockDim.x) {
+      const int s = s0 + e / d, j = e % d;
+      const long long row = (m.Ms >= m.Nq) ? s : ((long long)s * m.Nq) / m.Ms;
+      rows[e] = load_as_float(Q, qbase + row * d + j, m.dtype);
+    }
+    __syncthreads();
+    for (int k = 0; k < 16; ++k) {
+      const int e = threadIdx.x + k * blockDim.x;
+      if (e >= entries) break;
+      const int i = e / d, j = e % d;
+      double a = acc[k];
+      for (int s = 0; s < ns; ++s) a += (double)rows[s * d + i] * (double)rows[s * d + j];
+      acc[k] = a;
+    }
+  }
+  for (int k = 0; k < 16; ++k) {
+    const int e = threadIdx.x + k * blockDim.x;
+    if (e >= entries) break;
+    MK[(long long)h * entries + e] = acc[k] / (double)Ms;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// One-sided Jacobi: orthogonalise the `ncols` columns (length `rows`, column-major with
+// stride `rows`) of G in shared memory.  Parallel round-robin ordering: in each round
+// the column pairs are disjoint, one warp per pair.  Bounded sweeps.
+__device__ void hestenes(double* G, int rows, int ncols, int* flag) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int nn = ncols + (ncols & 1);   // pad to even with a phantom column
+  const int npairs = nn / 2;
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    if (threadIdx.x == 0) *flag = 0;
+    __syncthreads();
+    for (int round = 0; round < nn - 1; ++round) {
+      for (int k = warp; k < npairs; k += nwarps) {
+        // circle method: position 0 fixed, the others rotate by `round`
+        const int pa = k, pb = nn - 1 - k;
+        const int ia = pa == 0 ? 0 : 1 + (pa - 1 + round) % (nn - 1);
+        const int ib = pb == 0 ? 0 : 1 + (pb - 1 + round) % (nn - 1);
+        if (ia >= ncols || ib >= ncols) continue;
+        double* a = G + (long long)ia * rows;
+        double* b = G + (long long)ib * rows;
+        double al = 0.0, be = 0.0, ga = 0.0;
+        for (int i = lane; i < rows; i += 32) {
+          const double x = a[i], y = b[i];
+          al += x * x;
+          be += y * y;
+          ga += x * y;
+        }
+        al = warp_sum(al);
+        be = warp_sum(be);
+        ga = warp_sum(ga);
+        if (ga == 0.0 || fabs(ga) <= 1e-15 * sqrt(al * be)) continue;
+        const double zeta = (be - al) / (2.0 * ga);
+        const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
+        const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
+        for (int i = lane; i < rows; i += 32) {
+          const double x = a[i], y = b[i];
+          a[i] = c * x - s * y;
+          b[i] = s * x + c * y;
+        }
+        if (lane == 0) *flag = 1;
+      }
+      __syncthreads();
+    }
+    const int rotated = *flag;
+    __syncthreads();
+    if (!rotated) break;
+  }
+}
+
+// rank of column j when columns are ordered by decreasing key, ties by index
+__device__ __forceinline__ int desc_rank(const double* key, int n, int j) {
+  const double v = key[j];
+  int r = 0;
+  for (int k = 0; k < n; ++k) r += (key[k] > v) || (key[k] == v && k < j);
+  return r;
+}
+
+// Eigen-weighted factor of a symmetric PSD metric (paper S4.1, App. B.1):
+// F = [u_1 sqrt(l_1/mean) ... u_r sqrt(l_r/mean)], mean over the r kept eigenvalues
+// (negative eigenvalues clamped to zero).
+__global__ void __launch_bounds__(kLinThreads) eigen_factor_kernel(Dims m, const double* Mall,
+                                                                   int r, double* lam_out,
+                                                                   double* F64, float* F32,
+                                                                   int* err, int err_bit) {
+  extern __shared__ double G[];          // [d][d] column-major
+  __shared__ double norm[kMaxD], lam[kMaxD], red[32];
+  __shared__ int rank[kMaxD];
+  __shared__ int flag;
+  const int h = blockIdx.x, d = m.d;
+  const double* Mh = Mall + (long long)h * d * d;
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) G[e] = Mh[e];  // symmetric
+  __syncthreads();
+  hestenes(G, d, d, &flag);
+  // column norms = |eigenvalues|; the sign comes from the Rayleigh quotient
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int j = warp; j < d; j += nwarps) {
+    double s = 0.0;
+    for (int i = lane; i < d; i += 32) s += G[j * d + i] * G[j * d + i];
+    s = warp_sum(s);
+    if (lane == 0) norm[j] = sqrt(s);
+  }
+  __syncthreads();
+  for (int j = warp; j < d; j += nwarps) {
+    const double nj = norm[j];
+    double rq = 0.0;   // u^T M u * |lambda|^2 (sign only)
+    if (nj > 0.0) {
+      for (int i = lane; i < d; i += 32) {
+        double mu = 0.0;
+        for (int k = 0; k < d; ++k) mu += Mh[i * d + k] * G[j * d + k];
+        rq += G[j * d + i] * mu;
+      }
+      rq = warp_sum(rq);
+    }
+    if (lane == 0) lam[j] = (nj > 0.0 && rq > 0.0) ? nj : 0.0;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) rank[j] = desc_rank(lam, d, j);
+  __syncthreads();
+  double part = 0.0;
+  for (int j = threadIdx.x; j < d; j += blockDim.x)
+    if (rank[j] < r) part += lam[j];
+  const double mean = block_sum(part, red) / (double)r;
+  const bool ok = mean > 0.0 && isfinite(mean);
+  if (!ok && threadIdx.x == 0) atomicOr(err, err_bit);
+  for (int j = threadIdx.x; j < d; j += blockDim.x)
+    if (rank[j] < r) lam_out[(long long)h * r + rank[j]] = lam[j];
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int j = e / d, i = e % d;   // column j, row i
+    const int k = rank[j];
+    if (k >= r) continue;
+    double v = 0.0;
+    if (ok && norm[j] > 0.0) v = G[j * d + i] / norm[j] * sqrt(lam[j] / mean);
+    F64[((long long)h * d + i) * r + k] = v;
+    F32[((long long)h * d + i) * r + k] = (float)v;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Probe fit.  x_p = sparse output of probe p, R_p = exact output - x_p,
+// w_p = |G_a|/m_a (review page step 4).  Unit-sum weights give mu_x, mu_R and
+// s = sqrt(weighted variance + 1e-6) (App. A.3, App. D.3); unit-mean weights omega weigh
+// the ridge objective (App. A.3).  With A = Omega^{1/2} X_bar and Y = Omega^{1/2} R_bar,
+// B = (A^T A + lambda I)^-1 A^T Y = A^T (A A^T + lambda I)^-1 Y; the smaller system is
+// solved by Cholesky.  Psi_r = leading r right singular vectors of Y (App. D.2).
+// The correction is folded as B' = diag(1/s) B P, c = mu_R - (mu_x / s) B P.
+
+// In-place Cholesky of an n x n SPD matrix (row-major, smem). Returns false if not PD.
+__device__ bool cholesky(double* L, int n, int* bad) {
+  if (threadIdx.x == 0) *bad = 0;
+  __syncthreads();
+  for (int k = 0; k < n; ++k) {
+    if (threadIdx.x == 0) {
+      const double dkk = L[k * n + k];
+      if (!(dkk > 0.0) || !isfinite(dkk)) *bad = 1;
+      L[k * n + k] = dkk > 0.0 ? sqrt(dkk) : 1.0;
+    }
+    __syncthreads();
+    const double piv = L[k * n + k];
+    for (int i = k + 1 + threadIdx.x; i < n; i += blockDim.x) L[i * n + k] /= piv;
+    __syncthreads();
+    const int rem = n - k - 1;
+    for (int e = threadIdx.x; e < rem * rem; e += blockDim.x) {
+      const int i = k + 1 + e / rem, j = k + 1 + e % rem;
+      if (j <= i) L[i * n + j] -= L[i * n + k] * L[j * n + k];
+    }
+    __syncthreads();
+  }
+  return *bad == 0;
+}
+
+// Solve (L L^T) Z = Z in place for `ncols` right-hand-side columns of Z (n x ldz,
+// row-major, global); one thread per column.
+__device__ void cholesky_solve(const double* L, int n, double* Z, int ldz, int ncols) {
+  for (int c = threadIdx.x; c < ncols; c += blockDim.x) {
+    for (int i = 0; i < n; ++i) {
+      double v = Z[(long long)i * ldz + c];
+      for (int k = 0; k < i; ++k) v -= L[i * n + k] * Z[(long long)k * ldz + c];
+      Z[(long long)i * ldz + c] = v / L[i * n + i];
+    }
+    for (int i = n - 1; i >= 0; --i) {
+      double v = Z[(long long)i * ldz + c];
+      for (int k = i + 1; k < n; ++k) v -= L[k * n + i] * Z[(long long)k * ldz + c];
+      Z[(long long)i * ldz + c] = v / L[i * n + i];
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
+  extern __shared__ double S[];   // max(n*n, M*d) doubles
+  __shared__ double red[32];
+  __shared__ double sig[kMaxM];
+  __shared__ int srank[kMaxM];
+  __shared__ int flag, bad;
+  const int h = blockIdx.x, d = m.d, M = m.M;
+  const long long hd = (long long)h * d;
+  double* A = b.fitA + (long long)h * M * d;   // [M][d]
+  double* Y = b.fitY + (long long)h * M * d;   // [M][d]
+  double* Z = b.fitZ + (long long)h * (M > d ? M : d) * d;
+  const int* probes = b.probes + (long long)h * M;
+  const double* w = b.wP + (long long)h * M;
+
+  // weights
+  double wsum = 0.0;
+  for (int p = 0; p < M; ++p) wsum += w[p];   // every thread, same order
+  // x (sparse output at the probe rows) and R = dense - sparse, staged in A and Y
+  for (int e = threadIdx.x; e < M * d; e += blockDim.x) {
+    const int p = e / d, j = e % d;
+    const int pos = b.invQ[(long long)h * m.Nq + probes[p]];
+    const double x = (double)b.Osp[((long long)h * m.Nq + pos) * d + j];
+    const double dn = (double)b.Odense[((long long)h * M + p) * d + j];
+    A[e] = x;
+    Y[e] = dn - x;
+    if (!isfinite(x) || !isfinite(dn)) atomicOr(b.err, kErrNonFinite);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double mx = 0.0, mr = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const double wt = w[p] / wsum;
+      mx += wt * A[p * d + j];
+      mr += wt * Y[p * d + j];
+    }
+    double var = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const double t = A[p * d + j] - mx;
+      var += (w[p] / wsum) * t * t;
+    }
+    b.muX[hd + j] = mx;
+    b.muR[hd + j] = mr;
+    b.sX[hd + j] = sqrt(var + 1e-6);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < M * d; e += blockDim.x) {
+    const int p = e / d, j = e % d;
+    const double om = sqrt((double)M * w[p] / wsum);
+    A[e] = om * (A[e] - b.muX[hd + j]) / b.sX[hd + j];
+    Y[e] = om * (Y[e] - b.muR[hd + j]);
+  }
+  __syncthreads();
+
+  // ---- ridge: solve the smaller of the dual (M x M) and primal (d x d) systems
+  double* Bh = b.Bm + (long long)h * d * d;
+  const bool dual = M <= d;
+  const int n = dual ? M : d;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    double g = 0.0;
+    if (dual) for (int k = 0; k < d; ++k) g += A[i * d + k] * A[j * d + k];
+    else      for (int k = 0; k < M; ++k) g += A[k * d + i] * A[k * d + j];
+    S[e] = g + (i == j ? m.lambda : 0.0);
+  }
+  for (int e = threadIdx.x; e < n * d; e += blockDim.x) {
+    const int i = e / d, j = e % d;
+    if (dual) {
+      Z[e] = Y[e];
+    } else {
+      double g = 0.0;
+      for (int k = 0; k < M; ++k) g += A[k * d + i] * Y[k * d + j];
+      Z[e] = g;
+    }
+  }
+  __syncthreads();
+  const bool pd = cholesky(S, n, &bad);
+  if (!pd && threadIdx.x == 0) atomicOr(b.err, kErrNonFinite);
+  cholesky_solve(S, n, Z, d, d);
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    double v = 0.0;
+    if (pd) {
+      if (dual) {
+        const int i = e / d, j = e % d;
+        for (int p = 0; p < M; ++p) v += A[p * d + i] * Z[p * d + j];
+      } else {
+        v = Z[e];
+      }
+    }
+    Bh[e] = v;
+  }
+  __syncthreads();
+
+  // ---- residual subspace: orthogonalise the columns of Y^T (column p = Y[p][:])
+  double* Ph = b.Pm + (long long)h * d * d;
+  int reff;
+  if (m.r == 0) {
+    reff = d;
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) Ph[e] = (e / d == e % d) ? 1.0 : 0.0;
+  } else {
+    for (int e = threadIdx.x; e < M * d; e += blockDim.x) S[e] = Y[e];
+    __syncthreads();
+    hestenes(S, d, M, &flag);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int p = warp; p < M; p += nwarps) {
+      double s2 = 0.0;
+      for (int i = lane; i < d; i += 32) s2 += S[p * d + i] * S[p * d + i];
+      s2 = warp_sum(s2);
+      if (lane == 0) sig[p] = sqrt(s2);
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < M; p += blockDim.x) srank[p] = desc_rank(sig, M, p);
+    __syncthreads();
+    double smax = 0.0;
+    for (int p = 0; p < M; ++p) smax = sig[p] > smax ? sig[p] : smax;
+    int keep = 0;
+    if (smax > 0.0)
+      for (int p = 0; p < M; ++p) keep += sig[p] > 1e-10 * smax;
+    reff = m.r < keep ? m.r : keep;
+    for (int p = threadIdx.x; p < M; p += blockDim.x) b.sig[(long long)h * kMaxM + srank[p]] = sig[p];
+    // P = sum over kept columns of u u^T
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+      const int i = e / d, j = e % d;
+      double v = 0.0;
+      for (int p = 0; p < M; ++p)
+        if (srank[p] < reff) v += S[p * d + i] * S[p * d + j] / (sig[p] * sig[p]);
+      Ph[e] = v;
+    }
+  }
+  if (threadIdx.x == 0) b.reff[h] = reff;
+  __syncthreads();
+
+  // ---- fold: BP = B P (into Z), B' = diag(1/s) BP, c = mu_R - (mu_x/s) BP
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int i = e / d, j = e % d;
+    double v = 0.0;
+    for (int k = 0; k < d; ++k) v += Bh[i * d + k] * Ph[k * d + j];
+    Z[e] = v;
+    b.Bp[(long long)h * d * d + e] = (float)(v / b.sX[hd + i]);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double v = b.muR[hd + j];
+    for (int i = 0; i < d; ++i) v -= (b.muX[hd + i] / b.sX[hd + i]) * Z[i * d + j];
+    b.cvec[hd + j] = (float)v;
+  }
+}
+
+}  // namespace
+
+sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st) {
+  const size_t smem = 64 * p.dm.d * sizeof(float);
+  key_metric_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.Q, p.b.MK);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st) {
+  const size_t smem = (size_t)p.dm.d * p.dm.d * sizeof(double);
+  SPR_CUDA_OK(cudaFuncSetAttribute(eigen_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (query)
+    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MQ, p.dm.rQ, p.b.lamQ, p.b.FQ64, p.b.FQ, p.b.err, kErrEigQ);
+  else
+    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MK, p.dm.rK, p.b.lamK, p.b.FK64, p.b.FK, p.b.err, kErrEigK);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_fit(const Plan& p, cudaStream_t st) {
+  const int d = p.dm.d, M = p.dm.M;
+  const int n = M <= d ? M : d;
+  const size_t smem = (size_t)((n * n > M * d) ? n * n : M * d) * sizeof(double);
+  SPR_CUDA_OK(cudaFuncSetAttribute(fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  fit_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+}  // namespace spr

@@ -1,0 +1,309 @@
+// Routing, group-major permutation and probe selection.
+//   Routing (paper App. B.3, S4.3): a score per (query group, K/V group) cell from the
+//   query, key and value centroids; each query group keeps the shortest prefix of K/V
+//   groups ranked by decreasing score whose key-token count reaches the common budget
+//   beta = (rho* - M/N_q) N_k.  The score is a reading of the SVG-EAR value error score
+//   the paper names: l_ab = tau qbar_a.kbar_b + ln|G_b|, pi_ab = softmax_b(l_ab),
+//   ohat_a = sum_b pi_ab vbar_b, score_ab = pi_ab ||vbar_b - ohat_a||, in fp64.
+//   Permutation (review page step 3): Q, K, V copied into group-major order.
+//   Probes (App. A.2, Algorithm A.1): stratified radial round robin.
+#include <cmath>
+
+#include "common.cuh"
+
+namespace spr {
+namespace {
+
+__global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
+  __shared__ double qa[kMaxD], oh[kMaxD];
+  __shared__ double lg[kMaxC];
+  __shared__ double red[32];
+  const int h = blockIdx.y, a = blockIdx.x, d = m.d;
+  if (a >= b.nQ[h]) return;
+  const int n = b.nK[h];
+  const double tau = 1.0 / sqrt((double)d);
+  const double* kb = b.kbar + (long long)h * m.Ck * d;
+  const double* vb = b.vbar + (long long)h * m.Ck * d;
+  const int* sz = b.sizeK + (long long)h * m.Ck;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) qa[j] = b.qbar[((long long)h * m.Cq + a) * d + j];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int k = warp; k < n; k += nw) {
+    double s = 0.0;
+    for (int j = lane; j < d; j += 32) s += qa[j] * kb[(long long)k * d + j];
+    s = warp_sum(s);
+    if (lane == 0) lg[k] = tau * s + log((double)sz[k]);
+  }
+  __syncthreads();
+  double mx = -INFINITY;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) mx = fmax(mx, lg[k]);
+  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int w = 1; w < nw; ++w) mx = fmax(mx, red[w]);
+  __syncthreads();
+  double part = 0.0;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const double e = exp(lg[k] - mx);
+    lg[k] = e;
+    part += e;
+  }
+  const double tot = block_sum(part, red);
+  for (int k = threadIdx.x; k < n; k += blockDim.x) lg[k] /= tot;
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double s = 0.0;
+    for (int k = 0; k < n; ++k) s += lg[k] * vb[(long long)k * d + j];
+    oh[j] = s;
+  }
+  __syncthreads();
+  double* out = b.scores + ((long long)h * m.Cq + a) * m.Ck;
+  for (int k = warp; k < n; k += nw) {
+    double s = 0.0;
+    for (int j = lane; j < d; j += 32) {
+      const double t = vb[(long long)k * d + j] - oh[j];
+      s += t * t;
+    }
+    s = warp_sum(s);
+    if (lane == 0) out[k] = lg[k] * sqrt(s);
+  }
+}
+
+// Prefix budget selection for one query group; selected ids written ascending.
+__global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
+  __shared__ double key[kMaxC];
+  __shared__ int id[kMaxC];
+  __shared__ int flag[kMaxC];
+  __shared__ int sh[32];
+  __shared__ int cut;
+  const int h = blockIdx.y, a = blockIdx.x;
+  if (a >= b.nQ[h]) return;
+  const int n = b.nK[h];
+  int P2 = 1;
+  while (P2 < n) P2 <<= 1;
+  const double* S = b.scores + ((long long)h * m.Cq + a) * m.Ck;
+  for (int t = threadIdx.x; t < P2; t += blockDim.x) {
+    key[t] = t < n ? S[t] : -INFINITY;
+    id[t] = t < n ? t : (1 << 30) + t;
+  }
+  if (threadIdx.x == 0) cut = n;
+  __syncthreads();
+  // bitonic sort: decreasing score, ties by increasing id
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < P2; t += blockDim.x) {
+        const int u = t ^ j;
+        if (u > t) {
+          const bool up = (t & k) == 0;
+          const bool t_first = key[t] > key[u] || (key[t] == key[u] && id[t] < id[u]);
+          if (t_first != up) {
+            const double kk = key[t]; key[t] = key[u]; key[u] = kk;
+            const int ii = id[t]; id[t] = id[u]; id[u] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int* sz = b.sizeK + (long long)h * m.Ck;
+  const int t = threadIdx.x;
+  const int mine = t < n ? sz[id[t]] : 0;
+  int tot;
+  const int excl = block_exclusive_scan(mine, sh, &tot);
+  const long long incl = (long long)excl + mine;
+  if (t < n && (double)incl >= m.beta && (t == 0 || (double)excl < m.beta)) cut = t + 1;
+  __syncthreads();
+  const int cnt = cut;
+  for (int u = threadIdx.x; u < n; u += blockDim.x) flag[u] = 0;
+  __syncthreads();
+  if (t < cnt) flag[id[t]] = 1;
+  __syncthreads();
+  const int f = t < n ? flag[t] : 0;
+  const int pos = block_exclusive_scan(f, sh, &tot);
+  int* ids = b.cellIds + ((long long)h * m.Cq + a) * m.Ck;
+  if (f) ids[pos] = t;
+  // routed pairs: |G_a| * (selected key tokens)
+  long long keys = 0;
+  if (t < n && flag[t]) keys = sz[t];
+  for (int o = 16; o > 0; o >>= 1) keys += __shfl_xor_sync(0xffffffffu, keys, o);
+  if ((t & 31) == 0 && keys)
+    atomicAdd(reinterpret_cast<unsigned long long*>(b.pairs + h),
+              (unsigned long long)(keys * (long long)b.sizeQ[(long long)h * m.Cq + a]));
+  if (t == 0) b.cellCnt[(long long)h * m.Cq + a] = cnt;
+}
+
+// Group-major copies of Q, K, V with 16-byte vector loads; inverse query permutation.
+__global__ void gather_kernel(const void* src, void* dst, const int* perm, int* inv, int H, int N,
+                              int row_chunks) {
+  const long long total = (long long)H * N * row_chunks;
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const long long row = t / row_chunks;          // h * N + pos
+    const int c = (int)(t % row_chunks);
+    const long long h = row / N;
+    const int srow = perm[row];
+    const uint4* s = reinterpret_cast<const uint4*>(src) + (h * N + srow) * row_chunks + c;
+    uint4* o = reinterpret_cast<uint4*>(dst) + row * row_chunks + c;
+    *o = __ldg(s);
+    if (inv && c == 0) inv[h * N + srow] = (int)(row - h * N);
+  }
+}
+
+// Squared distance of each query's phi_Q to its group centre (fp32, ascending dims).
+__global__ void probe_dist_kernel(Dims m, Buffers b) {
+  const int h = blockIdx.y;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= m.Nq) return;
+  const int lab = b.labQ[(long long)h * m.Nq + i];
+  const float* x = b.phiQ + ((long long)h * m.Nq + i) * m.rQ;
+  const float* c = b.centQ + ((long long)h * m.Cq + lab) * m.rQ;
+  float s = 0.0f;
+  for (int k = 0; k < m.rQ; ++k) {
+    const float t = x[k] - c[k];
+    s = fmaf(t, t, s);
+  }
+  b.dist[(long long)h * m.Nq + i] = s;
+}
+
+// Passes P of the round robin: smallest p with sum_a min(|G_a|, p) >= M.
+__device__ int probe_passes(const int* sz, int n, int M) {
+  int p = 1;
+  for (;; ++p) {
+    long long c = 0;
+    for (int a = 0; a < n; ++a) c += sz[a] < p ? sz[a] : p;
+    if (c >= M || p >= M) return p;
+  }
+}
+
+// Per query group: its first min(P, |G_a|) rows by (d_i, row) ascending. One warp.
+__global__ void __launch_bounds__(32) probe_rank_kernel(Dims m, Buffers b) {
+  const int h = blockIdx.y, a = blockIdx.x, lane = threadIdx.x;
+  const int n = b.nQ[h];
+  if (a >= n) return;
+  const int* sz = b.sizeQ + (long long)h * m.Cq;
+  const int P = probe_passes(sz, n, m.M);
+  const int lab = b.usedQ[(long long)h * m.Cq + a];
+  const int m0 = b.offQ[(long long)h * (m.Cq + 1) + lab], m1 = b.offQ[(long long)h * (m.Cq + 1) + lab + 1];
+  const int take = (m1 - m0) < P ? (m1 - m0) : P;
+  const int* perm = b.permQ + (long long)h * m.Nq;
+  const float* dist = b.dist + (long long)h * m.Nq;
+  float pd = -INFINITY;
+  int pi = -1;
+  for (int t = 0; t < take; ++t) {
+    float bd = INFINITY;
+    int bi = 0x7fffffff;
+    for (int mm = m0 + lane; mm < m1; mm += 32) {
+      const int row = perm[mm];
+      const float dv = dist[row];
+      const bool after = dv > pd || (dv == pd && row > pi);
+      const bool better = dv < bd || (dv == bd && row < bi);
+      if (after && better) {
+        bd = dv;
+        bi = row;
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (od < bd || (od == bd && oi < bi)) {
+        bd = od;
+        bi = oi;
+      }
+    }
+    if (lane == 0) b.probeTop[((long long)h * m.Cq + a) * m.M + t] = bi;
+    pd = bd;
+    pi = bi;
+  }
+}
+
+// Round robin over groups by decreasing size (ties by index); weights w_p = |G_a|/m_a.
+__global__ void __launch_bounds__(1024) probe_pick_kernel(Dims m, Buffers b) {
+  __shared__ int ord[kMaxC];
+  __shared__ int ksz[kMaxC];
+  __shared__ int cnt[kMaxC];
+  const int h = blockIdx.x, n = b.nQ[h];
+  const int* sz = b.sizeQ + (long long)h * m.Cq;
+  int P2 = 1;
+  while (P2 < n) P2 <<= 1;
+  for (int t = threadIdx.x; t < P2; t += blockDim.x) {
+    ord[t] = t;
+    ksz[t] = t < n ? sz[t] : -1;
+  }
+  for (int t = threadIdx.x; t < m.Cq; t += blockDim.x) cnt[t] = 0;
+  __syncthreads();
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < P2; t += blockDim.x) {
+        const int u = t ^ j;
+        if (u > t) {
+          const bool up = (t & k) == 0;
+          const bool t_first = ksz[t] > ksz[u] || (ksz[t] == ksz[u] && ord[t] < ord[u]);
+          if (t_first != up) {
+            int x = ksz[t]; ksz[t] = ksz[u]; ksz[u] = x;
+            x = ord[t]; ord[t] = ord[u]; ord[u] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x == 0) {
+    const int P = probe_passes(sz, n, m.M);
+    int taken = 0;
+    for (int t = 0; t < P && taken < m.M; ++t) {
+      for (int k = 0; k < n && taken < m.M; ++k) {
+        const int a = ord[k];
+        if (sz[a] > t) {
+          b.probes[(long long)h * m.M + taken] = b.probeTop[((long long)h * m.Cq + a) * m.M + t];
+          b.probeA[(long long)h * m.M + taken] = a;
+          cnt[a] += 1;
+          ++taken;
+        }
+      }
+    }
+    if (taken < m.M) atomicOr(b.err, kErrProbe);
+  }
+  __syncthreads();
+  for (int a = threadIdx.x; a < m.Cq; a += blockDim.x) b.mA[(long long)h * m.Cq + a] = cnt[a];
+  for (int p = threadIdx.x; p < m.M; p += blockDim.x) {
+    const int a = b.probeA[(long long)h * m.M + p];
+    b.wP[(long long)h * m.M + p] = (double)sz[a] / (double)cnt[a];
+  }
+}
+
+}  // namespace
+
+sparsepr_status launch_route(const Plan& p, cudaStream_t st) {
+  const Dims& m = p.dm;
+  score_kernel<<<dim3(m.Cq, m.H), 256, 0, st>>>(m, p.b);
+  SPR_LAUNCH_OK();
+  select_kernel<<<dim3(m.Cq, m.H), 1024, 0, st>>>(m, p.b);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_permute(const Plan& p, cudaStream_t st) {
+  const Dims& m = p.dm;
+  const int es = m.dtype == SPARSEPR_BF16 ? 2 : 4;
+  const int chunks = m.d * es / 16;
+  const int blocks = 148 * 8;
+  gather_kernel<<<blocks, 256, 0, st>>>(p.Q, p.b.Qp, p.b.permQ, p.b.invQ, m.H, m.Nq, chunks);
+  gather_kernel<<<blocks, 256, 0, st>>>(p.K, p.b.Kp, p.b.permK, nullptr, m.H, m.Nk, chunks);
+  gather_kernel<<<blocks, 256, 0, st>>>(p.V, p.b.Vp, p.b.permK, nullptr, m.H, m.Nk, chunks);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_select_probes(const Plan& p, cudaStream_t st) {
+  const Dims& m = p.dm;
+  probe_dist_kernel<<<dim3(cdiv(m.Nq, 256), m.H), 256, 0, st>>>(m, p.b);
+  SPR_LAUNCH_OK();
+  probe_rank_kernel<<<dim3(m.Cq, m.H), 32, 0, st>>>(m, p.b);
+  SPR_LAUNCH_OK();
+  probe_pick_kernel<<<m.H, 1024, 0, st>>>(m, p.b);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+}  // namespace spr

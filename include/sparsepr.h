@@ -1,0 +1,237 @@
+/*
+ * sparsepr.h -- C ABI of the B200 SparsePR per-call sparse attention library.
+ *
+ * SparsePR ("Partition the Support, Reconstruct the Residual: Training-Free Sparse
+ * Attention for Video Generation and World Models") replaces one dense attention call
+ * O = softmax(Q K^T / sqrt(d)) V, per head, by four stages:
+ *
+ *   sparsepr_plan       Response-Coupled Partitioning and routing (paper S4.1, App. B):
+ *                       key response metric from M_s evenly spaced query rows, its
+ *                       eigen-weighted rank-r_K factor, k-means of the key coordinates
+ *                       into C_k paired K/V groups, the query metric of the centred
+ *                       non-empty K/V centroids, RMS-normalised rank-r_Q query
+ *                       coordinates, k-means into C_q query groups; routing scores per
+ *                       (query group, K/V group) cell and the shortest score-ranked
+ *                       prefix reaching the per-query key budget (App. B.3, S4.3);
+ *                       group-major permutation of Q, K, V; Algorithm A.1 probe rows.
+ *   sparsepr_attend     renormalised hard-drop block-sparse attention over the
+ *                       selected cells (paper S2).
+ *   sparsepr_probe_fit  exact attention of the M probe rows against all keys, the
+ *                       coverage-weighted statistics and ridge fit of the residual on
+ *                       the sparse output, and the leading-r residual subspace
+ *                       (paper S4.2, App. A.2-A.3, App. D.2).
+ *   sparsepr_correct    corrected output for unprobed rows, dense output for probe
+ *                       rows, restored to the original token order.
+ *
+ * Conventions (every entry point):
+ *   - Q is [H, N_q, d], K and V are [H, N_k, d], contiguous row-major DEVICE memory in
+ *     the dtype of sparsepr_params.dtype (fp32 or bf16).  Out is [H, N_q, d] in the same
+ *     dtype.  d must be a multiple of 8 and at most 128.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every call except sparsepr_get_stats, sparsepr_export and sparsepr_check only
+ *     enqueues work on it and never synchronises the host.
+ *   - The caller owns Q, K, V, Out and the workspace (device memory of at least
+ *     sparsepr_workspace_size bytes, 256-byte aligned).  A plan handle is host memory
+ *     owned by the library until sparsepr_destroy; it refers to, but does not own, the
+ *     workspace and the input tensors, which must stay valid until the last call on the
+ *     plan has completed on the GPU.
+ *   - Errors: arguments are validated on the host before any launch (SPARSEPR_ERR_ARG,
+ *     SPARSEPR_ERR_SHAPE, SPARSEPR_ERR_DTYPE, SPARSEPR_ERR_WORKSPACE); a CUDA launch
+ *     error returns SPARSEPR_ERR_CUDA; calls out of order return SPARSEPR_ERR_STATE.
+ *     Inconsistencies found on the device (a metric with no positive eigenvalue,
+ *     non-finite values) set a device error word that sparsepr_check and
+ *     sparsepr_get_stats report as SPARSEPR_ERR_DEVICE_CHECK.  No call traps or aborts
+ *     the CUDA context.
+ */
+#ifndef SPARSEPR_H
+#define SPARSEPR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPARSEPR_OK = 0,
+  SPARSEPR_ERR_ARG = 1,          /* a parameter is out of its valid range */
+  SPARSEPR_ERR_SHAPE = 2,        /* H, N, d or a group count is unsupported */
+  SPARSEPR_ERR_DTYPE = 3,        /* dtype is neither SPARSEPR_F32 nor SPARSEPR_BF16 */
+  SPARSEPR_ERR_WORKSPACE = 4,    /* workspace missing, misaligned or too small */
+  SPARSEPR_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+  SPARSEPR_ERR_DEVICE_CHECK = 6, /* the device error word is set (see sparsepr_check) */
+  SPARSEPR_ERR_STATE = 7         /* call out of order for this plan */
+} sparsepr_status;
+
+typedef enum { SPARSEPR_F32 = 0, SPARSEPR_BF16 = 1 } sparsepr_dtype;
+
+/* Attention engine used by sparsepr_attend and sparsepr_dense_attention. */
+typedef enum {
+  SPARSEPR_ENGINE_AUTO = 0,   /* tensor-core engine for bf16, CUDA-core engine for fp32 */
+  SPARSEPR_ENGINE_SIMT = 1    /* fp32 CUDA-core engine for every dtype (reference path) */
+} sparsepr_engine;
+
+/*
+ * Problem and hyper-parameters of one call (paper S2, S4; values of the review page's
+ * hyper-parameter table: r_K=48, r_Q=64, M=64, r=16, lambda=0.1).
+ *   H                 heads (each head is an independent problem)
+ *   N_q, N_k          query and key/value tokens per head
+ *   d                 head dimension (multiple of 8, <= 128)
+ *   dtype             sparsepr_dtype of Q, K, V and Out
+ *   M_s               sampled query rows for the key metric (rows floor(s*N_q/M_s))
+ *   r_K, r_Q          ranks of the key and query response coordinates (1..min(d,64))
+ *   C_q, C_k          requested query / K-V group counts (1..1024, <= N_q / N_k)
+ *   M                 probe rows (1..128, <= N_q)
+ *   r                 residual-subspace rank (0 = no projection; else 1..M)
+ *   lambda            ridge strength (>= 0)
+ *   target_density    executed-pair target rho* including probes (M/N_q < rho* <= 1)
+ *   kmeans_max_iter   Lloyd assignment steps at most (1..1000; the paper uses 25)
+ *   engine            sparsepr_engine
+ *   seed              seed of the SplitMix64 stream that draws the k-means initial rows
+ */
+typedef struct {
+  int32_t H, N_q, N_k, d;
+  int32_t dtype;
+  int32_t M_s, r_K, r_Q, C_q, C_k, M, r;
+  double lambda;
+  double target_density;
+  int32_t kmeans_max_iter;
+  int32_t engine;
+  uint64_t seed;
+} sparsepr_params;
+
+typedef struct sparsepr_plan_s* sparsepr_plan_t;
+
+/* Whole-call statistics (summed over heads).  Realised densities follow paper S2/S4.3:
+ * rho_route = routed pairs / (H N_q N_k), rho_exec = (routed pairs + H M N_k)/(H N_q N_k). */
+typedef struct {
+  int64_t pairs_route;
+  int64_t pairs_exec;
+  double rho_route;
+  double rho_exec;
+  int32_t kmeans_iters_k_max;
+  int32_t kmeans_iters_q_max;
+  int32_t groups_k_min;      /* smallest per-head count of non-empty K/V groups */
+  int32_t groups_q_min;      /* smallest per-head count of non-empty query groups */
+  int32_t device_error;      /* device error word (0 = none) */
+} sparsepr_stats;
+
+/* Bytes of device workspace a plan with these parameters needs.  Host only. */
+sparsepr_status sparsepr_workspace_size(const sparsepr_params* params, size_t* bytes);
+
+/*
+ * Response-Coupled Partitioning, routing, permutation and probe selection for all heads.
+ * Q, K, V: device [H,N,d].  workspace: device, >= sparsepr_workspace_size bytes.
+ * On success *out receives a new plan handle (host memory).  Asynchronous on `stream`.
+ */
+sparsepr_status sparsepr_plan(const sparsepr_params* params, const void* Q, const void* K,
+                              const void* V, void* workspace, size_t workspace_bytes,
+                              void* stream, sparsepr_plan_t* out);
+
+/*
+ * As sparsepr_plan, but the k-means labels are given: labQ [H,N_q] and labK [H,N_k] are
+ * device int32 arrays with values in [0,C_q) and [0,C_k).  Every later step (groups,
+ * centroids, query coordinates, routing, permutation, probes) is computed from them
+ * exactly as sparsepr_plan computes it from its own k-means labels.  For testing the
+ * stages after clustering against a reference given identical labels.
+ */
+sparsepr_status sparsepr_plan_from_labels(const sparsepr_params* params, const void* Q,
+                                          const void* K, const void* V,
+                                          const int32_t* labQ, const int32_t* labK,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream, sparsepr_plan_t* out);
+
+/* Renormalised hard-drop attention over the selected cells; the sparse output stays in
+ * the workspace (group-major, fp32).  Requires a plan.  Asynchronous. */
+sparsepr_status sparsepr_attend(sparsepr_plan_t plan, void* stream);
+
+/* Exact probe attention, residual statistics, ridge fit, residual subspace and the folded
+ * correction.  Requires sparsepr_attend.  Asynchronous. */
+sparsepr_status sparsepr_probe_fit(sparsepr_plan_t plan, void* stream);
+
+/* Writes the corrected output Out (device [H,N_q,d], params dtype) in the original token
+ * order: O_sp + mu_R + ((O_sp - mu_x)/s) B P for unprobed rows, the exact dense output
+ * for probe rows.  Requires sparsepr_probe_fit.  Asynchronous. */
+sparsepr_status sparsepr_correct(sparsepr_plan_t plan, void* Out, void* stream);
+
+/* The four calls above in order, on one stream, followed by sparsepr_destroy of the
+ * internal plan (host memory only).  Asynchronous. */
+sparsepr_status sparsepr_forward(const sparsepr_params* params, const void* Q, const void* K,
+                                 const void* V, void* Out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Dense attention softmax(Q K^T / sqrt(d)) V for all rows through the same attention
+ * engine (every key selected).  Only H, N_q, N_k, d, dtype and engine of params are read.
+ * Needs no workspace.  Asynchronous. */
+sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const void* Q,
+                                         const void* K, const void* V, void* Out,
+                                         void* stream);
+
+/* Synchronises `stream` and reports the device error word: SPARSEPR_OK or
+ * SPARSEPR_ERR_DEVICE_CHECK (with the word in *device_error when non-NULL). */
+sparsepr_status sparsepr_check(sparsepr_plan_t plan, void* stream, int32_t* device_error);
+
+/* Synchronises `stream` and fills *stats.  Valid after sparsepr_plan. */
+sparsepr_status sparsepr_get_stats(sparsepr_plan_t plan, void* stream, sparsepr_stats* stats);
+
+/* Internal arrays a plan exposes for inspection (all per head, leading dimension H). */
+typedef enum {
+  SPARSEPR_X_LABELS_K = 0,    /* int32 [H,N_k]   final k-means labels of the keys */
+  SPARSEPR_X_LABELS_Q = 1,    /* int32 [H,N_q]   final k-means labels of the queries */
+  SPARSEPR_X_PERM_K = 2,      /* int32 [H,N_k]   group-major order: row at each position */
+  SPARSEPR_X_PERM_Q = 3,      /* int32 [H,N_q] */
+  SPARSEPR_X_GROUPS_K = 4,    /* int32 [H]       non-empty K/V groups C_k' */
+  SPARSEPR_X_GROUPS_Q = 5,    /* int32 [H]       non-empty query groups C_q' */
+  SPARSEPR_X_SIZES_K = 6,     /* int32 [H,C_k]   sizes of compact K/V groups (first C_k') */
+  SPARSEPR_X_SIZES_Q = 7,     /* int32 [H,C_q] */
+  SPARSEPR_X_CELL_COUNT = 8,  /* int32 [H,C_q]   selected K/V groups per compact query group */
+  SPARSEPR_X_CELL_IDS = 9,    /* int32 [H,C_q,C_k] selected compact K/V ids, ascending */
+  SPARSEPR_X_PROBES = 10,     /* int32 [H,M]     probe rows in selection order */
+  SPARSEPR_X_PROBE_COUNT = 11,/* int32 [H,C_q]   probes per compact query group m_a */
+  SPARSEPR_X_KMEANS_ITERS = 12,/* int32 [H,2]    assignment steps (keys, queries) */
+  SPARSEPR_X_OBJECTIVE = 13,  /* double [H,2]    final k-means objectives (keys, queries) */
+  SPARSEPR_X_PAIRS = 14,      /* int64 [H]       routed pairs per head */
+  SPARSEPR_X_FACTOR_K = 15,   /* double [H,d,r_K] F_K */
+  SPARSEPR_X_FACTOR_Q = 16,   /* double [H,d,r_Q] F_Q */
+  SPARSEPR_X_EIG_K = 17,      /* double [H,r_K]  kept eigenvalues of M_K (descending) */
+  SPARSEPR_X_EIG_Q = 18,      /* double [H,r_Q]  kept eigenvalues of M_Q */
+  SPARSEPR_X_METRIC_K = 19,   /* double [H,d,d]  M_K */
+  SPARSEPR_X_METRIC_Q = 20,   /* double [H,d,d]  M_Q */
+  SPARSEPR_X_PHI_K = 21,      /* float [H,N_k,r_K] key coordinates */
+  SPARSEPR_X_PHI_Q = 22,      /* float [H,N_q,r_Q] query coordinates */
+  SPARSEPR_X_CENTRES_Q = 23,  /* float [H,C_q,r_Q] query-group centres in phi_Q space (raw labels) */
+  SPARSEPR_X_SCORES = 24,     /* double [H,C_q,C_k] routing scores (compact ids) */
+  SPARSEPR_X_OSP = 25,        /* float [H,N_q,d] sparse output, group-major order */
+  SPARSEPR_X_ODENSE_PROBE = 26,/* float [H,M,d]  exact output of the probe rows */
+  SPARSEPR_X_FIT_MU_X = 27,   /* double [H,d] */
+  SPARSEPR_X_FIT_MU_R = 28,   /* double [H,d] */
+  SPARSEPR_X_FIT_S = 29,      /* double [H,d] */
+  SPARSEPR_X_FIT_B = 30,      /* double [H,d,d] ridge coefficients B_lambda */
+  SPARSEPR_X_FIT_P = 31,      /* double [H,d,d] projector Psi_r Psi_r^T */
+  SPARSEPR_X_FIT_REFF = 32,   /* int32 [H]      rank kept in the projector */
+  SPARSEPR_X_PROBE_DIST = 33, /* float [H,N_q]  squared phi_Q distance to the group centre */
+  SPARSEPR_X_KBAR = 34,       /* double [H,C_k,d] K/V group key centroids (compact ids) */
+  SPARSEPR_X_QBAR = 35,       /* double [H,C_q,d] query group centroids (compact ids) */
+  SPARSEPR_X_COUNT = 36
+} sparsepr_export_what;
+
+/* Size in bytes of an exported array for this plan. Host only. */
+sparsepr_status sparsepr_export_size(sparsepr_plan_t plan, int32_t what, size_t* bytes);
+
+/* Synchronises `stream`, then copies the array `what` into HOST memory `dst` of exactly
+ * sparsepr_export_size bytes (SPARSEPR_ERR_ARG otherwise). */
+sparsepr_status sparsepr_export(sparsepr_plan_t plan, int32_t what, void* dst, size_t bytes,
+                                void* stream);
+
+/* Frees the plan handle (host memory only; the workspace stays the caller's). */
+void sparsepr_destroy(sparsepr_plan_t plan);
+
+/* Static text for a status code. */
+const char* sparsepr_status_string(sparsepr_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEPR_H */

@@ -1,0 +1,367 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Two modes, as the acceptance rules of the method's reproduction fix them:
+  * free running: the GPU runs its own k-means (same SplitMix64 initial rows as the
+    oracle); labels must agree on >= 99.9% of rows and objectives within 1e-4 relative;
+  * labels injected: the GPU plan is built from the ORACLE's final labels; then every
+    indexing result (permutations, group sizes, selected cells, routed pairs, probe rows)
+    must be bit-exact and the corrected output within 1e-5 (fp32) / 1e-2 (bf16) relative
+    Frobenius error.
+Full-size workloads (the shapes the benchmark times) are checked on sampled heads and
+2048 evenly spaced rows per head, the oracle computing only those rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from free_block_sparse_plan_b200 import native as N
+from free_block_sparse_plan_b200 import workloads as W
+from oracle import sparsepr_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 1e-2}
+_oracle_cache = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import __graft_entry__
+    __graft_entry__.build()
+
+
+def oracle_head(w: W.Workload, h: int, rows=None):
+    """Oracle call for head h of workload w (cached partition per head)."""
+    key = (w.name, w.seed, h)
+    p = O.Params.from_dict(w.params())
+    if key not in _oracle_cache:
+        q, k, v = W.make_head(w, h)
+        _oracle_cache[key] = (q, k, v, O.partition(q, k, v, p, h))
+    q, k, v, part = _oracle_cache[key]
+    return q, k, v, O.sparsepr_call(q, k, v, p, head=h, rows=rows, part=part)
+
+
+def gpu_call(w, inputs=None, labels=None, engine=N.SPARSEPR_ENGINE_AUTO, params=None):
+    Q, K, V = inputs if inputs is not None else W.make_inputs_torch(w, device="cuda")
+    params = params or N.params_from_dict(w.params(), engine)
+    plan = N.Plan(params, Q, K, V, labels=labels)
+    plan.attend()
+    plan.probe_fit()
+    out = plan.correct()
+    torch.cuda.synchronize()
+    return plan, out, (Q, K, V)
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def tie_ambiguous_probes(res: O.CallResult, gpu_probes: np.ndarray, tol=1e-5) -> bool:
+    """True if every mismatch between the GPU's and the oracle's probe list is a swap of
+    rows of one group whose oracle distances agree to `tol` relative."""
+    if np.array_equal(gpu_probes, res.probes):
+        return True
+    comp = res.part.gq.compact
+    for g, o in zip(gpu_probes, res.probes):
+        if g == o:
+            continue
+        if comp[g] != comp[o]:
+            return False
+        dg, do = res.probe_dist[g], res.probe_dist[o]
+        if abs(dg - do) > tol * max(abs(dg), abs(do), 1e-30):
+            return False
+    return True
+
+
+def check_injected_head(plan, out_h, res: O.CallResult, h, w, exact_probes=True):
+    """Bit-exact indexing and output tolerance for head h of a label-injected plan."""
+    gq, gk = res.part.gq, res.part.gk
+    ex = {k: plan.export(k) for k in ("PERM_Q", "PERM_K", "GROUPS_Q", "GROUPS_K", "SIZES_Q",
+                                      "SIZES_K", "CELL_COUNT", "CELL_IDS", "PAIRS", "PROBES",
+                                      "PROBE_COUNT")}
+    assert np.array_equal(ex["PERM_Q"][h], res.permQ)
+    assert np.array_equal(ex["PERM_K"][h], res.permK)
+    assert ex["GROUPS_Q"][h] == gq.sizes.size and ex["GROUPS_K"][h] == gk.sizes.size
+    assert np.array_equal(ex["SIZES_Q"][h][:gq.sizes.size], gq.sizes)
+    assert np.array_equal(ex["SIZES_K"][h][:gk.sizes.size], gk.sizes)
+    for a, sel in enumerate(res.sel):
+        assert ex["CELL_COUNT"][h][a] == sel.size, a
+        assert np.array_equal(ex["CELL_IDS"][h][a][:sel.size], sel), a
+    assert int(ex["PAIRS"][h]) == res.pairs_route
+    if exact_probes:
+        assert tie_ambiguous_probes(res, ex["PROBES"][h]), (ex["PROBES"][h], res.probes)
+        if np.array_equal(ex["PROBES"][h], res.probes):
+            assert np.array_equal(ex["PROBE_COUNT"][h][:gq.sizes.size], res.m_a)
+    err = rel(out_h[res.rows], res.out)
+    assert err < TOL[w.dtype], err
+    return err
+
+
+# ---------------------------------------------------------------------------------- tiny
+def test_tiny_free_running_matches_oracle():
+    w = W.TINY
+    plan, out, _ = gpu_call(w)
+    _, _, _, res = oracle_head(w, 0)
+    labK, labQ = plan.export("LABELS_K")[0], plan.export("LABELS_Q")[0]
+    assert np.mean(labK == res.part.km_K.labels) >= 0.999
+    assert np.mean(labQ == res.part.km_Q.labels) >= 0.999
+    obj = plan.export("OBJECTIVE")[0]
+    assert abs(obj[0] - res.part.km_K.objective) <= 1e-4 * res.part.km_K.objective
+    assert abs(obj[1] - res.part.km_Q.objective) <= 1e-4 * res.part.km_Q.objective
+    iters = plan.export("KMEANS_ITERS")[0]
+    assert tuple(iters) == (res.part.km_K.iterations, res.part.km_Q.iterations)
+    assert plan.check() == 0
+    if np.array_equal(labK, res.part.km_K.labels) and np.array_equal(labQ, res.part.km_Q.labels):
+        assert rel(out[0].double().cpu().numpy(), res.out) < 1e-5
+
+
+def _align_signs(F_gpu, F_ref):
+    s = np.sign((F_gpu * F_ref).sum(axis=0))
+    s[s == 0] = 1
+    return s
+
+
+def test_tiny_injected_stagewise():
+    w = W.TINY
+    _, _, _, res = oracle_head(w, 0)
+    part = res.part
+    labQ = torch.tensor(part.km_Q.labels[None], dtype=torch.int32, device="cuda")
+    labK = torch.tensor(part.km_K.labels[None], dtype=torch.int32, device="cuda")
+    plan, out, _ = gpu_call(w, labels=(labQ, labK))
+    assert plan.check() == 0
+    # key metric and factor (fp64 on both sides)
+    assert rel(plan.export("METRIC_K")[0], part.M_K) < 1e-12
+    assert rel(plan.export("EIG_K")[0], part.lam_K) < 1e-10
+    FK = plan.export("FACTOR_K")[0]
+    s = _align_signs(FK, part.F_K)
+    assert rel(FK * s, part.F_K) < 1e-8
+    assert rel(plan.export("PHI_K")[0] * s, part.phiK) < 1e-5
+    # centroids, query metric, factor, coordinates
+    nk, nq = part.gk.sizes.size, part.gq.sizes.size
+    assert rel(plan.export("KBAR")[0][:nk], part.kbar) < 1e-13
+    assert rel(plan.export("QBAR")[0][:nq], part.qbar) < 1e-13
+    assert rel(plan.export("METRIC_Q")[0], part.M_Q) < 1e-12
+    FQ = plan.export("FACTOR_Q")[0]
+    sq = _align_signs(FQ, part.F_Q)
+    assert rel(FQ * sq, part.F_Q) < 1e-8
+    assert rel(plan.export("PHI_Q")[0] * sq, part.phiQ) < 1e-5
+    # routing scores (fp64), then indexing bit-exact and output
+    assert rel(plan.export("SCORES")[0][:nq, :nk], res.scores) < 1e-12
+    assert rel(plan.export("PROBE_DIST")[0], res.probe_dist) < 1e-5
+    perm = plan.export("PERM_Q")[0]
+    osp = plan.export("OSP")[0]
+    osp_rows = np.empty_like(osp)
+    osp_rows[perm] = osp
+    assert rel(osp_rows, res.osp) < 1e-5
+    assert rel(plan.export("ODENSE_PROBE")[0], res.dense_probe) < 1e-5
+    assert rel(plan.export("FIT_MU_X")[0], res.fit.mu_x) < 1e-5
+    assert rel(plan.export("FIT_S")[0], res.fit.s) < 1e-5
+    assert int(plan.export("FIT_REFF")[0]) == res.fit.r_eff
+    check_injected_head(plan, out[0].double().cpu().numpy(), res, 0, w)
+
+
+def test_tiny_simt_engine_equals_auto():
+    w = W.TINY
+    _, out_a, inputs = gpu_call(w)
+    _, out_s, _ = gpu_call(w, inputs=inputs, engine=N.SPARSEPR_ENGINE_SIMT)
+    assert rel(out_a.cpu().numpy(), out_s.cpu().numpy()) < 1e-6
+
+
+def test_deterministic_reruns():
+    w = W.MID.with_(H=3)
+    _, o1, inputs = gpu_call(w)
+    _, o2, _ = gpu_call(w, inputs=inputs)
+    assert torch.equal(o1, o2)
+
+
+# ---------------------------------------------------------------------------------- mid
+@pytest.fixture(scope="module")
+def mid_runs():
+    w = W.MID
+    inputs = W.make_inputs_torch(w, device="cuda")
+    free_plan, free_out, _ = gpu_call(w, inputs=inputs)
+    ref = [oracle_head(w, h)[3] for h in range(w.H)]
+    labQ = torch.tensor(np.stack([r.part.km_Q.labels for r in ref]), dtype=torch.int32, device="cuda")
+    labK = torch.tensor(np.stack([r.part.km_K.labels for r in ref]), dtype=torch.int32, device="cuda")
+    inj_plan, inj_out, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK))
+    return w, ref, free_plan, free_out, inj_plan, inj_out
+
+
+def test_mid_free_running_labels_and_objective(mid_runs):
+    w, ref, plan, _, _, _ = mid_runs
+    labK, labQ, obj = plan.export("LABELS_K"), plan.export("LABELS_Q"), plan.export("OBJECTIVE")
+    for h, r in enumerate(ref):
+        assert np.mean(labK[h] == r.part.km_K.labels) >= 0.999, h
+        assert np.mean(labQ[h] == r.part.km_Q.labels) >= 0.999, h
+        assert abs(obj[h, 0] - r.part.km_K.objective) <= 1e-4 * r.part.km_K.objective
+        assert abs(obj[h, 1] - r.part.km_Q.objective) <= 1e-4 * r.part.km_Q.objective
+
+
+def test_mid_injected_bit_exact_and_output(mid_runs):
+    w, ref, _, _, plan, out = mid_runs
+    assert plan.check() == 0
+    out_np = out.float().cpu().numpy()
+    errs = [check_injected_head(plan, out_np[h], r, h, w) for h, r in enumerate(ref)]
+    pairs = sum(r.pairs_route for r in ref)
+    st = plan.stats()
+    assert st["pairs_route"] == pairs
+    assert st["pairs_exec"] == pairs + w.H * w.M * w.N
+    assert max(errs) < TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------------- full size
+def _full_size_check(w, heads, nrows=2048):
+    inputs = W.make_inputs_torch(w, device="cuda")
+    free_plan, _, _ = gpu_call(w, inputs=inputs)
+    labK = free_plan.export("LABELS_K")
+    labQ = free_plan.export("LABELS_Q")
+    obj = free_plan.export("OBJECTIVE")
+    rows = np.unique(np.linspace(0, w.N - 1, nrows).astype(np.int64))
+    refs = {}
+    for h in heads:
+        _, _, _, res = oracle_head(w, h, rows=rows)
+        refs[h] = res
+        assert np.mean(labK[h] == res.part.km_K.labels) >= 0.999, h
+        assert np.mean(labQ[h] == res.part.km_Q.labels) >= 0.999, h
+        assert abs(obj[h, 0] - res.part.km_K.objective) <= 1e-4 * res.part.km_K.objective
+        assert abs(obj[h, 1] - res.part.km_Q.objective) <= 1e-4 * res.part.km_Q.objective
+        labK[h] = res.part.km_K.labels
+        labQ[h] = res.part.km_Q.labels
+    del free_plan
+    plan, out, _ = gpu_call(w, inputs=inputs, labels=(torch.tensor(labQ, device="cuda"),
+                                                      torch.tensor(labK, device="cuda")))
+    assert plan.check() == 0
+    for h in heads:
+        check_injected_head(plan, out[h].float().cpu().numpy(), refs[h], h, w)
+
+
+def test_wan_full_size_sampled_heads():
+    _full_size_check(W.WAN, heads=(0, 20, 39))
+
+
+def test_hunyuan_full_size_sampled_heads():
+    _full_size_check(W.HUNYUAN, heads=(0, 23))
+
+
+def test_operating_point_sweep_head0():
+    base = W.WAN
+    q, k, v, _ = oracle_head(base, 0, rows=np.arange(4))
+    part = _oracle_cache[(base.name, base.seed, 0)][3]
+    dt = torch.bfloat16
+    Q, K, V = (torch.from_numpy(x.astype(np.float32))[None].to(dt).cuda() for x in (q, k, v))
+    labQ = torch.tensor(part.km_Q.labels[None], dtype=torch.int32, device="cuda")
+    labK = torch.tensor(part.km_K.labels[None], dtype=torch.int32, device="cuda")
+    rows = np.unique(np.linspace(0, base.N - 1, 1024).astype(np.int64))
+    for rho, M in [(0.12, 64), (0.17, 64), (0.26, 64), (0.35, 64), (0.22, 32), (0.22, 128)]:
+        w = base.with_(H=1, rho=rho, M=M)
+        p = O.Params.from_dict(w.params())
+        res = O.sparsepr_call(q, k, v, p, head=0, rows=rows, part=part)
+        plan, out, _ = gpu_call(w, inputs=(Q, K, V), labels=(labQ, labK))
+        check_injected_head(plan, out[0].float().cpu().numpy(), res, 0, w)
+        st = plan.stats()
+        assert abs(st["rho_exec"] - res.rho_exec) < 1e-15
+
+
+# ---------------------------------------------------------------------------------- edges
+def test_full_density_returns_dense():
+    # rho* = 1 with every group larger than M: every cell is selected, residuals vanish
+    # and the whole call returns dense attention (paper S2: all cells recover dense).
+    w = W.MID.with_(H=2, rho=1.0, M=16, C_q=32, C_k=32)
+    plan, out, (Q, K, V) = gpu_call(w)
+    sizes = plan.export("SIZES_K")
+    ng = plan.export("GROUPS_K")
+    assert all(sizes[h][:ng[h]].min() > w.M for h in range(w.H))
+    st = plan.stats()
+    assert st["rho_route"] == 1.0
+    dense = N.dense_attention(Q, K, V)
+    assert rel(out.float().cpu().numpy(), dense.float().cpu().numpy()) < 1e-2
+    q, k, v = W.make_head(w, 1)
+    rows = np.arange(0, w.N, 97)
+    ref = O.dense_attention(q, k, v, rows)
+    assert rel(out[1].float().cpu().numpy()[rows], ref) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_dense_attention_engine_ragged(dtype):
+    rng = np.random.default_rng(5)
+    H, Nq, Nk, d = 2, 333, 517, 64
+    arrs = [rng.standard_normal((H, n, d)) * s for n, s in ((Nq, 0.7), (Nk, 0.7), (Nk, 1.0))]
+    if dtype == "bf16":
+        arrs = [W.round_to_bf16(a) for a in arrs]
+    td = W.torch_dtype(dtype)
+    Q, K, V = (torch.from_numpy(a.astype(np.float32)).to(td).cuda() for a in arrs)
+    out = N.dense_attention(Q, K, V).float().cpu().numpy()
+    for h in range(H):
+        ref = O.dense_attention(arrs[0][h], arrs[1][h], arrs[2][h])
+        assert rel(out[h], ref) < (1e-5 if dtype == "f32" else 1e-2)
+
+
+def test_ragged_cross_attention_and_empty_groups():
+    # N_q != N_k, neither a multiple of any tile, more requested groups than the data
+    # supports (empty clusters), d = 32, fp32: labels injected from the oracle.
+    rng = np.random.default_rng(9)
+    Nq, Nk, d = 301, 457, 32
+    mu = rng.standard_normal((12, d)) * 2
+    q = mu[rng.integers(0, 12, Nq)] + 0.3 * rng.standard_normal((Nq, d))
+    k = mu[rng.integers(0, 12, Nk)] + 0.3 * rng.standard_normal((Nk, d))
+    v = rng.standard_normal((Nk, d))
+    q, k, v = (x.astype(np.float32).astype(np.float64) for x in (q, k, v))
+    pdict = dict(H=1, N_q=Nq, N_k=Nk, d=d, dtype="f32", M_s=50, r_K=6, r_Q=5, C_q=40, C_k=60,
+                 M=24, r=5, lam=0.1, target_density=0.3, kmeans_max_iter=25, seed=3)
+    p = O.Params.from_dict(pdict)
+    res = O.sparsepr_call(q, k, v, p, head=0)
+    assert res.part.gk.sizes.size < 60 or res.part.gq.sizes.size < 40   # empty groups occurred
+    Q, K, V = (torch.from_numpy(x.astype(np.float32))[None].cuda() for x in (q, k, v))
+    labQ = torch.tensor(res.part.km_Q.labels[None], dtype=torch.int32, device="cuda")
+    labK = torch.tensor(res.part.km_K.labels[None], dtype=torch.int32, device="cuda")
+    params = N.params_from_dict(pdict)
+    plan = N.Plan(params, Q, K, V, labels=(labQ, labK))
+    plan.attend()
+    plan.probe_fit()
+    out = plan.correct()
+    torch.cuda.synchronize()
+    w = W.TINY.with_(N=Nq)
+    check_injected_head(plan, out[0].double().cpu().numpy(), res, 0, w)
+    # free running on the same problem: labels agree with the oracle's own k-means
+    plan2 = N.Plan(params, Q, K, V)
+    assert np.mean(plan2.export("LABELS_K")[0] == res.part.km_K.labels) >= 0.999
+    assert np.mean(plan2.export("LABELS_Q")[0] == res.part.km_Q.labels) >= 0.999
+
+
+def test_probe_rows_are_exact_dense_rows():
+    # Probe rows carry the exact dense output (review page step 5), here with most rows
+    # probed (M = 120 of 128).
+    w = W.TINY.with_(N=128, grid=(2, 8, 8), M=120, r=4, rho=1.0, C_q=8, C_k=8)
+    plan, out, _ = gpu_call(w)
+    q, k, v = W.make_head(w, 0)
+    probes = plan.export("PROBES")[0]
+    assert len(set(probes.tolist())) == 120
+    assert rel(out[0].double().cpu().numpy()[probes], O.dense_attention(q, k, v, probes)) < 1e-5
+
+
+def test_zero_queries_set_device_error_without_fault():
+    # A zero query sample makes the key metric zero: no positive eigenvalue.  The call
+    # completes, the device error word is set and the context stays usable.
+    w = W.TINY
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    Q.zero_()
+    params = N.params_from_dict(w.params())
+    plan = N.Plan(params, Q, K, V)
+    assert plan.check() & 1
+    assert torch.cuda.is_available() and float(torch.ones(1, device="cuda").sum()) == 1.0
+
+
+def test_out_of_range_injected_labels_are_flagged():
+    w = W.TINY
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    labQ = torch.zeros((1, w.N), dtype=torch.int32, device="cuda")
+    labK = torch.zeros((1, w.N), dtype=torch.int32, device="cuda")
+    labK[0, 5] = w.C_k + 3
+    plan = N.Plan(N.params_from_dict(w.params()), Q, K, V, labels=(labQ, labK))
+    assert plan.check() & 16

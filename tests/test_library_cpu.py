@@ -1,0 +1,99 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every entry point
+include/sparsepr.h declares, and validates arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from free_block_sparse_plan_b200 import native as N
+from free_block_sparse_plan_b200 import workloads as W
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    import __graft_entry__
+    __graft_entry__.build()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "sparsepr.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:sparsepr_status|void|const char\*)\s+(sparsepr_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_functions()
+    assert len(declared) >= 14
+    lib = ctypes.CDLL(N._LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(N.SYMBOLS) == sorted(declared)
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(N.sparsepr_params) == 80
+    assert N.sparsepr_params.lam.offset == 48
+    assert N.sparsepr_params.seed.offset == 72
+
+
+def test_status_strings():
+    assert N.status_string(0) == "ok"
+    assert "argument" in N.status_string(1)
+    assert N.status_string(99) == "unknown status"
+
+
+def _params(**kw):
+    base = W.TINY.params()
+    base.update(kw)
+    return N.params_from_dict(base)
+
+
+def test_workspace_size_positive_and_monotone():
+    small = N.sparsepr_workspace_size(_params())
+    big = N.sparsepr_workspace_size(N.params_from_dict(W.HUNYUAN.params()))
+    assert 0 < small < big
+    assert big % 256 == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d", 60, N.SPARSEPR_ERR_SHAPE), ("d", 256, N.SPARSEPR_ERR_SHAPE),
+    ("dtype", 7, N.SPARSEPR_ERR_DTYPE), ("H", 0, N.SPARSEPR_ERR_SHAPE),
+    ("r_K", 0, N.SPARSEPR_ERR_ARG), ("r_Q", 65, N.SPARSEPR_ERR_ARG),
+    ("C_q", 2000, N.SPARSEPR_ERR_ARG), ("C_k", 0, N.SPARSEPR_ERR_ARG),
+    ("M", 0, N.SPARSEPR_ERR_ARG), ("M", 129, N.SPARSEPR_ERR_ARG),
+    ("r", 17, N.SPARSEPR_ERR_ARG), ("r", -1, N.SPARSEPR_ERR_ARG),
+    ("lam", -0.5, N.SPARSEPR_ERR_ARG), ("lam", float("nan"), N.SPARSEPR_ERR_ARG),
+    ("target_density", 1.5, N.SPARSEPR_ERR_ARG), ("target_density", 0.01, N.SPARSEPR_ERR_ARG),
+    ("kmeans_max_iter", 0, N.SPARSEPR_ERR_ARG), ("engine", 3, N.SPARSEPR_ERR_ARG),
+])
+def test_invalid_parameters_rejected_on_host(field, value, status):
+    p = _params()
+    setattr(p, field, value)
+    with pytest.raises(N.SparsePRError) as ei:
+        N.sparsepr_workspace_size(p)
+    assert ei.value.status == status
+    # the plan entry point rejects them before touching the (fake) device pointers
+    h = ctypes.c_void_p()
+    st = N.lib().sparsepr_plan(ctypes.byref(p), 256, 256, 256, 256, 1 << 40, None, ctypes.byref(h))
+    assert st == status and not h.value
+
+
+def test_plan_rejects_missing_or_small_workspace():
+    p = _params()
+    h = ctypes.c_void_p()
+    need = N.sparsepr_workspace_size(p)
+    L = N.lib()
+    assert L.sparsepr_plan(ctypes.byref(p), 256, 256, 256, None, need, None, ctypes.byref(h)) == N.SPARSEPR_ERR_WORKSPACE
+    assert L.sparsepr_plan(ctypes.byref(p), 256, 256, 256, 512 + 8, need, None, ctypes.byref(h)) == N.SPARSEPR_ERR_WORKSPACE
+    assert L.sparsepr_plan(ctypes.byref(p), 256, 256, 256, 512, need - 1, None, ctypes.byref(h)) == N.SPARSEPR_ERR_WORKSPACE
+    assert L.sparsepr_plan(ctypes.byref(p), None, 256, 256, 512, need, None, ctypes.byref(h)) == N.SPARSEPR_ERR_ARG
+
+
+def test_calls_out_of_order_or_null_are_rejected():
+    L = N.lib()
+    assert L.sparsepr_attend(None, None) == N.SPARSEPR_ERR_ARG
+    assert L.sparsepr_probe_fit(None, None) == N.SPARSEPR_ERR_ARG
+    assert L.sparsepr_correct(None, 256, None) == N.SPARSEPR_ERR_ARG
+    L.sparsepr_destroy(None)
