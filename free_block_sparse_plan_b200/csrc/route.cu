@@ -3,8 +3,10 @@
 //   query, key and value centroids; each query group keeps the shortest prefix of K/V
 //   groups ranked by decreasing score whose key-token count reaches the common budget
 //   beta = (rho* - M/N_q) N_k.  The score is a reading of the SVG-EAR value error score
-//   the paper names: l_ab = tau qbar_a.kbar_b + ln|G_b|, pi_ab = softmax_b(l_ab),
-//   ohat_a = sum_b pi_ab vbar_b, score_ab = pi_ab ||vbar_b - ohat_a||, in fp64.
+//   the paper names: the centroid estimate of the hard-drop residual (App. A.1) of
+//   omitting group b alone, l_ab = tau qbar_a.kbar_b + ln|G_b|, pi_ab = softmax_b(l_ab),
+//   ohat_a^(-b) = sum_{c != b} pi_ac vbar_c / (1 - pi_ab),
+//   score_ab = pi_ab ||vbar_b - ohat_a^(-b)||, in fp64.
 //   Permutation (review page step 3): Q, K, V copied into group-major order.
 //   Probes (App. A.2, Algorithm A.1): stratified radial round robin.
 #include <cmath>
@@ -14,10 +16,14 @@
 namespace spr {
 namespace {
 
+// Routing score of every (query group a, K/V group b) cell, fp64.  For b other than the
+// largest-mass group, vbar_b - ohat^(-b) = (vbar_b - ohat) / (1 - pi_b) exactly, with
+// 1 - pi_b >= 1/2; for the largest-mass group ohat^(-b) is formed from the others.
 __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
-  __shared__ double qa[kMaxD], oh[kMaxD];
-  __shared__ double lg[kMaxC];
+  __shared__ double qa[kMaxD], oh[kMaxD], orest[kMaxD];
+  __shared__ double zz[kMaxC], zr[kMaxC];
   __shared__ double red[32];
+  __shared__ int redi[32];
   const int h = blockIdx.y, a = blockIdx.x, d = m.d;
   if (a >= b.nQ[h]) return;
   const int n = b.nK[h];
@@ -25,48 +31,77 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
   const double* kb = b.kbar + (long long)h * m.Ck * d;
   const double* vb = b.vbar + (long long)h * m.Ck * d;
   const int* sz = b.sizeK + (long long)h * m.Ck;
+  double* out = b.scores + ((long long)h * m.Cq + a) * m.Ck;
+  if (n == 1) {
+    if (threadIdx.x == 0) out[0] = 0.0;
+    return;
+  }
   for (int j = threadIdx.x; j < d; j += blockDim.x) qa[j] = b.qbar[((long long)h * m.Cq + a) * d + j];
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int k = warp; k < n; k += nw) {
+  for (int k = warp; k < n; k += nw) {      // logits, kept in zr for now
     double s = 0.0;
     for (int j = lane; j < d; j += 32) s += qa[j] * kb[(long long)k * d + j];
     s = warp_sum(s);
-    if (lane == 0) lg[k] = tau * s + log((double)sz[k]);
+    if (lane == 0) zr[k] = tau * s + log((double)sz[k]);
   }
   __syncthreads();
+  // largest logit and its first index; then the largest among the others
   double mx = -INFINITY;
-  for (int k = threadIdx.x; k < n; k += blockDim.x) mx = fmax(mx, lg[k]);
-  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[warp] = mx;
+  int top = 0x7fffffff;
+  for (int k = threadIdx.x; k < n; k += blockDim.x)
+    if (zr[k] > mx || (zr[k] == mx && k < top)) { mx = zr[k]; top = k; }
+  for (int o = 16; o > 0; o >>= 1) {
+    const double om = __shfl_xor_sync(0xffffffffu, mx, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, top, o);
+    if (om > mx || (om == mx && oi < top)) { mx = om; top = oi; }
+  }
+  if (lane == 0) { red[warp] = mx; redi[warp] = top; }
   __syncthreads();
   mx = red[0];
-  for (int w = 1; w < nw; ++w) mx = fmax(mx, red[w]);
+  top = redi[0];
+  for (int w = 1; w < nw; ++w)
+    if (red[w] > mx || (red[w] == mx && redi[w] < top)) { mx = red[w]; top = redi[w]; }
   __syncthreads();
-  double part = 0.0;
+  double m2 = -INFINITY;
+  for (int k = threadIdx.x; k < n; k += blockDim.x)
+    if (k != top) m2 = fmax(m2, zr[k]);
+  for (int o = 16; o > 0; o >>= 1) m2 = fmax(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  if (lane == 0) red[warp] = m2;
+  __syncthreads();
+  m2 = red[0];
+  for (int w = 1; w < nw; ++w) m2 = fmax(m2, red[w]);
+  __syncthreads();
+  double pz = 0.0, pr = 0.0;
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
-    const double e = exp(lg[k] - mx);
-    lg[k] = e;
-    part += e;
+    const double l = zr[k];
+    zz[k] = exp(l - mx);
+    zr[k] = (k == top) ? 0.0 : exp(l - m2);
+    pz += zz[k];
+    pr += zr[k];
   }
-  const double tot = block_sum(part, red);
-  for (int k = threadIdx.x; k < n; k += blockDim.x) lg[k] /= tot;
-  __syncthreads();
+  const double Z = block_sum(pz, red);
+  const double Zr = block_sum(pr, red);
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    double s = 0.0;
-    for (int k = 0; k < n; ++k) s += lg[k] * vb[(long long)k * d + j];
-    oh[j] = s;
+    double s = 0.0, t = 0.0;
+    for (int k = 0; k < n; ++k) {
+      const double v = vb[(long long)k * d + j];
+      s += zz[k] * v;
+      t += zr[k] * v;
+    }
+    oh[j] = s / Z;
+    orest[j] = t / Zr;
   }
   __syncthreads();
-  double* out = b.scores + ((long long)h * m.Cq + a) * m.Ck;
   for (int k = warp; k < n; k += nw) {
+    const double* ref = (k == top) ? orest : oh;
     double s = 0.0;
     for (int j = lane; j < d; j += 32) {
-      const double t = vb[(long long)k * d + j] - oh[j];
+      const double t = vb[(long long)k * d + j] - ref[j];
       s += t * t;
     }
     s = warp_sum(s);
-    if (lane == 0) out[k] = lg[k] * sqrt(s);
+    if (lane == 0) out[k] = (k == top) ? (zz[k] / Z) * sqrt(s) : zz[k] * sqrt(s) / (Z - zz[k]);
   }
 }
 

@@ -27,9 +27,11 @@ Readings where the pages are silent (each is listed in the design doc):
   S7  k-means stops after max_iter assignment steps or when an assignment changes no label
   S8  k-means init: C rows drawn with replacement by SplitMix64 (counter-based)
   S9  phi_Q = z / max(rms(z), 1e-6)
-  S11 routing score (the SVG-EAR value-error score is not on the pages):
+  S11 routing score (the SVG-EAR value error score is not on the pages): the centroid
+      estimate of the hard-drop residual of omitting K/V group b alone,
       l_ab = tau qbar_a.kbar_b + ln|G_b|, pi_ab = softmax_b l_ab,
-      ohat_a = sum_b pi_ab vbar_b, score_ab = pi_ab * ||vbar_b - ohat_a||_2
+      ohat_a^(-b) = sum_{c != b} pi_ac vbar_c / (1 - pi_ab),
+      score_ab = pi_ab * ||vbar_b - ohat_a^(-b)||_2
   S12 score ties ranked by ascending KV group id
   S14 group-major order keeps ascending original index inside a group
   S16 probe distance d_i is the squared distance to the group centre in phi_Q space
@@ -222,19 +224,34 @@ def route_scores(qbar: np.ndarray, kbar: np.ndarray, vbar: np.ndarray,
                  size_b: np.ndarray, d: int) -> np.ndarray:
     """S11 (reading; the SVG-EAR formula is not on the pages; parity unpinned against it).
 
-    Centroid estimate of how much dropping KV group b moves query group a's output:
-    the estimated attention mass of b times the distance of b's value centroid from
-    the estimated output, following the hard-drop identity of [P] App. A.1.
+    Centroid estimate of the residual left by omitting K/V group b alone from query group
+    a: by the hard-drop identity of [P] App. A.1 with U = {b}, ||R|| = p_b ||O_b - O_sp||,
+    estimated with pi_ab = softmax_b(tau qbar_a.kbar_b + ln|G_b|) for p_b, vbar_b for O_b
+    and ohat_a^(-b) = sum_{c != b} pi_ac vbar_c / (1 - pi_ab) for O_sp:
+        score_ab = pi_ab * ||vbar_b - ohat_a^(-b)||.
+    For every b but the largest-mass one, vbar_b - ohat^(-b) = (vbar_b - ohat)/(1 - pi_b)
+    exactly, with ohat the estimate over all groups and 1 - pi_b >= 1/2; for the largest-
+    mass group ohat^(-b) is formed directly from the other groups.  One group: score 0.
     """
     tau = 1.0 / math.sqrt(d)
-    logits = tau * (qbar @ kbar.T) + np.log(size_b.astype(np.float64))[None, :]
-    logits -= logits.max(axis=1, keepdims=True)
-    pi = np.exp(logits)
-    pi /= pi.sum(axis=1, keepdims=True)
-    ohat = pi @ vbar
-    S = np.empty_like(pi)
-    for a in range(pi.shape[0]):
-        S[a] = pi[a] * np.sqrt(((vbar - ohat[a][None, :]) ** 2).sum(axis=1))
+    L = tau * (qbar @ kbar.T) + np.log(size_b.astype(np.float64))[None, :]
+    n = L.shape[1]
+    S = np.zeros_like(L)
+    if n == 1:
+        return S
+    for a in range(L.shape[0]):
+        l = L[a]
+        top = int(np.argmax(l))                      # first index of the maximum
+        z = np.exp(l - l[top])
+        Z = z.sum()
+        ohat = (z @ vbar) / Z
+        rest = Z - z
+        rest[top] = 1.0                              # replaced below
+        S[a] = z * np.sqrt(((vbar - ohat[None, :]) ** 2).sum(axis=1)) / rest
+        others = np.arange(n) != top
+        zo = np.exp(l[others] - l[others].max())
+        ohat_rest = (zo @ vbar[others]) / zo.sum()
+        S[a, top] = (z[top] / Z) * np.linalg.norm(vbar[top] - ohat_rest)
     return S
 
 

@@ -209,20 +209,43 @@ def test_route_score_hand_worked():
 
 def test_route_score_singletons_match_hard_drop_of_one_key():
     # With one key per group and the query at its centroid, pi is the exact attention and
-    # the score equals (1 - pi_b) * || O_dense - O_sp(without b) || (App. A.1 identity).
+    # the score equals || O_dense - O_sp(without b) || (App. A.1 identity, U = {b}).
     rng = _rng(8)
     d = 4
-    q = rng.standard_normal((1, d))
+    q = rng.standard_normal((1, d)) * 3
     K = rng.standard_normal((6, d))
     V = rng.standard_normal((6, d))
     S = O.route_scores(q, K, V, np.ones(6, dtype=np.int64), d)[0]
     dense = O.attention_rows(q, K, V)[0]
-    z = np.exp(q @ K.T / math.sqrt(d))[0]
-    pi = z / z.sum()
     for b in range(6):
         keep = [j for j in range(6) if j != b]
         osp = O.attention_rows(q, K[keep], V[keep])[0]
-        assert abs(S[b] - (1 - pi[b]) * np.linalg.norm(dense - osp)) < 1e-12
+        assert abs(S[b] - np.linalg.norm(dense - osp)) < 1e-12
+
+
+def test_route_score_matches_definition_by_brute_force():
+    # ohat^(-b) formed literally from the other groups for every b, including a group
+    # holding nearly all the mass (where the closed form would cancel).
+    rng = _rng(81)
+    C, d = 7, 5
+    kbar = rng.standard_normal((C, d))
+    kbar[3] *= 12.0
+    qbar = np.vstack([kbar[3] * 2.0, rng.standard_normal(d)])
+    vbar = rng.standard_normal((C, d))
+    sizes = rng.integers(1, 50, C)
+    S = O.route_scores(qbar, kbar, vbar, sizes, d)
+    for a in range(2):
+        l = [float(qbar[a] @ kbar[b]) / math.sqrt(d) + math.log(sizes[b]) for b in range(C)]
+        mx = max(l)
+        z = [math.exp(x - mx) for x in l]
+        for b in range(C):
+            pb = z[b] / sum(z)
+            zo = [(c, math.exp(l[c] - max(l[cc] for cc in range(C) if cc != b))) for c in range(C) if c != b]
+            tot = sum(x for _, x in zo)
+            orest = sum(x * vbar[c] for c, x in zo) / tot
+            want = pb * float(np.linalg.norm(vbar[b] - orest))
+            assert abs(S[a, b] - want) <= 1e-12 * max(want, 1e-300) + 1e-300, (a, b, S[a, b], want)
+    assert S[0, 3] > 0.1 and np.argmax(S[0]) == 3    # the dominant group ranks first
 
 
 def test_select_cells_hand_worked():
