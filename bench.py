@@ -166,6 +166,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="mid")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling cases)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -175,6 +176,8 @@ def main():
 
     from free_block_sparse_plan_b200 import workloads as W
     w = W.get(args.workload)
+    if args.heads:
+        w = w.with_(H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
         return

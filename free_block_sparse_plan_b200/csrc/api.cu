@@ -132,6 +132,8 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->reff = c.take<int>(H);
   b->Bp = c.take<float>(H * d * d);
   b->cvec = c.take<float>(H * d);
+  b->work = c.take<int>(H * (size_t)tc_max_items(m));
+  b->nwork = c.take<int>(H);
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);
 }

@@ -279,9 +279,9 @@ sparsepr_status launch_sparse_attention_simt(const Plan& p, cudaStream_t st) {
   });
 }
 
-sparsepr_status launch_probe_attention(const Plan& p, cudaStream_t st) {
+sparsepr_status launch_probe_attention_simt(const Plan& p, cudaStream_t st) {
   const Dims& m = p.dm;
-  sparsepr_status s = with_d(m.d, [&](auto DD) -> sparsepr_status {
+  return with_d(m.d, [&](auto DD) -> sparsepr_status {
     constexpr int D = decltype(DD)::value;
     const size_t smem = 2 * kKeys * D * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(probe_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -289,8 +289,10 @@ sparsepr_status launch_probe_attention(const Plan& p, cudaStream_t st) {
     SPR_LAUNCH_OK();
     return SPARSEPR_OK;
   });
-  if (s != SPARSEPR_OK) return s;
-  probe_combine_kernel<<<dim3(m.M, m.H), kMaxD, 0, st>>>(m, p.b);
+}
+
+sparsepr_status launch_probe_combine(const Plan& p, cudaStream_t st) {
+  probe_combine_kernel<<<dim3(p.dm.M, p.dm.H), kMaxD, 0, st>>>(p.dm, p.b);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -307,13 +309,24 @@ sparsepr_status launch_dense_attention_simt(const Dims& m, const void* Q, const 
   });
 }
 
-// Engine choice: the tensor-core engine is not built yet, so every dtype runs here.
+// Engine choice: the tensor-core engine for bf16 with d in {64, 128} unless the CUDA-core
+// engine is requested; the CUDA-core engine for everything else.
 sparsepr_status launch_sparse_attention(const Plan& p, cudaStream_t st) {
+  if (tc_engine_applies(p.dm.dtype, p.dm.d, p.dm.engine)) return launch_sparse_attention_tc(p, st);
   return launch_sparse_attention_simt(p, st);
+}
+
+sparsepr_status launch_probe_attention(const Plan& p, cudaStream_t st) {
+  sparsepr_status s = tc_engine_applies(p.dm.dtype, p.dm.d, p.dm.engine)
+                          ? launch_probe_attention_tc(p, st)
+                          : launch_probe_attention_simt(p, st);
+  if (s != SPARSEPR_OK) return s;
+  return launch_probe_combine(p, st);
 }
 
 sparsepr_status launch_dense_attention(const Dims& m, const void* Q, const void* K, const void* V,
                                        void* Out, cudaStream_t st) {
+  if (tc_engine_applies(m.dtype, m.d, m.engine)) return launch_dense_attention_tc(m, Q, K, V, Out, nullptr, st);
   return launch_dense_attention_simt(m, Q, K, V, Out, st);
 }
 

@@ -24,6 +24,7 @@ enum : int {
   kErrNonFinite = 4,   // a non-finite value reached the fit
   kErrProbe = 8,       // probe selection could not find M rows
   kErrLabels = 16,     // an injected label was outside [0, C)
+  kErrHang = 32,       // a pipeline wait timed out (the kernel abandoned its work)
 };
 
 // Problem dimensions, passed by value to kernels.
@@ -73,6 +74,7 @@ struct Buffers {
   double *sig;               // [H][kMaxM]
   int *reff;                 // [H]
   float *Bp, *cvec;          // folded correction [H][d][d], [H][d]
+  int *work, *nwork;         // tensor-core attention work list [H][max items], [H]
   int *err;                  // device error word
 };
 
@@ -194,6 +196,14 @@ sparsepr_status launch_correct(const Plan& p, void* Out, cudaStream_t st);
 sparsepr_status launch_sparse_attention_simt(const Plan& p, cudaStream_t st);
 sparsepr_status launch_dense_attention_simt(const Dims& dm, const void* Q, const void* K,
                                             const void* V, void* Out, cudaStream_t st);
+bool tc_engine_applies(int dtype, int d, int engine);
+int tc_max_items(const Dims& m);
+sparsepr_status launch_sparse_attention_tc(const Plan& p, cudaStream_t st);
+sparsepr_status launch_probe_attention_tc(const Plan& p, cudaStream_t st);
+sparsepr_status launch_probe_attention_simt(const Plan& p, cudaStream_t st);
+sparsepr_status launch_probe_combine(const Plan& p, cudaStream_t st);
+sparsepr_status launch_dense_attention_tc(const Dims& m, const void* Q, const void* K, const void* V,
+                                          void* Out, int* err, cudaStream_t st);
 sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void* K,
                                        const void* V, void* Out, cudaStream_t st);
 

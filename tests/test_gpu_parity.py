@@ -36,7 +36,7 @@ def _cuda():
 
 def oracle_head(w: W.Workload, h: int, rows=None):
     """Oracle call for head h of workload w (cached partition per head)."""
-    key = (w.name, w.seed, h)
+    key = (w, h)
     p = O.Params.from_dict(w.params())
     if key not in _oracle_cache:
         q, k, v = W.make_head(w, h)
@@ -252,7 +252,7 @@ def test_hunyuan_full_size_sampled_heads():
 def test_operating_point_sweep_head0():
     base = W.WAN
     q, k, v, _ = oracle_head(base, 0, rows=np.arange(4))
-    part = _oracle_cache[(base.name, base.seed, 0)][3]
+    part = _oracle_cache[(base, 0)][3]
     dt = torch.bfloat16
     Q, K, V = (torch.from_numpy(x.astype(np.float32))[None].to(dt).cuda() for x in (q, k, v))
     labQ = torch.tensor(part.km_Q.labels[None], dtype=torch.int32, device="cuda")
@@ -287,10 +287,10 @@ def test_full_density_returns_dense():
     assert rel(out[1].float().cpu().numpy()[rows], ref) < 1e-2
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_dense_attention_engine_ragged(dtype):
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 64), ("bf16", 128)])
+def test_dense_attention_engine_ragged(dtype, d):
     rng = np.random.default_rng(5)
-    H, Nq, Nk, d = 2, 333, 517, 64
+    H, Nq, Nk = 2, 333, 517
     arrs = [rng.standard_normal((H, n, d)) * s for n, s in ((Nq, 0.7), (Nk, 0.7), (Nk, 1.0))]
     if dtype == "bf16":
         arrs = [W.round_to_bf16(a) for a in arrs]
@@ -300,6 +300,24 @@ def test_dense_attention_engine_ragged(dtype):
     for h in range(H):
         ref = O.dense_attention(arrs[0][h], arrs[1][h], arrs[2][h])
         assert rel(out[h], ref) < (1e-5 if dtype == "f32" else 1e-2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_tensor_core_engine_matches_cuda_core_engine(d):
+    # Same plan (oracle labels injected), attention by both engines: the sparse outputs
+    # agree to bf16 rounding of the probabilities, the corrected outputs to the tolerance.
+    w = (W.MID if d == 64 else W.WAN.with_(N=16800, grid=(21, 20, 40), C_q=128, C_k=128)).with_(H=2)
+    inputs = W.make_inputs_torch(w, device="cuda")
+    ref = [oracle_head(w, h)[3] for h in range(w.H)]
+    labQ = torch.tensor(np.stack([r.part.km_Q.labels for r in ref]), dtype=torch.int32, device="cuda")
+    labK = torch.tensor(np.stack([r.part.km_K.labels for r in ref]), dtype=torch.int32, device="cuda")
+    p_tc, o_tc, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK))
+    p_ct, o_ct, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK), engine=N.SPARSEPR_ENGINE_SIMT)
+    assert p_tc.check() == 0 and p_ct.check() == 0
+    assert rel(p_tc.export("OSP"), p_ct.export("OSP")) < 5e-3
+    assert rel(p_tc.export("ODENSE_PROBE"), p_ct.export("ODENSE_PROBE")) < 5e-3
+    for h, r in enumerate(ref):
+        check_injected_head(p_tc, o_tc[h].float().cpu().numpy(), r, h, w)
 
 
 def test_ragged_cross_attention_and_empty_groups():
