@@ -14,7 +14,7 @@ constexpr int kMaxD = 128;      // head dimension limit
 constexpr int kMaxC = 1024;     // requested group count limit
 constexpr int kMaxR = 64;       // response-coordinate rank limit
 constexpr int kMaxM = 128;      // probe count limit
-constexpr int kSortChunk = 256; // rows per block of the stable counting sort
+constexpr int kSortChunk = 1024; // rows per block of the stable counting sort
 constexpr int kProbeSplit = 4096;  // keys per partial of the exact probe attention
 
 // Device error word bits.
@@ -52,6 +52,10 @@ struct Buffers {
   int *kmK, *kmQ;            // per-head k-means state [H][4]: done, changed, iters, -
   double *objK, *objQ;       // per-cluster objective partials [H][C]
   double *objH;              // [H][2] final objectives
+  float *ubK, *lbK, *ubQ, *lbQ;  // k-means exact squared distances: own / best other [H][N]
+  int *movedfK, *movedfQ;    // centre changed in the last update [H][C]
+  int *movedK, *movedQ;      // moved centre ids [H][C]
+  int *nmovedK, *nmovedQ;    // moved centre counts [H]
   int *compK, *compQ;        // raw label -> compact id (-1 if empty) [H][C]
   int *usedK, *usedQ;        // compact id -> raw label [H][C]
   int *nK, *nQ;              // [H] non-empty group counts

@@ -57,12 +57,18 @@ __global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const v
 // ---------------------------------------------------------------------------------
 // One-sided Jacobi: orthogonalise the `ncols` columns (length `rows`, column-major with
 // stride `rows`) of G in shared memory.  Parallel round-robin ordering: in each round
-// the column pairs are disjoint, one warp per pair.  Bounded sweeps.
-__device__ void hestenes(double* G, int rows, int ncols, int* flag) {
+// the column pairs are disjoint, one warp per pair.  A pair counts as orthogonal when
+// |a.b| <= 1e-14 |a||b| or |a.b| <= 1e-15 ||G||_F^2: the second (absolute) test ends the
+// sweeps when only columns near the null space still carry rounding-level overlap, which
+// no relative test can remove.  Bounded sweeps.
+__device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  double f = 0.0;
+  for (int e = threadIdx.x; e < rows * ncols; e += blockDim.x) f += G[e] * G[e];
+  const double abs_tol = 1e-15 * block_sum(f, red);
   const int nn = ncols + (ncols & 1);   // pad to even with a phantom column
   const int npairs = nn / 2;
-  for (int sweep = 0; sweep < 40; ++sweep) {
+  for (int sweep = 0; sweep < 30; ++sweep) {
     if (threadIdx.x == 0) *flag = 0;
     __syncthreads();
     for (int round = 0; round < nn - 1; ++round) {
@@ -84,7 +90,7 @@ __device__ void hestenes(double* G, int rows, int ncols, int* flag) {
         al = warp_sum(al);
         be = warp_sum(be);
         ga = warp_sum(ga);
-        if (ga == 0.0 || fabs(ga) <= 1e-15 * sqrt(al * be)) continue;
+        if (ga == 0.0 || fabs(ga) <= 1e-14 * sqrt(al * be) || fabs(ga) <= abs_tol) continue;
         const double zeta = (be - al) / (2.0 * ga);
         const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
         const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
@@ -112,8 +118,7 @@ __device__ __forceinline__ int desc_rank(const double* key, int n, int j) {
 }
 
 // Eigen-weighted factor of a symmetric PSD metric (paper S4.1, App. B.1):
-// F = [u_1 sqrt(l_1/mean) ... u_r sqrt(l_r/mean)], mean over the r kept eigenvalues
-// (negative eigenvalues clamped to zero).
+// F = [u_1 sqrt(l_1/mean) ... u_r sqrt(l_r/mean)], mean over the r kept eigenvalues.
 __global__ void __launch_bounds__(kLinThreads) eigen_factor_kernel(Dims m, const double* Mall,
                                                                    int r, double* lam_out,
                                                                    double* F64, float* F32,
@@ -126,28 +131,19 @@ __global__ void __launch_bounds__(kLinThreads) eigen_factor_kernel(Dims m, const
   const double* Mh = Mall + (long long)h * d * d;
   for (int e = threadIdx.x; e < d * d; e += blockDim.x) G[e] = Mh[e];  // symmetric
   __syncthreads();
-  hestenes(G, d, d, &flag);
-  // column norms = |eigenvalues|; the sign comes from the Rayleigh quotient
+  hestenes(G, d, d, &flag, red);
+  // The metrics are Gram matrices (symmetric PSD), so the converged column norms are the
+  // eigenvalues; negative eigenvalues exist only at rounding level, where |lambda| and
+  // the clamp to zero differ by far less than any distance that decides a label.
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int j = warp; j < d; j += nwarps) {
     double s = 0.0;
     for (int i = lane; i < d; i += 32) s += G[j * d + i] * G[j * d + i];
     s = warp_sum(s);
-    if (lane == 0) norm[j] = sqrt(s);
-  }
-  __syncthreads();
-  for (int j = warp; j < d; j += nwarps) {
-    const double nj = norm[j];
-    double rq = 0.0;   // u^T M u * |lambda|^2 (sign only)
-    if (nj > 0.0) {
-      for (int i = lane; i < d; i += 32) {
-        double mu = 0.0;
-        for (int k = 0; k < d; ++k) mu += Mh[i * d + k] * G[j * d + k];
-        rq += G[j * d + i] * mu;
-      }
-      rq = warp_sum(rq);
+    if (lane == 0) {
+      norm[j] = sqrt(s);
+      lam[j] = norm[j];
     }
-    if (lane == 0) lam[j] = (nj > 0.0 && rq > 0.0) ? nj : 0.0;
   }
   __syncthreads();
   for (int j = threadIdx.x; j < d; j += blockDim.x) rank[j] = desc_rank(lam, d, j);
@@ -323,7 +319,7 @@ __global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
   } else {
     for (int e = threadIdx.x; e < M * d; e += blockDim.x) S[e] = Y[e];
     __syncthreads();
-    hestenes(S, d, M, &flag);
+    hestenes(S, d, M, &flag, red);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     for (int p = warp; p < M; p += nwarps) {
       double s2 = 0.0;
