@@ -92,16 +92,6 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->objK = c.take<double>(H * Ck);
   b->objQ = c.take<double>(H * Cq);
   b->objH = c.take<double>(H * 2);
-  b->ubK = c.take<float>(H * Nk);
-  b->lbK = c.take<float>(H * Nk);
-  b->ubQ = c.take<float>(H * Nq);
-  b->lbQ = c.take<float>(H * Nq);
-  b->movedfK = c.take<int>(H * Ck);
-  b->movedfQ = c.take<int>(H * Cq);
-  b->movedK = c.take<int>(H * Ck);
-  b->movedQ = c.take<int>(H * Cq);
-  b->nmovedK = c.take<int>(H);
-  b->nmovedQ = c.take<int>(H);
   b->compK = c.take<int>(H * Ck);
   b->compQ = c.take<int>(H * Cq);
   b->usedK = c.take<int>(H * Ck);

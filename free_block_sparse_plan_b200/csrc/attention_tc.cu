@@ -1,27 +1,33 @@
 // Attention on the 5th-generation tensor cores (tcgen05 + TMEM), bf16 in, fp32 accumulate.
 //
-// One CTA computes a 128-row query tile against a key sequence in 128-key tiles:
+// One CTA computes up to two 128-row query tiles (A, B) against one key sequence in
+// 128-key tiles:
 //   sparse  rows of one query group (group-major) against the concatenated key ranges of
 //           the K/V groups selected for it: renormalised hard drop (paper S2);
-//   dense   128 consecutive rows against all keys (the dense baseline, same engine);
+//   dense   256 consecutive rows against all keys (the dense baseline, same engine);
 //   probe   the M probe rows against one chunk of keys, written as partial
 //           (max, sum, numerator) for a later combine (paper S4.2, App. A.2).
 //
-// Warp roles (288 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r; reads S rows from TMEM,
-//              online softmax in base 2, writes P (bf16) to shared memory, rescales the
-//              O accumulator row in TMEM when the running max grows, final epilogue;
-//   warps 4-7  producers: 16-byte cp.async gathers of the Q tile and of each K/V tile
-//              (arbitrary key rows: the selected groups need not be contiguous) into
-//              128-byte-swizzled shared memory, two stages;
-//   warp 8     one thread issues tcgen05.mma: S_j = Q K_j^T into one of two TMEM S
-//              buffers, O += P_j V_j into the TMEM accumulator (V read MN-major), with
-//              tcgen05.commit arriving on mbarriers.  The warp owns the TMEM allocation.
-// Issue order S_0, S_1, PV_0, S_2, PV_1, ... keeps the tensor cores busy with S_{j+1}
-// while the softmax warps work on tile j.
+// Warp roles (384 threads; twelve warps so each SM sub-partition holds three):
+//   warps 0-3, 4-7  softmax of tile A, of tile B: thread r owns query row r = TMEM lane r;
+//              reads its S row from TMEM, online softmax in base 2 with lazy rescaling
+//              (O is rescaled only when the row max grows by more than 2^8), writes P as
+//              bf16 pairs into the TMEM columns of S already read, epilogue;
+//   warps 8-10 producers: 16-byte cp.async gathers of the Q tiles and of each K/V tile
+//              (arbitrary key rows, so the selected groups need not be contiguous) into
+//              128-byte-swizzled shared memory, two stages shared by both query tiles;
+//   warp 11    one thread issues tcgen05.mma: S_t = Q_t K_j^T (both operands in shared
+//              memory) and O_t += P_t V_j (P read from TMEM, V MN-major), and commits to
+//              mbarriers.  The warp owns the TMEM allocation: S_A, S_B (128 columns each),
+//              O_A, O_B (128 each).
+// Issue order per key tile: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): the softmax of one tile
+// overlaps the matrix products of the other.  tcgen05.commit arrives only when every
+// earlier tcgen05 operation of the thread is complete, so "S_t(j) ready" also certifies
+// that PV_t(j-1) has finished reading P_t and updating O_t.
 //
 // Every mbarrier wait is bounded: on timeout the CTA records kErrHang, all roles stop,
 // the MMA thread drains its outstanding MMAs and the TMEM is freed before returning.
+// Warp-collective TMEM loads/stores sit only in warp-uniform control flow.
 #include <cmath>
 
 #include "common.cuh"
@@ -32,8 +38,11 @@ namespace {
 
 constexpr int kTileRows = 128;
 constexpr int kTileKeys = 128;
-constexpr int kTcThreads = 288;
+constexpr int kItemRows = 2 * kTileRows;
+constexpr int kTcThreads = 384;
+constexpr int kProducers = 96;                   // warps 8-10
 constexpr long long kWaitCycles = 2000000000LL;   // about one second: a hung pipeline
+constexpr float kRescaleLog2 = 8.0f;              // lazy rescale threshold (factor 256)
 
 enum Mode { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
@@ -47,7 +56,7 @@ struct TcArgs {
   const __nv_bfloat16* K;
   const __nv_bfloat16* V;
   Buffers b;
-  const int* work;     // sparse: [H][max_items] (a << 16 | tile)
+  const int* work;     // sparse: [H][max_items] (a << 16 | item)
   const int* nwork;    // sparse: [H]
   int max_items;
   void* out;           // dense: output in the input dtype
@@ -58,17 +67,16 @@ template <int D>
 struct Layout {
   static constexpr uint32_t kTile = kTileRows * D * 2;         // bytes of a Q/K/V tile
   static constexpr uint32_t kPanel = kTileRows * 128;          // one 64-column panel
-  static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK0 = kTile, oK1 = 2 * kTile;
-  static constexpr uint32_t oV0 = 3 * kTile, oV1 = 4 * kTile;
-  static constexpr uint32_t oP = 5 * kTile;                    // 128 x 128 bf16 = 32 KB
-  static constexpr uint32_t oMisc = oP + 2 * kPanel;
-  static constexpr uint32_t kBytes = oMisc + 12 * 1024;
+  static constexpr uint32_t oQ0 = 0, oQ1 = kTile;
+  static constexpr uint32_t oK0 = 2 * kTile, oK1 = 3 * kTile;
+  static constexpr uint32_t oV0 = 4 * kTile, oV1 = 5 * kTile;
+  static constexpr uint32_t oMisc = 6 * kTile;
+  static constexpr uint32_t kBytes = oMisc + 14 * 1024;
 };
 
 struct Misc {
   unsigned long long bars[16];
-  long long qrow[kTileRows];
+  long long qrow[kItemRows];
   long long krow[2][kTileKeys];
   int csum[kMaxC + 1];
   int cbase[kMaxC];
@@ -77,7 +85,9 @@ struct Misc {
   int sh[32];
 };
 
-enum Bar { bQFull = 0, bFull0 = 1, bEmpty0 = 3, bSFull0 = 5, bSFree0 = 7, bPFull = 9, bPvDone = 10, bDrain = 11 };
+enum Bar {
+  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 3, bSFull0 = 5, bPFull0 = 7, bPvDone0 = 9, bDrain = 11
+};
 
 __device__ __forceinline__ bool wait_bar(Misc* ms, uint32_t bar, uint32_t parity, int* err) {
   if (tc::mbar_try_wait(bar, parity)) return true;
@@ -115,8 +125,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     const int labq = g.b.usedQ[(long long)h * m.Cq + a];
     const int gs = g.b.offQ[(long long)h * (m.Cq + 1) + labq];
     const int ge = g.b.offQ[(long long)h * (m.Cq + 1) + labq + 1];
-    q0 = gs + t * kTileRows;
-    nrows = min(kTileRows, ge - q0);
+    q0 = gs + t * kItemRows;
+    nrows = min(kItemRows, ge - q0);
     cnt = g.b.cellCnt[(long long)h * m.Cq + a];
     const int* ids = g.b.cellIds + ((long long)h * m.Cq + a) * m.Ck;
     for (int base_i = 0; base_i < cnt; base_i += blockDim.x) {
@@ -140,8 +150,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     }
     nkeys = ms->csum[cnt];
   } else if (g.mode == kModeDense) {
-    q0 = blockIdx.x * kTileRows;
-    nrows = min(kTileRows, m.Nq - q0);
+    q0 = blockIdx.x * kItemRows;
+    nrows = min(kItemRows, m.Nq - q0);
     nkeys = m.Nk;
   } else {
     split = blockIdx.x;
@@ -151,24 +161,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   }
   const int nt = (int)((nkeys + kTileKeys - 1) / kTileKeys);
   const int last_valid = (int)(nkeys - (long long)(nt - 1) * kTileKeys);
+  const bool hasB = nrows > kTileRows;
 
   // ---------------------------------------------------------------- setup
   const uint32_t bars = tc::smem_u32(ms->bars);
   auto BAR = [&](int i) -> uint32_t { return bars + 8u * i; };
   if (tid == 0) {
-    tc::mbar_init(BAR(bQFull), 128);
+    tc::mbar_init(BAR(bQFull), kProducers);
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(BAR(bFull0 + s), 128);
-      tc::mbar_init(BAR(bEmpty0 + s), 1);
+      tc::mbar_init(BAR(bKVFull0 + s), kProducers);
+      tc::mbar_init(BAR(bKVEmpty0 + s), 1);
       tc::mbar_init(BAR(bSFull0 + s), 1);
-      tc::mbar_init(BAR(bSFree0 + s), 128);
+      tc::mbar_init(BAR(bPFull0 + s), 128);
+      tc::mbar_init(BAR(bPvDone0 + s), 1);
     }
-    tc::mbar_init(BAR(bPFull), 128);
-    tc::mbar_init(BAR(bPvDone), 1);
     tc::mbar_init(BAR(bDrain), 1);
     ms->abort_flag = 0;
   }
-  if (warp == 8) {
+  if (warp == 11) {
     tc::tmem_alloc(tc::smem_u32(&ms->tmem_base), 512);
     tc::tmem_relinquish();
   }
@@ -176,29 +186,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = ms->tmem_base;
-  const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
 
-  const uint32_t sQ = base + L::oQ, sP = base + L::oP;
-  const uint32_t sK[2] = {base + L::oK0, base + L::oK1};
-  const uint32_t sV[2] = {base + L::oV0, base + L::oV1};
+  // tile addresses: Q tile t, K stage s, V stage s (consecutive tiles of kTile bytes)
+  auto sQ = [&](int t) -> uint32_t { return base + L::oQ0 + (uint32_t)t * L::kTile; };
+  auto sK = [&](int s) -> uint32_t { return base + L::oK0 + (uint32_t)s * L::kTile; };
+  auto sV = [&](int s) -> uint32_t { return base + L::oV0 + (uint32_t)s * L::kTile; };
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < 11) {
     // ============================================================ producers
-    const int p = tid - 128;
+    const int p = tid - 256;
     const long long hq = (long long)h * m.Nq * d, hk = (long long)h * m.Nk * d;
-    // query row p
-    long long qr = -1;
-    if (p < nrows) {
-      if (g.mode == kModeProbe) qr = hq + (long long)g.b.probes[(long long)h * m.M + p] * d;
-      else qr = hq + (long long)(q0 + p) * d;
+    for (int row = p; row < kItemRows; row += kProducers) {
+      long long qr = -1;
+      if (row < nrows) {
+        if (g.mode == kModeProbe) qr = hq + (long long)g.b.probes[(long long)h * m.M + row] * d;
+        else qr = hq + (long long)(q0 + row) * d;
+      }
+      ms->qrow[row] = qr;
     }
-    ms->qrow[p] = qr;
-    tc::named_sync(1, 128);
+    tc::named_sync(1, kProducers);
     constexpr int CPR = D / 8;                // 16-byte chunks per row
-    for (int e = p; e < kTileRows * CPR; e += 128) {
+    for (int e = p; e < kItemRows * CPR; e += kProducers) {
       const int row = e / CPR, c = e % CPR;
       const long long off = ms->qrow[row];
-      const uint32_t dst = sQ + (c >> 3) * L::kPanel + tc::sw128_offset(row, c & 7);
+      const uint32_t dst = sQ(row >> 7) + (c >> 3) * L::kPanel + tc::sw128_offset(row & 127, c & 7);
       tc::cp_async16(dst, off >= 0 ? (const void*)(g.Q + off + c * 8) : (const void*)g.Q, off >= 0 ? 16u : 0u);
     }
     tc::cp_async_commit();
@@ -208,9 +219,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
       // every producer thread takes the same decision (they meet at named barriers)
-      const bool got = j < 2 || wait_bar(ms, BAR(bEmpty0 + s), ((j >> 1) + 1) & 1, g.err);
-      if (!tc::named_sync_and(1, 128, got)) break;
-      const long long v = (long long)j * kTileKeys + p;
+      const bool got = j < 2 || wait_bar(ms, BAR(bKVEmpty0 + s), ((j >> 1) + 1) & 1, g.err);
+      if (!tc::named_sync_and(1, kProducers, got)) break;
+      for (int kk = p; kk < kTileKeys; kk += kProducers) {
+      const long long v = (long long)j * kTileKeys + kk;
       long long kr = -1;
       if (v < nkeys) {
         if (g.mode == kModeSparse) {
@@ -226,58 +238,71 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           kr = hk + ((long long)split * kProbeSplit + v) * d;
         }
       }
-      ms->krow[s][p] = kr;
-      tc::named_sync(1, 128);
-      for (int e = p; e < kTileKeys * CPR; e += 128) {
+      ms->krow[s][kk] = kr;
+      }
+      tc::named_sync(1, kProducers);
+      for (int e = p; e < kTileKeys * CPR; e += kProducers) {
         const int row = e / CPR, c = e % CPR;
         const long long off = ms->krow[s][row];
         const uint32_t o = (c >> 3) * L::kPanel + tc::sw128_offset(row, c & 7);
         const bool ok = off >= 0;
-        tc::cp_async16(sK[s] + o, ok ? (const void*)(g.K + off + c * 8) : (const void*)g.K, ok ? 16u : 0u);
-        tc::cp_async16(sV[s] + o, ok ? (const void*)(g.V + off + c * 8) : (const void*)g.V, ok ? 16u : 0u);
+        tc::cp_async16(sK(s) + o, ok ? (const void*)(g.K + off + c * 8) : (const void*)g.K, ok ? 16u : 0u);
+        tc::cp_async16(sV(s) + o, ok ? (const void*)(g.V + off + c * 8) : (const void*)g.V, ok ? 16u : 0u);
       }
       tc::cp_async_commit();
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
-      tc::mbar_arrive(BAR(bFull0 + s));
+      tc::mbar_arrive(BAR(bKVFull0 + s));
     }
     tc::cp_async_wait_all();
-  } else if (warp == 8) {
+  } else if (warp == 11) {
     // ============================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idQK = tc::idesc_bf16_f32(kTileRows, kTileKeys, false);
       constexpr uint32_t idPV = tc::idesc_bf16_f32(kTileRows, D, true);
-      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err);
-      auto issue_pv = [&](int j) -> bool {
-        if (!wait_bar(ms, BAR(bPFull), j & 1, g.err)) return false;
-        tc::fence_after_sync();
+      auto issue_s = [&](int t, int j) {
+        const int s = j & 1;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = tc::sw128_desc(sQ(t) + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(sK(s) + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
+          tc::mma_ss(tmem + 128 * t, ad, bd, idQK, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(BAR(bSFull0 + t));
+      };
+      auto issue_pv = [&](int t, int j) {
         const int s = j & 1;
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(sP + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(sV[s] + kk * 2048, L::kPanel, 1024);
-          tc::mma_ss(tO, ad, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = tc::sw128_desc(sV(s) + kk * 2048, L::kPanel, 1024);
+          tc::mma_ts(tmem + 256 + 128 * t, tmem + 128 * t + 8 * kk, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::mma_commit(BAR(bPvDone));
-        tc::mma_commit(BAR(bEmpty0 + s));
-        return true;
+        tc::mma_commit(BAR(bPvDone0 + t));
       };
-      for (int j = 0; ok && j < nt; ++j) {
-        const int s = j & 1;
-        if (!wait_bar(ms, BAR(bFull0 + s), (j >> 1) & 1, g.err)) { ok = false; break; }
-        if (j >= 2 && !wait_bar(ms, BAR(bSFree0 + s), ((j >> 1) + 1) & 1, g.err)) { ok = false; break; }
+      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && wait_bar(ms, BAR(bKVFull0), 0, g.err);
+      if (ok) {
         tc::fence_after_sync();
-        const uint32_t tS = s ? tS1 : tS0;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(sQ + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(sK[s] + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
-          tc::mma_ss(tS, ad, bd, idQK, kk > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(BAR(bSFull0 + s));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        issue_s(0, 0);
+        if (hasB) issue_s(1, 0);
       }
-      if (ok) issue_pv(nt - 1);
+      for (int j = 0; ok && j < nt; ++j) {
+        if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(0, j);
+        const bool more = j + 1 < nt;
+        if (more) {
+          if (!wait_bar(ms, BAR(bKVFull0 + ((j + 1) & 1)), ((j + 1) >> 1) & 1, g.err)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_s(0, j + 1);
+        }
+        if (hasB) {
+          if (!wait_bar(ms, BAR(bPFull0 + 1), j & 1, g.err)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_pv(1, j);
+        }
+        tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
+        if (hasB && more) issue_s(1, j + 1);
+      }
       tc::mma_commit(BAR(bDrain));
       // bounded: completes when every MMA issued above has finished
       const long long t0 = clock64();
@@ -286,20 +311,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8 && (warp < 4 || hasB)) {
     // ============================================================ softmax / epilogue
-    const int r = tid;                                  // query row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int t = warp >> 2;                            // query tile
+    const int r = tid - 128 * t;                        // its row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem + 128 * t + lane_off, tO = tmem + 256 + 128 * t + lane_off;
     const float sl2 = 1.4426950408889634f / sqrtf((float)d);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
-    // tcgen05.ld/st are warp-collective (.sync.aligned): every branch around them below
-    // is uniform across the warp, including the outcome of bounded waits.
     for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + s), (j >> 1) & 1, g.err))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + t), j & 1, g.err))) { ok = false; break; }
       tc::fence_after_sync();
-      const uint32_t tS = (s ? tS1 : tS0) + lane_off;
       const int valid = (j == nt - 1) ? last_valid : kTileKeys;
       float mx = -INFINITY;
 #pragma unroll
@@ -311,27 +334,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         for (int i = 0; i < 32; ++i)
           if (32 * c + i < valid) mx = fmaxf(mx, v[i]);
       }
-      const float m_new = fmaxf(m_run, mx * sl2);
-      // PV of the previous tile must be complete: P is reused and O is rescaled below
-      if (j >= 1) {
-        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone), (j - 1) & 1, g.err))) { ok = false; break; }
-        tc::fence_after_sync();
-      }
-      const float alpha = exp2f(m_run - m_new);         // 0 on the first tile, 1 if unchanged
-      if (j >= 1 && __any_sync(0xffffffffu, m_new > m_run)) {
+      const float m_tile = mx * sl2;
+      // lazy rescale: keep the running max unless it grows by more than 2^8
+      if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleLog2)) {
+        const float m_new = fmaxf(m_run, m_tile);
+        const float alpha = tc::ex2(m_run - m_new);     // 0 on the first tile
+        if (j > 0) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tc::tmem_ld32(tO + lane_off + 32 * c, o);
-          tc::tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc::tmem_ld32(tO + 32 * c, o);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tc::tmem_st32(tO + lane_off + 32 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tc::tmem_st32(tO + 32 * c, o);
+          }
         }
-        tc::tmem_wait_st();
+        l_run *= alpha;
+        m_run = m_new;
       }
       float rs = 0.0f;
-      uint8_t* prow = gbase + L::oP;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
@@ -340,55 +362,42 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = (32 * c + 2 * i < valid) ? exp2f(fmaf(v[2 * i], sl2, -m_new)) : 0.0f;
-          const float p1 = (32 * c + 2 * i + 1 < valid) ? exp2f(fmaf(v[2 * i + 1], sl2, -m_new)) : 0.0f;
+          const float p0 = (32 * c + 2 * i < valid) ? tc::ex2(fmaf(v[2 * i], sl2, -m_run)) : 0.0f;
+          const float p1 = (32 * c + 2 * i + 1 < valid) ? tc::ex2(fmaf(v[2 * i + 1], sl2, -m_run)) : 0.0f;
           rs += p0 + p1;
-          const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-          pk[i] = *reinterpret_cast<const uint32_t*>(&bb);
+          pk[i] = tc::pack_bf16x2(p0, p1);
         }
-        // columns 32c..32c+31 = four 16-byte chunks of panel (c >> 1)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
-          uint4* dst = reinterpret_cast<uint4*>(prow + (c >> 1) * L::kPanel + tc::sw128_offset(r, chunk));
-          *dst = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        // P columns 16c..16c+15 lie inside S columns already read (chunks 0..c)
+        tc::tmem_st16(tS + 16 * c, pk);
       }
+      tc::tmem_wait_st();
+      l_run += rs;
       tc::fence_before_sync();
-      tc::mbar_arrive(BAR(bSFree0 + s));
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      tc::fence_proxy_async();
-      tc::fence_before_sync();
-      tc::mbar_arrive(BAR(bPFull));
+      tc::mbar_arrive(BAR(bPFull0 + t));
     }
-    if (ok && __all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone), (nt - 1) & 1, g.err))) {
+    if (ok && __all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err))) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
+      const int row = kTileRows * t + r;
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tc::tmem_ld32(tO + lane_off + 32 * c, o);
+        tc::tmem_ld32(tO + 32 * c, o);
         tc::tmem_wait_ld();
-        if (r < nrows) {
+        if (row < nrows) {
           if (g.mode == kModeSparse) {
-            float4* dst = reinterpret_cast<float4*>(g.b.Osp + ((long long)h * m.Nq + q0 + r) * d + 32 * c);
+            float4* dst = reinterpret_cast<float4*>(g.b.Osp + ((long long)h * m.Nq + q0 + row) * d + 32 * c);
 #pragma unroll
             for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
           } else if (g.mode == kModeDense) {
-            const long long ob = ((long long)h * m.Nq + q0 + r) * d + 32 * c;
-            if (m.dtype == SPARSEPR_BF16) {
-              uint32_t pk[16];
+            const long long ob = ((long long)h * m.Nq + q0 + row) * d + 32 * c;
+            uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const __nv_bfloat162 bb = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
-                pk[i] = *reinterpret_cast<const uint32_t*>(&bb);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(g.out) + ob);
+            for (int i = 0; i < 16; ++i) pk[i] = tc::pack_bf16x2(o[2 * i] * inv, o[2 * i + 1] * inv);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(g.out) + ob);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            }
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           } else {
-            const long long slot = ((long long)h * m.M + r) * m.nsplit + split;
+            const long long slot = ((long long)h * m.M + row) * m.nsplit + split;
             float4* dst = reinterpret_cast<float4*>(g.b.Opart + slot * d + 32 * c);
 #pragma unroll
             for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
@@ -403,19 +412,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 11) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
 }
 
-// Work list of the sparse mode: one item per 128-row tile of every non-empty query group.
+// Work list of the sparse mode: one item per 256 rows (two query tiles) of every
+// non-empty query group.
 __global__ void __launch_bounds__(1024) build_work_kernel(Dims m, Buffers b, int* work, int* nwork,
                                                           int max_items) {
   __shared__ int sh[32];
   const int h = blockIdx.x, a = threadIdx.x;
   const int n = b.nQ[h];
-  const int tiles = a < n ? (b.sizeQ[(long long)h * m.Cq + a] + kTileRows - 1) / kTileRows : 0;
+  const int tiles = a < n ? (b.sizeQ[(long long)h * m.Cq + a] + kItemRows - 1) / kItemRows : 0;
   int tot;
   const int off = block_exclusive_scan(tiles, sh, &tot);
   for (int t = 0; t < tiles; ++t) work[(long long)h * max_items + off + t] = (a << 16) | t;
@@ -443,7 +453,7 @@ bool tc_engine_applies(int dtype, int d, int engine) {
   return engine == SPARSEPR_ENGINE_AUTO && dtype == SPARSEPR_BF16 && (d == 64 || d == 128);
 }
 
-int tc_max_items(const Dims& m) { return m.Cq + cdiv(m.Nq, kTileRows); }
+int tc_max_items(const Dims& m) { return m.Cq + cdiv(m.Nq, kItemRows); }
 
 sparsepr_status launch_sparse_attention_tc(const Plan& p, cudaStream_t st) {
   const Dims& m = p.dm;
@@ -488,7 +498,7 @@ sparsepr_status launch_dense_attention_tc(const Dims& m, const void* Q, const vo
   a.out = Out;
   a.err = err;
   if (!a.err) SPR_CUDA_OK(cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_dense_err));
-  return with_tc_d(m.d, [&](auto DD) { return launch_tc<decltype(DD)::value>(a, dim3(cdiv(m.Nq, kTileRows), m.H), st); });
+  return with_tc_d(m.d, [&](auto DD) { return launch_tc<decltype(DD)::value>(a, dim3(cdiv(m.Nq, kItemRows), m.H), st); });
 }
 
 }  // namespace spr

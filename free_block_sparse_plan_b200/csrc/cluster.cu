@@ -29,11 +29,6 @@ struct KmView {         // one k-means instance (keys or queries) for all heads
   int* off;             // [H][C+1]
   int* km;              // [H][4]: done, changed[0], changed[1], iterations
   double* obj;          // [H][C]
-  float* ub2;           // [H][N] exact squared distance to the assigned centre
-  float* lb2;           // [H][N] smallest squared distance to another centre, last scan
-  int* movedflag;       // [H][C] 1 if the centre changed in the last update
-  int* moved;           // [H][C] ids of the moved centres
-  int* nmoved;          // [H] how many
   int N, C, r, nch, stage;
 };
 
@@ -41,10 +36,8 @@ KmView view(const Plan& p, bool query) {
   const Buffers& b = p.b;
   const Dims& m = p.dm;
   if (query)
-    return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, b.ubQ, b.lbQ,
-            b.movedfQ, b.movedQ, b.nmovedQ, m.Nq, m.Cq, m.rQ, m.nchQ, 1};
-  return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, b.ubK, b.lbK,
-          b.movedfK, b.movedK, b.nmovedK, m.Nk, m.Ck, m.rK, m.nchK, 0};
+    return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, m.Nq, m.Cq, m.rQ, m.nchQ, 1};
+  return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, m.Nk, m.Ck, m.rK, m.nchK, 0};
 }
 
 // ---------------------------------------------------------------------------------
@@ -134,126 +127,53 @@ __global__ void km_init_kernel(KmView v, unsigned long long seed) {
   }
 }
 
-// Squared distance, direct sum of squared differences in fp32 over ascending dimensions
-// (zero padding beyond r adds exact zeros).  Every distance that decides a label is
-// computed this way, so labels do not depend on which centres a search visits.
-template <int R>
-__device__ __forceinline__ float dist2(const float (&x)[R], const float* c, int r) {
-  float s = 0.0f;
-#pragma unroll
-  for (int k = 0; k < R; ++k) {
-    const float t = x[k] - (k < r ? c[k] : 0.0f);
-    s = fmaf(t, t, s);
-  }
-  return s;
-}
-
-// Assignment: label = argmin_c ||x - c||^2, ties to the lowest index -- exactly the
-// result of a full scan over all centres, computed by scanning only the centres that
-// moved in the last update.  Every distance that decides a label comes from dist2(), so
-// an unmoved centre has the bit-identical distance it had when it was last scanned:
-//   ub2  exact squared distance to the assigned centre;
-//   lb2  smallest exact squared distance to any other centre when last scanned (for
-//        unmoved centres still exact, so still a lower bound).
-// A point takes the best of its own centre and the moved ones; if that is strictly below
-// lb2 no unmoved centre can win (equal would need the index rule) and the label is
-// final, else the point rescans all centres.  The first step scans every centre.
+// Assignment: label = argmin_c ||x - c||^2 (direct sum of squared differences in fp32,
+// dimensions in ascending order; ties to the lowest index).
 template <int R>
 __global__ void __launch_bounds__(128) km_assign_kernel(KmView v, int it) {
   constexpr int TILE = 64;
   __shared__ float cs[TILE * R];
-  __shared__ int cid[TILE];
   const int h = blockIdx.y;
   int* km = v.km + 4 * h;
   if (km[0]) return;
-  if (blockIdx.x == 0 && threadIdx.x == 0) km[3] += 1;
-  const int C = v.C, r = v.r;
   const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const bool valid = row < v.N;
   float x[R];
-  const float* xp = v.X + ((long long)h * v.N + (valid ? row : 0)) * r;
+  const float* xp = v.X + ((long long)h * v.N + (valid ? row : 0)) * v.r;
 #pragma unroll
-  for (int k = 0; k < R; ++k) x[k] = (k < r) ? xp[k] : 0.0f;
-  const long long pi = (long long)h * v.N + (valid ? row : 0);
-  const int lab = valid ? v.lab[pi] : -1;
-  const float* cent = v.cent + (long long)h * C * r;
-  const int nmoved = (it == 0) ? C : v.nmoved[h];
-  const int* moved = v.moved + (long long)h * C;
-  const bool own_moved = lab < 0 || (it == 0) || v.movedflag[(long long)h * C + lab];
-  // candidates: the own centre (if it did not move its distance is ub2) and the moved set
-  int best = -1;
-  float bestd2 = 3.402823466e38f, second = 3.402823466e38f;
-  if (!own_moved) {
-    best = lab;
-    bestd2 = v.ub2[pi];
-  }
-  for (int c0 = 0; c0 < nmoved; c0 += TILE) {
-    const int nc = (nmoved - c0) < TILE ? (nmoved - c0) : TILE;
+  for (int k = 0; k < R; ++k) x[k] = (k < v.r) ? xp[k] : 0.0f;
+  float best = 3.402823466e38f;
+  int bi = 0;
+  const float* ch = v.cent + (long long)h * v.C * v.r;
+  for (int c0 = 0; c0 < v.C; c0 += TILE) {
+    const int nc = (v.C - c0) < TILE ? (v.C - c0) : TILE;
     __syncthreads();
     for (int e = threadIdx.x; e < nc * R; e += blockDim.x) {
       const int c = e / R, k = e % R;
-      const int id = (it == 0) ? c0 + c : moved[c0 + c];
-      if (k == 0) cid[c] = id;
-      cs[e] = k < r ? cent[(long long)id * r + k] : 0.0f;
+      cs[e] = k < v.r ? ch[(long long)(c0 + c) * v.r + k] : 0.0f;
     }
     __syncthreads();
     for (int c = 0; c < nc; ++c) {
-      float d2 = 0.0f;
+      float dsum = 0.0f;
 #pragma unroll
       for (int k = 0; k < R; ++k) {
         const float t = x[k] - cs[c * R + k];
-        d2 = fmaf(t, t, d2);
+        dsum = fmaf(t, t, dsum);
       }
-      const int b = cid[c];
-      if (d2 < bestd2 || (d2 == bestd2 && b < best)) {
-        second = fminf(second, bestd2);
-        bestd2 = d2;
-        best = b;
-      } else {
-        second = fminf(second, d2);
+      if (dsum < best) {
+        best = dsum;
+        bi = c0 + c;
       }
     }
   }
-  if (!valid) return;
-  float lb2 = v.lb2[pi];
-  const bool all_scanned = (it == 0) || nmoved == C;
-  if (all_scanned || bestd2 < lb2) {
-    if (!all_scanned) second = fminf(second, lb2);
-  } else {
-    // an unmoved centre might tie or win: rescan everything (rare)
-    best = -1;
-    bestd2 = 3.402823466e38f;
-    second = 3.402823466e38f;
-    for (int b = 0; b < C; ++b) {
-      const float d2 = dist2<R>(x, cent + (long long)b * r, r);
-      if (d2 < bestd2 || (d2 == bestd2 && b < best)) {
-        second = fminf(second, bestd2);
-        bestd2 = d2;
-        best = b;
-      } else {
-        second = fminf(second, d2);
-      }
+  if (valid) {
+    int* lp = v.lab + (long long)h * v.N + row;
+    if (*lp != bi) {
+      *lp = bi;
+      km[1 + (it & 1)] = 1;
     }
   }
-  v.ub2[pi] = bestd2;
-  v.lb2[pi] = second;
-  if (best != lab) {
-    v.lab[pi] = best;
-    km[1 + (it & 1)] = 1;
-  }
-}
-
-// Moved-centre list of every head after an update: centres whose coordinates changed.
-__global__ void __launch_bounds__(1024) km_moved_kernel(KmView v) {
-  __shared__ int sh[32];
-  const int h = blockIdx.x, C = v.C;
-  if (v.km[4 * h]) return;
-  const int c = threadIdx.x;
-  const int f = c < C ? v.movedflag[(long long)h * C + c] : 0;
-  int tot;
-  const int pos = block_exclusive_scan(f, sh, &tot);
-  if (f) v.moved[(long long)h * C + pos] = c;
-  if (threadIdx.x == 0) v.nmoved[h] = tot;
+  if (blockIdx.x == 0 && threadIdx.x == 0) km[3] += 1;
 }
 
 // Should the update of iteration `it` run?  force: always (final pass / given labels).
@@ -357,12 +277,6 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
     double s = 0.0;
     for (int q = 0; q < kMeanSub; ++q) s += part[q][k];
     mean = cnt > 0 ? s / (double)cnt : (double)cent[k];
-  }
-  if (!force) {
-    // did this centre change?  (identical members give a bit-identical mean)
-    const int ch = (sub == 0 && k < v.r && cnt > 0 && (float)mean != cent[k]) ? 1 : 0;
-    const int any = __syncthreads_or(ch);
-    if (threadIdx.x == 0) v.movedflag[(long long)h * v.C + c] = any;
   }
   __syncthreads();
   if (cnt > 0 && sub == 0 && k < v.r) cent[k] = (float)mean;
@@ -559,10 +473,6 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
     SPR_LAUNCH_OK();
     sparsepr_status s = run_update(p, v, it, false, st);
     if (s != SPARSEPR_OK) return s;
-    if (it + 1 < p.dm.max_iter) {
-      km_moved_kernel<<<H, 1024, 0, st>>>(v);
-      SPR_LAUNCH_OK();
-    }
   }
   return SPARSEPR_OK;
 }

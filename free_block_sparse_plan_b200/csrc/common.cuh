@@ -52,10 +52,6 @@ struct Buffers {
   int *kmK, *kmQ;            // per-head k-means state [H][4]: done, changed, iters, -
   double *objK, *objQ;       // per-cluster objective partials [H][C]
   double *objH;              // [H][2] final objectives
-  float *ubK, *lbK, *ubQ, *lbQ;  // k-means exact squared distances: own / best other [H][N]
-  int *movedfK, *movedfQ;    // centre changed in the last update [H][C]
-  int *movedK, *movedQ;      // moved centre ids [H][C]
-  int *nmovedK, *nmovedQ;    // moved centre counts [H]
   int *compK, *compQ;        // raw label -> compact id (-1 if empty) [H][C]
   int *usedK, *usedQ;        // compact id -> raw label [H][C]
   int *nK, *nQ;              // [H] non-empty group counts
