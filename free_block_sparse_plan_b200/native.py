@@ -43,7 +43,7 @@ SYMBOLS = [
     "sparsepr_workspace_size", "sparsepr_plan", "sparsepr_plan_from_labels", "sparsepr_attend",
     "sparsepr_probe_fit", "sparsepr_correct", "sparsepr_forward", "sparsepr_dense_attention",
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
-    "sparsepr_destroy", "sparsepr_status_string",
+    "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
 ]
 
 
@@ -99,6 +99,8 @@ def lib():
             "sparsepr_export_size": (c_int32, [c_void_p, c_int32, POINTER(c_size_t)]),
             "sparsepr_export": (c_int32, [c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
             "sparsepr_destroy": (None, [c_void_p]),
+            "sparsepr_dense_rows_noalloc": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                      c_int32, c_void_p, c_void_p]),
             "sparsepr_status_string": (c_char_p, [c_int32]),
         }
         for name, (res, args) in sig.items():
@@ -212,6 +214,11 @@ def sparsepr_destroy(plan):
 
 def sparsepr_status_string(status: int) -> str:
     return status_string(status)
+
+
+def sparsepr_dense_rows_noalloc(params, Q, K, V, rows, nrows, Out, stream):
+    _check(lib().sparsepr_dense_rows_noalloc(ctypes.byref(params), Q, K, V, rows, nrows, Out,
+                                             stream), "sparsepr_dense_rows_noalloc")
 
 
 # ----------------------------------------------------------------------------------

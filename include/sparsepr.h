@@ -168,6 +168,29 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
                                          const void* K, const void* V, void* Out,
                                          void* stream);
 
+/*
+ * Exact attention of selected query rows without any device allocation.  The paper has
+ * no counterpart: this is a library convenience for callers that cannot allocate device
+ * memory around the call -- code whose device memory is owned by another allocator (a
+ * framework's caching pool that has reserved the GPU) and latency-critical loops that
+ * must not pay the implicit device synchronisation of cudaMalloc/cudaFree.
+ *   Q [H,N_q,d], K, V [H,N_k,d]: device, params dtype; only H, N_q, N_k, d, dtype and
+ *   engine of params are read.  rows: device int32 [nrows], 1 <= nrows <= 128, indices
+ *   into [0,N_q) (out-of-range indices are clamped, never read outside Q).  Out: device
+ *   [H,nrows,d], params dtype: softmax(q K^T / sqrt(d)) V for each requested row.
+ * Work space is a fixed 16 MiB device array inside the library, held on every GPU that
+ * loads it until the process exits; a call needing more (about
+ * H * nrows * ceil(N_k/4096) * (d+2) * 4 bytes) returns SPARSEPR_ERR_WORKSPACE before
+ * launching anything.  The first call on a device looks up that array's address (with
+ * that device current), so make it before any stream capture.  All calls share the
+ * array: calls whose work overlaps on the GPU race and must be serialised by the caller.
+ * Asynchronous on `stream`; calls no allocator.
+ */
+sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* params, const void* Q,
+                                            const void* K, const void* V,
+                                            const int32_t* rows, int32_t nrows, void* Out,
+                                            void* stream);
+
 /* Synchronises `stream` and reports the device error word: SPARSEPR_OK or
  * SPARSEPR_ERR_DEVICE_CHECK (with the word in *device_error when non-NULL). */
 sparsepr_status sparsepr_check(sparsepr_plan_t plan, void* stream, int32_t* device_error);
