@@ -74,10 +74,10 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->FQ64 = c.take<double>(H * d * m.rQ);
   b->FK = c.take<float>(H * d * m.rK);
   b->FQ = c.take<float>(H * d * m.rQ);
-  b->phiK = c.take<float>(H * Nk * m.rK);
-  b->phiQ = c.take<float>(H * Nq * m.rQ);
-  b->centK = c.take<float>(H * Ck * m.rK);
-  b->centQ = c.take<float>(H * Cq * m.rQ);
+  b->phiK = c.take<double>(H * Nk * m.rK);
+  b->phiQ = c.take<double>(H * Nq * m.rQ);
+  b->centK = c.take<double>(H * Ck * m.rK);
+  b->centQ = c.take<double>(H * Cq * m.rQ);
   b->labK = c.take<int>(H * Nk);
   b->labQ = c.take<int>(H * Nq);
   b->histK = c.take<int>(H * Ck * m.nchK);
@@ -110,7 +110,7 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->Qp = c.take<char>(H * Nq * d * es);
   b->Kp = c.take<char>(H * Nk * d * es);
   b->Vp = c.take<char>(H * Nk * d * es);
-  b->dist = c.take<float>(H * Nq);
+  b->dist = c.take<double>(H * Nq);
   b->probeTop = c.take<int>(H * Cq * M);
   b->probes = c.take<int>(H * M);
   b->probeA = c.take<int>(H * M);
@@ -131,9 +131,23 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->sig = c.take<double>(H * kMaxM);
   b->reff = c.take<int>(H);
   b->Bp = c.take<float>(H * d * d);
+  b->BpT = c.take<float>(H * d * d);
   b->cvec = c.take<float>(H * d);
   b->work = c.take<int>(H * (size_t)tc_max_items(m));
   b->nwork = c.take<int>(H);
+  {
+    const size_t Nm = Nk > Nq ? Nk : Nq, Cm = Ck > Cq ? Ck : Cq;
+    const size_t Np = (size_t)km_tc_npad((int)Nm), Cp = (size_t)km_tc_cpad((int)Cm);
+    b->kmXhi = c.take<__nv_bfloat16>(H * Np * 64);
+    b->kmXlo = c.take<__nv_bfloat16>(H * Np * 64);
+    b->kmXn = c.take<float>(H * Nm);
+    b->kmChi = c.take<__nv_bfloat16>(H * Cp * 64);
+    b->kmClo = c.take<__nv_bfloat16>(H * Cp * 64);
+    b->kmCn = c.take<float>(H * Cp);
+    b->kmCmaxb = c.take<int>(2 * H);
+    b->kmQueue = c.take<int4>((size_t)km_tc_queue_cap((int)H, (int)Nm));
+    b->kmQcnt = c.take<int>(2);
+  }
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);
 }
@@ -231,9 +245,9 @@ ExportDesc export_desc(const Plan& p, int what) {
     case SPARSEPR_X_EIG_Q: return {b.lamQ, H * m.rQ * D};
     case SPARSEPR_X_METRIC_K: return {b.MK, H * d * d * D};
     case SPARSEPR_X_METRIC_Q: return {b.MQ, H * d * d * D};
-    case SPARSEPR_X_PHI_K: return {b.phiK, H * m.Nk * m.rK * F};
-    case SPARSEPR_X_PHI_Q: return {b.phiQ, H * m.Nq * m.rQ * F};
-    case SPARSEPR_X_CENTRES_Q: return {b.centQ, H * m.Cq * m.rQ * F};
+    case SPARSEPR_X_PHI_K: return {b.phiK, H * m.Nk * m.rK * D};
+    case SPARSEPR_X_PHI_Q: return {b.phiQ, H * m.Nq * m.rQ * D};
+    case SPARSEPR_X_CENTRES_Q: return {b.centQ, H * m.Cq * m.rQ * D};
     case SPARSEPR_X_SCORES: return {b.scores, H * m.Cq * m.Ck * D};
     case SPARSEPR_X_OSP: return {b.Osp, H * m.Nq * d * F};
     case SPARSEPR_X_ODENSE_PROBE: return {b.Odense, H * m.M * d * F};
@@ -243,7 +257,7 @@ ExportDesc export_desc(const Plan& p, int what) {
     case SPARSEPR_X_FIT_B: return {b.Bm, H * d * d * D};
     case SPARSEPR_X_FIT_P: return {b.Pm, H * d * d * D};
     case SPARSEPR_X_FIT_REFF: return {b.reff, H * I};
-    case SPARSEPR_X_PROBE_DIST: return {b.dist, H * m.Nq * F};
+    case SPARSEPR_X_PROBE_DIST: return {b.dist, H * m.Nq * D};
     case SPARSEPR_X_KBAR: return {b.kbar, H * m.Ck * d * D};
     case SPARSEPR_X_QBAR: return {b.qbar, H * m.Cq * d * D};
     default: return {nullptr, 0};

@@ -43,6 +43,7 @@ constexpr int kTcThreads = 384;
 constexpr int kProducers = 96;                   // warps 8-10
 constexpr long long kWaitCycles = 2000000000LL;   // about one second: a hung pipeline
 constexpr float kRescaleLog2 = 8.0f;              // lazy rescale threshold (factor 256)
+constexpr int kPolyPairs = 4;                     // of every 16 column pairs: exp2 on the FMA pipe
 
 enum Mode { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
@@ -86,20 +87,24 @@ struct Misc {
 };
 
 enum Bar {
-  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 3, bSFull0 = 5, bPFull0 = 7, bPvDone0 = 9, bDrain = 11
+  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 3, bSFull0 = 5, bPFull0 = 7, bPvDone0 = 9, bDrain = 11, bOReady = 12
 };
 
+// Bounded wait; the clock and the abort flag are read once every 32 polls so that
+// waiting warps take few issue slots from the working ones.
 __device__ __forceinline__ bool wait_bar(Misc* ms, uint32_t bar, uint32_t parity, int* err) {
   if (tc::mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!tc::mbar_try_wait(bar, parity)) {
-    if (*reinterpret_cast<volatile int*>(&ms->abort_flag)) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      if (atomicExch(&ms->abort_flag, 1) == 0) atomicOr(err, kErrHang);
-      return false;
+  for (unsigned n = 1;; ++n) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if ((n & 31) == 0) {
+      if (*reinterpret_cast<volatile int*>(&ms->abort_flag)) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        if (atomicExch(&ms->abort_flag, 1) == 0) atomicOr(err, kErrHang);
+        return false;
+      }
     }
   }
-  return true;
 }
 
 template <int D>
@@ -176,6 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       tc::mbar_init(BAR(bPvDone0 + s), 1);
     }
     tc::mbar_init(BAR(bDrain), 1);
+    tc::mbar_init(BAR(bOReady), 1);
     ms->abort_flag = 0;
   }
   if (warp == 11) {
@@ -260,48 +266,78 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     if (lane == 0) {
       constexpr uint32_t idQK = tc::idesc_bf16_f32(kTileRows, kTileKeys, false);
       constexpr uint32_t idPV = tc::idesc_bf16_f32(kTileRows, D, true);
-      auto issue_s = [&](int t, int j) {
+      // S of query tile t against key tile j into S buffer `buf` (TMEM columns 128 buf)
+      auto issue_s = [&](int t, int j, int buf) {
         const int s = j & 1;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = tc::sw128_desc(sQ(t) + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = tc::sw128_desc(sK(s) + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
-          tc::mma_ss(tmem + 128 * t, ad, bd, idQK, kk > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + 128 * buf, ad, bd, idQK, kk > 0 ? 1u : 0u);
         }
-        tc::mma_commit(BAR(bSFull0 + t));
+        tc::mma_commit(BAR(bSFull0 + buf));
       };
-      auto issue_pv = [&](int t, int j) {
+      // O_t += P V_j with P in S buffer `buf`
+      auto issue_pv = [&](int t, int j, int buf) {
         const int s = j & 1;
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk) {
           const uint64_t bd = tc::sw128_desc(sV(s) + kk * 2048, L::kPanel, 1024);
-          tc::mma_ts(tmem + 256 + 128 * t, tmem + 128 * t + 8 * kk, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tmem + 256 + 128 * t, tmem + 128 * buf + 8 * kk, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(BAR(bPvDone0 + t));
       };
       bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && wait_bar(ms, BAR(bKVFull0), 0, g.err);
-      if (ok) {
-        tc::fence_after_sync();
-        issue_s(0, 0);
-        if (hasB) issue_s(1, 0);
-      }
-      for (int j = 0; ok && j < nt; ++j) {
-        if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err)) { ok = false; break; }
-        tc::fence_after_sync();
-        issue_pv(0, j);
-        const bool more = j + 1 < nt;
-        if (more) {
-          if (!wait_bar(ms, BAR(bKVFull0 + ((j + 1) & 1)), ((j + 1) >> 1) & 1, g.err)) { ok = false; break; }
+      if (hasB) {
+        // two query tiles: the softmax of one overlaps the products of the other
+        if (ok) {
           tc::fence_after_sync();
-          issue_s(0, j + 1);
+          issue_s(0, 0, 0);
+          issue_s(1, 0, 1);
         }
-        if (hasB) {
+        for (int j = 0; ok && j < nt; ++j) {
+          if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_pv(0, j, 0);
+          const bool more = j + 1 < nt;
+          if (more) {
+            if (!wait_bar(ms, BAR(bKVFull0 + ((j + 1) & 1)), ((j + 1) >> 1) & 1, g.err)) { ok = false; break; }
+            tc::fence_after_sync();
+            issue_s(0, j + 1, 0);
+          }
           if (!wait_bar(ms, BAR(bPFull0 + 1), j & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
-          issue_pv(1, j);
+          issue_pv(1, j, 1);
+          tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
+          if (more) issue_s(1, j + 1, 1);
         }
-        tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
-        if (hasB && more) issue_s(1, j + 1);
+      } else {
+        // one query tile: S alternates between the two S buffers, so S(j+1) is ready
+        // while the softmax of tile j runs
+        if (ok) {
+          tc::fence_after_sync();
+          issue_s(0, 0, 0);
+          if (nt > 1) {
+            ok = wait_bar(ms, BAR(bKVFull0 + 1), 0, g.err);
+            if (ok) {
+              tc::fence_after_sync();
+              issue_s(0, 1, 1);
+            }
+          }
+        }
+        for (int j = 0; ok && j < nt; ++j) {
+          const int buf = j & 1;
+          if (!wait_bar(ms, BAR(bPFull0 + buf), (j >> 1) & 1, g.err)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_pv(0, j, buf);
+          tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
+          if (j + 2 < nt) {
+            if (!wait_bar(ms, BAR(bKVFull0 + (j & 1)), ((j + 2) >> 1) & 1, g.err)) { ok = false; break; }
+            tc::fence_after_sync();
+            issue_s(0, j + 2, buf);
+          }
+        }
+        if (ok) tc::mma_commit(BAR(bOReady));
       }
       tc::mma_commit(BAR(bDrain));
       // bounded: completes when every MMA issued above has finished
@@ -316,29 +352,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     const int t = warp >> 2;                            // query tile
     const int r = tid - 128 * t;                        // its row = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + 128 * t + lane_off, tO = tmem + 256 + 128 * t + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * t + lane_off;
     const float sl2 = 1.4426950408889634f / sqrtf((float)d);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + t), j & 1, g.err))) { ok = false; break; }
+      // S buffer: the tile's own with two tiles, alternating with one
+      const int buf = hasB ? t : (j & 1);
+      const uint32_t sfp = hasB ? (j & 1) : ((j >> 1) & 1);
+      const uint32_t tS = tmem + 128 * buf + lane_off;
+      if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + buf), sfp, g.err))) { ok = false; break; }
       tc::fence_after_sync();
       const int valid = (j == nt - 1) ? last_valid : kTileKeys;
+      const bool whole = valid == kTileKeys;           // uniform: no key column masked
       float mx = -INFINITY;
+      if (whole) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(tS + 32 * c, v);
-        tc::tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(tS + 32 * c, v);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * c + i < valid) mx = fmaxf(mx, v[i]);
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(tS + 32 * c, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i < valid) mx = fmaxf(mx, v[i]);
+        }
       }
       const float m_tile = mx * sl2;
       // lazy rescale: keep the running max unless it grows by more than 2^8
       if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleLog2)) {
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = tc::ex2(m_run - m_new);     // 0 on the first tile
+        // one tile: S(j) may be ready before PV(j-1) has finished updating O
+        if (!hasB && j > 0 && !__all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone0), (j - 1) & 1, g.err))) {
+          ok = false;
+          break;
+        }
         if (j > 0) {
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -354,28 +411,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         m_run = m_new;
       }
       float rs = 0.0f;
+      if (whole) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(tS + 32 * c, v);
-        tc::tmem_wait_ld();
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(tS + 32 * c, v);
+          tc::tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = (32 * c + 2 * i < valid) ? tc::ex2(fmaf(v[2 * i], sl2, -m_run)) : 0.0f;
-          const float p1 = (32 * c + 2 * i + 1 < valid) ? tc::ex2(fmaf(v[2 * i + 1], sl2, -m_run)) : 0.0f;
-          rs += p0 + p1;
-          pk[i] = tc::pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(v[2 * i], sl2, -m_run), x1 = fmaf(v[2 * i + 1], sl2, -m_run);
+            // a quarter of the exponentials on the FMA pipe, the rest on the SFU
+            const float p0 = i >= 16 - kPolyPairs ? tc::exp2_poly(x0) : tc::ex2(x0);
+            const float p1 = i >= 16 - kPolyPairs ? tc::exp2_poly(x1) : tc::ex2(x1);
+            rs += p0 + p1;
+            pk[i] = tc::pack_bf16x2(p0, p1);
+          }
+          // P columns 16c..16c+15 lie inside S columns already read (chunks 0..c)
+          tc::tmem_st16(tS + 16 * c, pk);
         }
-        // P columns 16c..16c+15 lie inside S columns already read (chunks 0..c)
-        tc::tmem_st16(tS + 16 * c, pk);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(tS + 32 * c, v);
+          tc::tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = (32 * c + 2 * i < valid) ? tc::ex2(fmaf(v[2 * i], sl2, -m_run)) : 0.0f;
+            const float p1 = (32 * c + 2 * i + 1 < valid) ? tc::ex2(fmaf(v[2 * i + 1], sl2, -m_run)) : 0.0f;
+            rs += p0 + p1;
+            pk[i] = tc::pack_bf16x2(p0, p1);
+          }
+          tc::tmem_st16(tS + 16 * c, pk);
+        }
       }
       tc::tmem_wait_st();
       l_run += rs;
       tc::fence_before_sync();
-      tc::mbar_arrive(BAR(bPFull0 + t));
+      tc::mbar_arrive(BAR(bPFull0 + buf));
     }
-    if (ok && __all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err))) {
+    const bool oready = hasB ? wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err) : wait_bar(ms, BAR(bOReady), 0, g.err);
+    if (ok && __all_sync(0xffffffffu, oready)) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
       const int row = kTileRows * t + r;

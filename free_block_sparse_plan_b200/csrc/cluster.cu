@@ -21,8 +21,8 @@ __device__ __forceinline__ unsigned long long sm64_mix(unsigned long long z) {
 constexpr unsigned long long kGamma = 0x9E3779B97F4A7C15ULL;
 
 struct KmView {         // one k-means instance (keys or queries) for all heads
-  const float* X;       // [H][N][r] features
-  float* cent;          // [H][C][r]
+  const double* X;      // [H][N][r] features (fp64)
+  double* cent;         // [H][C][r] centres (fp64)
   int* lab;             // [H][N]
   int* hist;            // [H][C][nch]
   int* perm;            // [H][N]
@@ -41,68 +41,109 @@ KmView view(const Plan& p, bool query) {
 }
 
 // ---------------------------------------------------------------------------------
-// Response coordinates: phi = X F (keys), phi = RMSnorm(X F) (queries, floor 1e-6).
+// Response coordinates in fp64: phi = X F (keys), phi = z / max(rms(z), 1e-6) with
+// z = X F (queries) (paper S4.1, App. B.1-B.2).  X is exact in its dtype; F is the fp64
+// factor; each coordinate is one fp64 dot product over d in ascending order.
+// A block takes 64 rows; thread (row, q) forms coordinates q*R/4 .. (q+1)*R/4 - 1 of its
+// row from the row staged in shared memory and F staged once per block.  When the
+// tensor-core k-means will cluster these coordinates, the block also writes its input:
+// each row split into two bf16 pieces (rows padded to 64 columns, zero rows up to Npad)
+// and |phi|.
+constexpr int kProjRows = 64;
 template <int R, bool RMS>
-__global__ void __launch_bounds__(128) project_kernel(Dims m, const void* X, int N,
-                                                     const float* Fall, int r, float* out) {
-  extern __shared__ float sm[];
+__global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int N, const double* Fall, int r,
+                                                      double* out, __nv_bfloat16* xhi, __nv_bfloat16* xlo,
+                                                      float* xn, int Npad) {
+  constexpr int P = R / 4;                 // coordinates per thread
+  extern __shared__ double smd[];
   const int d = m.d, h = blockIdx.y;
-  float* F = sm;                       // [d][R] zero padded
-  float* T = sm + d * R;               // [128][d+1]
-  const float* Fh = Fall + (long long)h * d * r;
+  double* F = smd;                         // [d][R], zero columns k >= r
+  float* T = reinterpret_cast<float*>(smd + d * R);   // [64][d + 1]
+  const double* Fh = Fall + (long long)h * d * r;
   for (int e = threadIdx.x; e < d * R; e += blockDim.x) {
     const int j = e / R, k = e % R;
-    F[e] = k < r ? Fh[j * r + k] : 0.0f;
+    F[e] = k < r ? Fh[j * r + k] : 0.0;
   }
-  const long long row0 = (long long)blockIdx.x * 128;
+  const long long row0 = (long long)blockIdx.x * kProjRows;
   const long long base = ((long long)h * N) * d;
-  for (int e = threadIdx.x; e < 128 * d; e += blockDim.x) {
+  for (int e = threadIdx.x; e < kProjRows * d; e += blockDim.x) {
     const int i = e / d, j = e % d;
     const long long row = row0 + i;
     T[i * (d + 1) + j] = row < N ? load_as_float(X, base + row * d + j, m.dtype) : 0.0f;
   }
   __syncthreads();
-  const long long row = row0 + threadIdx.x;
-  if (row >= N) return;
-  float acc[R];
+  const int ri = threadIdx.x >> 2, q = threadIdx.x & 3;
+  const long long row = row0 + ri;
+  double acc[P];
 #pragma unroll
-  for (int k = 0; k < R; ++k) acc[k] = 0.0f;
-  const float* x = T + threadIdx.x * (d + 1);
+  for (int k = 0; k < P; ++k) acc[k] = 0.0;
+  const float* x = T + ri * (d + 1);
   for (int j = 0; j < d; ++j) {
-    const float xv = x[j];
-    const float4* f4 = reinterpret_cast<const float4*>(F + j * R);
+    const double xv = (double)x[j];
+    const double2* f2 = reinterpret_cast<const double2*>(F + j * R + q * P);
 #pragma unroll
-    for (int k = 0; k < R / 4; ++k) {
-      const float4 f = f4[k];
-      acc[4 * k] = fmaf(xv, f.x, acc[4 * k]);
-      acc[4 * k + 1] = fmaf(xv, f.y, acc[4 * k + 1]);
-      acc[4 * k + 2] = fmaf(xv, f.z, acc[4 * k + 2]);
-      acc[4 * k + 3] = fmaf(xv, f.w, acc[4 * k + 3]);
+    for (int k = 0; k < P / 2; ++k) {
+      const double2 f = f2[k];
+      acc[2 * k] = fma(xv, f.x, acc[2 * k]);
+      acc[2 * k + 1] = fma(xv, f.y, acc[2 * k + 1]);
     }
   }
-  float scale = 1.0f;
+  // the row's four threads are adjacent lanes: sums over the row by shuffles in a fixed order
+  auto row_sum = [](double v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    return v;
+  };
+  double scale = 1.0;
   if (RMS) {
-    float ss = 0.0f;
+    double ss = 0.0;
 #pragma unroll
-    for (int k = 0; k < R; ++k) ss = fmaf(acc[k], acc[k], ss);
-    const float rms = sqrtf(ss / (float)r);
-    scale = 1.0f / fmaxf(rms, 1e-6f);
+    for (int k = 0; k < P; ++k) ss = fma(acc[k], acc[k], ss);
+    ss = row_sum(ss);
+    scale = 1.0 / fmax(sqrt(ss / (double)r), 1e-6);
   }
-  float* o = out + ((long long)h * N + row) * r;
 #pragma unroll
-  for (int k = 0; k < R; ++k)
-    if (k < r) o[k] = RMS ? acc[k] * scale : acc[k];
+  for (int k = 0; k < P; ++k) acc[k] = RMS ? acc[k] * scale : acc[k];
+  if (row < N) {
+    double* o = out + ((long long)h * N + row) * r;
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+      if (q * P + k < r) o[q * P + k] = acc[k];
+  }
+  if (xhi) {
+    double ss = 0.0;
+#pragma unroll
+    for (int k = 0; k < P; ++k) ss = fma(acc[k], acc[k], ss);
+    ss = row_sum(ss);
+    if (row < Npad) {
+      const long long xb = ((long long)h * Npad + row) * 64;
+#pragma unroll
+      for (int k = 0; k < P; ++k) {
+        const double v = row < N ? acc[k] : 0.0;
+        const __nv_bfloat16 hi = __double2bfloat16(v);
+        xhi[xb + q * P + k] = hi;
+        xlo[xb + q * P + k] = __double2bfloat16(v - (double)__bfloat162float(hi));
+      }
+      if (q == 3)
+        for (int k = R; k < 64; ++k) {
+          xhi[xb + k] = __float2bfloat16_rn(0.0f);
+          xlo[xb + k] = __float2bfloat16_rn(0.0f);
+        }
+      if (q == 0 && row < N) xn[(long long)h * N + row] = (float)sqrt(ss);
+    }
+  }
 }
 
 template <bool RMS>
-sparsepr_status launch_project(const Plan& p, const void* X, int N, const float* F, int r,
-                               float* out, cudaStream_t st) {
+sparsepr_status launch_project(const Plan& p, const void* X, int N, const double* F, int r, double* out,
+                               __nv_bfloat16* xhi, __nv_bfloat16* xlo, float* xn, int Npad, cudaStream_t st) {
   const int d = p.dm.d;
-  dim3 grid(cdiv(N, 128), p.dm.H);
+  const int rows = xhi ? Npad : N;
+  dim3 grid(cdiv(rows, kProjRows), p.dm.H);
   auto run = [&](auto kern, int R) -> sparsepr_status {
-    const size_t smem = (size_t)(d * R + 128 * (d + 1)) * sizeof(float);
+    const size_t smem = (size_t)d * R * sizeof(double) + (size_t)kProjRows * (d + 1) * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    kern<<<grid, 128, smem, st>>>(p.dm, X, N, F, r, out);
+    kern<<<grid, 4 * kProjRows, smem, st>>>(p.dm, X, N, F, r, out, xhi, xlo, xn, Npad);
     SPR_LAUNCH_OK();
     return SPARSEPR_OK;
   };
@@ -127,38 +168,40 @@ __global__ void km_init_kernel(KmView v, unsigned long long seed) {
   }
 }
 
-// Assignment: label = argmin_c ||x - c||^2 (direct sum of squared differences in fp32,
+// Assignment: label = argmin_c ||x - c||^2 (direct sum of squared differences in fp64,
 // dimensions in ascending order; ties to the lowest index).
 template <int R>
 __global__ void __launch_bounds__(128) km_assign_kernel(KmView v, int it) {
-  constexpr int TILE = 64;
-  __shared__ float cs[TILE * R];
+  constexpr int TILE = 32;
+  __shared__ double cs[TILE * R];
   const int h = blockIdx.y;
   int* km = v.km + 4 * h;
   if (km[0]) return;
   const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const bool valid = row < v.N;
-  float x[R];
-  const float* xp = v.X + ((long long)h * v.N + (valid ? row : 0)) * v.r;
+  double x[R];
+  const double* xp = v.X + ((long long)h * v.N + (valid ? row : 0)) * v.r;
 #pragma unroll
-  for (int k = 0; k < R; ++k) x[k] = (k < v.r) ? xp[k] : 0.0f;
-  float best = 3.402823466e38f;
+  for (int k = 0; k < R; ++k) x[k] = (k < v.r) ? xp[k] : 0.0;
+  double best = 1.7976931348623157e308;
   int bi = 0;
-  const float* ch = v.cent + (long long)h * v.C * v.r;
+  const double* ch = v.cent + (long long)h * v.C * v.r;
   for (int c0 = 0; c0 < v.C; c0 += TILE) {
     const int nc = (v.C - c0) < TILE ? (v.C - c0) : TILE;
     __syncthreads();
     for (int e = threadIdx.x; e < nc * R; e += blockDim.x) {
       const int c = e / R, k = e % R;
-      cs[e] = k < v.r ? ch[(long long)(c0 + c) * v.r + k] : 0.0f;
+      cs[e] = k < v.r ? ch[(long long)(c0 + c) * v.r + k] : 0.0;
     }
     __syncthreads();
     for (int c = 0; c < nc; ++c) {
-      float dsum = 0.0f;
+      double dsum = 0.0;
 #pragma unroll
       for (int k = 0; k < R; ++k) {
-        const float t = x[k] - cs[c * R + k];
-        dsum = fmaf(t, t, dsum);
+        if (k < v.r) {
+          const double t = x[k] - cs[c * R + k];
+          dsum = fma(t, t, dsum);
+        }
       }
       if (dsum < best) {
         best = dsum;
@@ -245,11 +288,15 @@ __global__ void __launch_bounds__(kSortChunk) cs_scatter_kernel(KmView v, int it
 }
 
 // Pass 4: centre = mean of members (fp64 sums in group-major order); empty clusters keep
-// their centre.  Also the cluster's share of the objective at its new centre.
+// their centre.  The final pass (force) also forms the cluster's share of the objective
+// at its new centre.  Member rows are read through the permutation, four at a time per
+// thread so that several gathers are in flight.
 constexpr int kMeanSub = 4;
+constexpr int kMeanIdx = 1024;      // member indices staged in shared memory per round
 __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int it, bool force) {
   __shared__ double part[kMeanSub][kMaxR];
   __shared__ double opart[kMeanSub * kMaxR / 32];
+  __shared__ int idx[kMeanIdx];
   const int h = blockIdx.y, c = blockIdx.x;
   int* km = v.km + 4 * h;
   if (!force) {
@@ -264,27 +311,48 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
   const int* off = v.off + (long long)h * (v.C + 1);
   const int m0 = off[c], m1 = off[c + 1];
   const int* perm = v.perm + (long long)h * v.N;
-  const float* X = v.X + (long long)h * v.N * v.r;
+  const double* X = v.X + (long long)h * v.N * v.r;
+  const bool kk = k < v.r;
+  // member rows in rounds of kMeanIdx; thread (sub, k) sums members sub, sub + 4, ...
   double acc = 0.0;
-  if (k < v.r)
-    for (int mm = m0 + sub; mm < m1; mm += kMeanSub) acc += (double)X[(long long)perm[mm] * v.r + k];
+  for (int b0 = m0; b0 < m1; b0 += kMeanIdx) {
+    const int nb = min(kMeanIdx, m1 - b0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) idx[i] = perm[b0 + i];
+    __syncthreads();
+    if (kk) {
+      int i = sub;
+      for (; i + 3 * kMeanSub < nb; i += 4 * kMeanSub) {
+        const double x0 = X[(long long)idx[i] * v.r + k];
+        const double x1 = X[(long long)idx[i + kMeanSub] * v.r + k];
+        const double x2 = X[(long long)idx[i + 2 * kMeanSub] * v.r + k];
+        const double x3 = X[(long long)idx[i + 3 * kMeanSub] * v.r + k];
+        acc += x0;
+        acc += x1;
+        acc += x2;
+        acc += x3;
+      }
+      for (; i < nb; i += kMeanSub) acc += X[(long long)idx[i] * v.r + k];
+    }
+  }
   part[sub][k] = acc;
   __syncthreads();
   const int cnt = m1 - m0;
-  float* cent = v.cent + ((long long)h * v.C + c) * v.r;
+  double* cent = v.cent + ((long long)h * v.C + c) * v.r;
   double mean = 0.0;
-  if (k < v.r) {
+  if (kk) {
     double s = 0.0;
     for (int q = 0; q < kMeanSub; ++q) s += part[q][k];
-    mean = cnt > 0 ? s / (double)cnt : (double)cent[k];
+    mean = cnt > 0 ? s / (double)cnt : cent[k];
   }
   __syncthreads();
-  if (cnt > 0 && sub == 0 && k < v.r) cent[k] = (float)mean;
+  if (cnt > 0 && sub == 0 && kk) cent[k] = mean;
+  if (!force) return;
   // objective share: sum over members of ||x - centre||^2
   double o = 0.0;
-  if (k < v.r)
+  if (kk)
     for (int mm = m0 + sub; mm < m1; mm += kMeanSub) {
-      const double t = (double)X[(long long)perm[mm] * v.r + k] - mean;
+      const double t = X[(long long)perm[mm] * v.r + k] - mean;
       o += t * t;
     }
   o = warp_sum(o);
@@ -449,13 +517,33 @@ sparsepr_status launch_check_labels(const Plan& p, bool query, cudaStream_t st) 
   return SPARSEPR_OK;
 }
 
-sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st) {
-  return launch_project<false>(p, p.K, p.dm.Nk, p.b.FK, p.dm.rK, p.b.phiK, st);
+// The tensor-core k-means serves a side when the engine allows it and C fits its tiles.
+bool km_uses_tc(const Plan& p, bool query) {
+  const KmView v = view(p, query);
+  return p.dm.engine == SPARSEPR_ENGINE_AUTO && km_tc_supported(v.C) && (long long)p.dm.H * v.N < (1LL << 31);
 }
 
-sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st) {
-  return launch_project<true>(p, p.Q, p.dm.Nq, p.b.FQ, p.dm.rQ, p.b.phiQ, st);
+// fp64 coordinates for either engine; the split coordinates of the tensor-core k-means
+// come with them when that k-means will run.
+sparsepr_status launch_project_side(const Plan& p, bool query, cudaStream_t st) {
+  const Dims& m = p.dm;
+  const Buffers& b = p.b;
+  const void* X = query ? p.Q : p.K;
+  const int N = query ? m.Nq : m.Nk, r = query ? m.rQ : m.rK;
+  double* out = query ? b.phiQ : b.phiK;
+  const double* F = query ? b.FQ64 : b.FK64;
+  const bool fuse = km_uses_tc(p, query);
+  __nv_bfloat16* xhi = fuse ? b.kmXhi : nullptr;
+  __nv_bfloat16* xlo = fuse ? b.kmXlo : nullptr;
+  float* xn = fuse ? b.kmXn : nullptr;
+  const int Npad = km_tc_npad(N);
+  return query ? launch_project<true>(p, X, N, F, r, out, xhi, xlo, xn, Npad, st)
+               : launch_project<false>(p, X, N, F, r, out, xhi, xlo, xn, Npad, st);
 }
+
+sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st) { return launch_project_side(p, false, st); }
+
+sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st) { return launch_project_side(p, true, st); }
 
 sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   const KmView v = view(p, query);
@@ -464,8 +552,20 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   SPR_CUDA_OK(cudaMemsetAsync(v.lab, 0xFF, sizeof(int) * (size_t)H * v.N, st));  // labels = -1
   km_init_kernel<<<H, 256, 0, st>>>(v, p.dm.seed);
   SPR_LAUNCH_OK();
+  // tensor-core scores with exact rescoring (labels identical to the fp32 full scan) when
+  // there are enough centres to fill the tiles; the full scan otherwise or on request
+  const bool tc = km_uses_tc(p, query);
+  const Buffers& b = p.b;
+  const KmTcBuffers kb{b.kmXhi, b.kmXlo, b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt};
+  if (tc) {
+    SPR_CUDA_OK(cudaMemsetAsync(b.kmCmaxb, 0, sizeof(int) * 2 * H, st));
+    SPR_CUDA_OK(cudaMemsetAsync(b.kmQcnt, 0, sizeof(int) * 2, st));
+  }
   for (int it = 0; it < p.dm.max_iter; ++it) {
-    if (v.r <= 8) assign<8>(v, H, it, st);
+    if (tc) {
+      sparsepr_status s = km_tc_assign(kb, v.X, v.cent, H, v.N, v.C, v.r, it, v.lab, v.km, b.err, st);
+      if (s != SPARSEPR_OK) return s;
+    } else if (v.r <= 8) assign<8>(v, H, it, st);
     else if (v.r <= 16) assign<16>(v, H, it, st);
     else if (v.r <= 32) assign<32>(v, H, it, st);
     else if (v.r <= 48) assign<48>(v, H, it, st);

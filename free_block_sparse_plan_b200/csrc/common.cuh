@@ -43,8 +43,8 @@ struct Dims {
 struct Buffers {
   double *MK, *MQ, *lamK, *lamQ, *FK64, *FQ64;
   float *FK, *FQ;
-  float *phiK, *phiQ;
-  float *centK, *centQ;
+  double *phiK, *phiQ;      // response coordinates [H][N][r] (fp64)
+  double *centK, *centQ;     // k-means centres [H][C][r] (fp64)
   int *labK, *labQ;
   int *histK, *histQ;
   int *permK, *permQ, *invQ;
@@ -61,7 +61,7 @@ struct Buffers {
   int *cellCnt, *cellIds;    // [H][Cq], [H][Cq][Ck]
   long long *pairs;          // [H]
   void *Qp, *Kp, *Vp;        // group-major copies [H][N][d]
-  float *dist;               // [H][Nq]
+  double *dist;              // [H][Nq]
   int *probeTop;             // [H][Cq][M]
   int *probes, *probeA, *mA; // [H][M], [H][M], [H][Cq]
   double *wP;                // [H][M]
@@ -74,7 +74,15 @@ struct Buffers {
   double *sig;               // [H][kMaxM]
   int *reff;                 // [H]
   float *Bp, *cvec;          // folded correction [H][d][d], [H][d]
+  float *BpT;                // B' transposed [H][d][d] (tensor-core correction)
   int *work, *nwork;         // tensor-core attention work list [H][max items], [H]
+  __nv_bfloat16 *kmXhi, *kmXlo;  // k-means features split into bf16 pieces [H][Npad][64]
+  float *kmXn;               // feature norms [H][Nmax]
+  __nv_bfloat16 *kmChi, *kmClo;  // centres split into bf16 pieces [H][Cpad][64]
+  float *kmCn;               // squared centre norms [H][Cpad]
+  int *kmCmaxb;              // largest squared centre norm as float bits [2][H]
+  int4 *kmQueue;             // points whose label needs exact rescoring
+  int *kmQcnt;               // queue lengths [2]
   int *err;                  // device error word
 };
 
@@ -204,6 +212,23 @@ sparsepr_status launch_probe_attention_simt(const Plan& p, cudaStream_t st);
 sparsepr_status launch_probe_combine(const Plan& p, cudaStream_t st);
 sparsepr_status launch_dense_attention_tc(const Dims& m, const void* Q, const void* K, const void* V,
                                           void* Out, int* err, cudaStream_t st);
+int km_tc_npad(int N);
+int km_tc_cpad(int C);
+bool km_tc_supported(int C);
+bool correct_tc_applies(int dtype, int d, int engine);
+sparsepr_status launch_correct_tc(const Plan& p, void* Out, cudaStream_t st);
+long long km_tc_queue_cap(int H, int N);
+struct KmTcBuffers {
+  const __nv_bfloat16 *xhi, *xlo;
+  const float* xn;
+  __nv_bfloat16 *chi, *clo;
+  float* cn;
+  int* cmaxb;
+  int4* queue;
+  int* qcnt;
+};
+sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const double* cent, int H, int N, int C,
+                             int r, int it, int* lab, int* kmstate, int* err, cudaStream_t st);
 sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void* K,
                                        const void* V, void* Out, cudaStream_t st);
 

@@ -55,51 +55,72 @@ __global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const v
 }
 
 // ---------------------------------------------------------------------------------
-// One-sided Jacobi: orthogonalise the `ncols` columns (length `rows`, column-major with
-// stride `rows`) of G in shared memory.  Parallel round-robin ordering: in each round
-// the column pairs are disjoint, one warp per pair.  A pair counts as orthogonal when
-// |a.b| <= 1e-14 |a||b| or |a.b| <= 1e-15 ||G||_F^2: the second (absolute) test ends the
-// sweeps when only columns near the null space still carry rounding-level overlap, which
-// no relative test can remove.  Bounded sweeps.
-__device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red) {
+// One-sided Jacobi: orthogonalise the `ncols` columns (length `rows` <= 128, column-major
+// with stride `rows`) of G in shared memory.  Parallel round-robin ordering: in each
+// round the column pairs are disjoint; each pair is handled by 16 lanes (half a warp),
+// so 1024 threads take all 64 pairs of a round at once.  Only a.b is summed per pair: the
+// squared column norms are computed at the start of each sweep and then carried through
+// the rotations (|a'|^2 = |a|^2 - t a.b, |b'|^2 = |b|^2 + t a.b for the rotation that
+// zeroes a.b).  A pair counts as orthogonal when |a.b| <= 1e-14 |a||b| or
+// |a.b| <= 1e-15 ||G||_F^2: the second (absolute) test ends the sweeps when only columns
+// near the null space still carry rounding-level overlap, which no relative test can
+// remove.  Bounded sweeps.  `nrm` is shared scratch of at least ncols doubles.
+__device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red, double* nrm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int sub = lane & 15, grp = 2 * warp + (lane >> 4), ngrp = 2 * nwarps;
+  const unsigned half = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
   double f = 0.0;
   for (int e = threadIdx.x; e < rows * ncols; e += blockDim.x) f += G[e] * G[e];
   const double abs_tol = 1e-15 * block_sum(f, red);
   const int nn = ncols + (ncols & 1);   // pad to even with a phantom column
   const int npairs = nn / 2;
+  constexpr int kPer = kMaxD / 16;      // rows per lane
   for (int sweep = 0; sweep < 30; ++sweep) {
+    // fresh squared norms
+    for (int j = warp; j < ncols; j += nwarps) {
+      double s = 0.0;
+      for (int i = lane; i < rows; i += 32) s += G[j * rows + i] * G[j * rows + i];
+      s = warp_sum(s);
+      if (lane == 0) nrm[j] = s;
+    }
     if (threadIdx.x == 0) *flag = 0;
     __syncthreads();
     for (int round = 0; round < nn - 1; ++round) {
-      for (int k = warp; k < npairs; k += nwarps) {
+      for (int k = grp; k < npairs; k += ngrp) {
         // circle method: position 0 fixed, the others rotate by `round`
         const int pa = k, pb = nn - 1 - k;
         const int ia = pa == 0 ? 0 : 1 + (pa - 1 + round) % (nn - 1);
         const int ib = pb == 0 ? 0 : 1 + (pb - 1 + round) % (nn - 1);
-        if (ia >= ncols || ib >= ncols) continue;
+        if (ia >= ncols || ib >= ncols) continue;     // uniform over the 16 lanes
         double* a = G + (long long)ia * rows;
         double* b = G + (long long)ib * rows;
-        double al = 0.0, be = 0.0, ga = 0.0;
-        for (int i = lane; i < rows; i += 32) {
-          const double x = a[i], y = b[i];
-          al += x * x;
-          be += y * y;
-          ga += x * y;
+        double ga = 0.0;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+          const int i = sub + 16 * q;
+          if (i < rows) ga += a[i] * b[i];
         }
-        al = warp_sum(al);
-        be = warp_sum(be);
-        ga = warp_sum(ga);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) ga += __shfl_xor_sync(half, ga, o);
+        const double al = nrm[ia], be = nrm[ib];
         if (ga == 0.0 || fabs(ga) <= 1e-14 * sqrt(al * be) || fabs(ga) <= abs_tol) continue;
         const double zeta = (be - al) / (2.0 * ga);
         const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
         const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
-        for (int i = lane; i < rows; i += 32) {
-          const double x = a[i], y = b[i];
-          a[i] = c * x - s * y;
-          b[i] = s * x + c * y;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+          const int i = sub + 16 * q;
+          if (i < rows) {
+            const double x = a[i], y = b[i];
+            a[i] = c * x - s * y;
+            b[i] = s * x + c * y;
+          }
         }
-        if (lane == 0) *flag = 1;
+        if (sub == 0) {
+          nrm[ia] = al - t * ga;
+          nrm[ib] = be + t * ga;
+          *flag = 1;
+        }
       }
       __syncthreads();
     }
@@ -124,14 +145,14 @@ __global__ void __launch_bounds__(kLinThreads) eigen_factor_kernel(Dims m, const
                                                                    double* F64, float* F32,
                                                                    int* err, int err_bit) {
   extern __shared__ double G[];          // [d][d] column-major
-  __shared__ double norm[kMaxD], lam[kMaxD], red[32];
+  __shared__ double norm[kMaxD], lam[kMaxD], red[32], hnrm[kMaxD];
   __shared__ int rank[kMaxD];
   __shared__ int flag;
   const int h = blockIdx.x, d = m.d;
   const double* Mh = Mall + (long long)h * d * d;
   for (int e = threadIdx.x; e < d * d; e += blockDim.x) G[e] = Mh[e];  // symmetric
   __syncthreads();
-  hestenes(G, d, d, &flag, red);
+  hestenes(G, d, d, &flag, red, hnrm);
   // The metrics are Gram matrices (symmetric PSD), so the converged column norms are the
   // eigenvalues; negative eigenvalues exist only at rounding level, where |lambda| and
   // the clamp to zero differ by far less than any distance that decides a label.
@@ -222,6 +243,7 @@ __global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
   extern __shared__ double S[];   // max(n*n, M*d) doubles
   __shared__ double red[32];
   __shared__ double sig[kMaxM];
+  __shared__ double hnrm[kMaxM];
   __shared__ int srank[kMaxM];
   __shared__ int flag, bad;
   const int h = blockIdx.x, d = m.d, M = m.M;
@@ -319,7 +341,7 @@ __global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
   } else {
     for (int e = threadIdx.x; e < M * d; e += blockDim.x) S[e] = Y[e];
     __syncthreads();
-    hestenes(S, d, M, &flag, red);
+    hestenes(S, d, M, &flag, red, hnrm);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     for (int p = warp; p < M; p += nwarps) {
       double s2 = 0.0;
@@ -365,6 +387,168 @@ __global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
   }
 }
 
+// Probe fit with every operand in shared memory (dual form, M <= d, and A, Y, S and the
+// M x M Gram fit): the same computation as fit_kernel, with B P formed as (B Psi) Psi^T
+// so no d x d product is needed.
+__global__ void __launch_bounds__(kLinThreads) fit_smem_kernel(Dims m, Buffers b) {
+  extern __shared__ double sm[];
+  __shared__ double red[32];
+  __shared__ double sig[kMaxM];
+  __shared__ double u[kMaxM];          // Jacobi norm scratch, then the fold's u
+  __shared__ int srank[kMaxM];
+  __shared__ int flag, bad;
+  const int h = blockIdx.x, d = m.d, M = m.M;
+  const long long hd = (long long)h * d;
+  double* A = sm;                 // [M][d] standardised, weighted features; later W = B Psi
+  double* Y = A + M * d;          // [M][d] centred, weighted residuals; then Z = G^-1 Y
+  double* S = Y + M * d;          // [M][d] columns of Y^T orthogonalised; then Psi
+  double* G = S + M * d;          // [M][M] A A^T + lambda I, then its Cholesky factor
+  const int* probes = b.probes + (long long)h * M;
+  const double* w = b.wP + (long long)h * M;
+  double wsum = 0.0;
+  for (int p = 0; p < M; ++p) wsum += w[p];
+  for (int e = threadIdx.x; e < M * d; e += blockDim.x) {
+    const int p = e / d, j = e % d;
+    const int pos = b.invQ[(long long)h * m.Nq + probes[p]];
+    const double x = (double)b.Osp[((long long)h * m.Nq + pos) * d + j];
+    const double dn = (double)b.Odense[((long long)h * M + p) * d + j];
+    A[e] = x;
+    Y[e] = dn - x;
+    if (!isfinite(x) || !isfinite(dn)) atomicOr(b.err, kErrNonFinite);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double mx = 0.0, mr = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const double wt = w[p] / wsum;
+      mx += wt * A[p * d + j];
+      mr += wt * Y[p * d + j];
+    }
+    double var = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const double t = A[p * d + j] - mx;
+      var += (w[p] / wsum) * t * t;
+    }
+    b.muX[hd + j] = mx;
+    b.muR[hd + j] = mr;
+    b.sX[hd + j] = sqrt(var + 1e-6);
+  }
+  __syncthreads();
+  const double* mux = b.muX + hd;
+  const double* mur = b.muR + hd;
+  const double* sdv = b.sX + hd;
+  for (int e = threadIdx.x; e < M * d; e += blockDim.x) {
+    const int p = e / d, j = e % d;
+    const double om = sqrt((double)M * w[p] / wsum);
+    A[e] = om * (A[e] - mux[j]) / sdv[j];
+    Y[e] = om * (Y[e] - mur[j]);
+    S[e] = Y[e];
+  }
+  __syncthreads();
+
+  // ---- residual subspace from the columns of Y^T
+  double* Ph = b.Pm + (long long)h * d * d;
+  int reff = d;
+  if (m.r > 0) {
+    hestenes(S, d, M, &flag, red, u);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int p = warp; p < M; p += nwarps) {
+      double s2 = 0.0;
+      for (int i = lane; i < d; i += 32) s2 += S[p * d + i] * S[p * d + i];
+      s2 = warp_sum(s2);
+      if (lane == 0) sig[p] = sqrt(s2);
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < M; p += blockDim.x) srank[p] = desc_rank(sig, M, p);
+    __syncthreads();
+    double smax = 0.0;
+    for (int p = 0; p < M; ++p) smax = sig[p] > smax ? sig[p] : smax;
+    int keep = 0;
+    if (smax > 0.0)
+      for (int p = 0; p < M; ++p) keep += sig[p] > 1e-10 * smax;
+    reff = m.r < keep ? m.r : keep;
+    for (int p = threadIdx.x; p < M; p += blockDim.x) b.sig[(long long)h * kMaxM + srank[p]] = sig[p];
+    // the kept columns, normalised in place, are the leading right singular vectors
+    for (int e = threadIdx.x; e < M * d; e += blockDim.x) {
+      const int p = e / d;
+      if (srank[p] < reff) S[e] /= sig[p];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+      const int i = e / d, j = e % d;
+      double v = 0.0;
+      for (int p = 0; p < M; ++p)
+        if (srank[p] < reff) v += S[p * d + i] * S[p * d + j];
+      Ph[e] = v;
+    }
+  } else {
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) Ph[e] = (e / d == e % d) ? 1.0 : 0.0;
+  }
+  if (threadIdx.x == 0) b.reff[h] = reff;
+  __syncthreads();
+
+  // ---- ridge, dual form: G = A A^T + lambda I, Z = G^-1 Y (in place), B = A^T Z
+  for (int e = threadIdx.x; e < M * M; e += blockDim.x) {
+    const int i = e / M, j = e % M;
+    double g = 0.0;
+    for (int k = 0; k < d; ++k) g += A[i * d + k] * A[j * d + k];
+    G[e] = g + (i == j ? m.lambda : 0.0);
+  }
+  __syncthreads();
+  const bool pd = cholesky(G, M, &bad);
+  if (!pd && threadIdx.x == 0) atomicOr(b.err, kErrNonFinite);
+  cholesky_solve(G, M, Y, d, d);
+  double* Bh = b.Bm + (long long)h * d * d;
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int i = e / d, j = e % d;
+    double v = 0.0;
+    if (pd)
+      for (int p = 0; p < M; ++p) v += A[p * d + i] * Y[p * d + j];
+    Bh[e] = v;
+  }
+  __syncthreads();
+
+  // ---- fold: B' = diag(1/s) B P, c = mu_R - (mu_x / s) B P, with B P = (B Psi) Psi^T
+  float* Bp = b.Bp + (long long)h * d * d;
+  if (m.r > 0) {
+    double* W = A;                 // [d][M]: column p holds B psi_p for kept p
+    for (int e = threadIdx.x; e < d * M; e += blockDim.x) {
+      const int i = e / M, p = e % M;
+      double v = 0.0;
+      if (srank[p] < reff)
+        for (int j = 0; j < d; ++j) v += Bh[i * d + j] * S[p * d + j];
+      W[e] = v;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < M; p += blockDim.x) {
+      double v = 0.0;
+      for (int i = 0; i < d; ++i) v += (mux[i] / sdv[i]) * W[i * M + p];
+      u[p] = v;
+    }
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+      const int i = e / d, j = e % d;
+      double v = 0.0;
+      for (int p = 0; p < M; ++p)
+        if (srank[p] < reff) v += W[i * M + p] * S[p * d + j];
+      Bp[e] = (float)(v / sdv[i]);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      double v = mur[j];
+      for (int p = 0; p < M; ++p)
+        if (srank[p] < reff) v -= u[p] * S[p * d + j];
+      b.cvec[hd + j] = (float)v;
+    }
+  } else {
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) Bp[e] = (float)(Bh[e] / sdv[e / d]);
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      double v = mur[j];
+      for (int i = 0; i < d; ++i) v -= (mux[i] / sdv[i]) * Bh[i * d + j];
+      b.cvec[hd + j] = (float)v;
+    }
+  }
+}
+
 }  // namespace
 
 sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st) {
@@ -387,6 +571,20 @@ sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st) 
 
 sparsepr_status launch_fit(const Plan& p, cudaStream_t st) {
   const int d = p.dm.d, M = p.dm.M;
+  // shared-memory path when the dual form applies and A, Y, S (M x d each) and the
+  // M x M Gram fit next to the kernel's static arrays
+  const size_t fast_smem = (size_t)(3 * M * d + M * M) * sizeof(double);
+  cudaFuncAttributes fa{};
+  int dev = 0, optin = 0;
+  SPR_CUDA_OK(cudaFuncGetAttributes(&fa, fit_smem_kernel));
+  SPR_CUDA_OK(cudaGetDevice(&dev));
+  SPR_CUDA_OK(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+  if (M <= d && fa.sharedSizeBytes + fast_smem <= (size_t)optin) {
+    SPR_CUDA_OK(cudaFuncSetAttribute(fit_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fast_smem));
+    fit_smem_kernel<<<p.dm.H, kLinThreads, fast_smem, st>>>(p.dm, p.b);
+    SPR_LAUNCH_OK();
+    return SPARSEPR_OK;
+  }
   const int n = M <= d ? M : d;
   const size_t smem = (size_t)((n * n > M * d) ? n * n : M * d) * sizeof(double);
   SPR_CUDA_OK(cudaFuncSetAttribute(fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

@@ -113,7 +113,10 @@ __global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
   __shared__ int sh[32];
   __shared__ int cut;
   const int h = blockIdx.y, a = blockIdx.x;
-  if (a >= b.nQ[h]) return;
+  if (a >= b.nQ[h]) {            // no such group: the count is defined as zero
+    if (threadIdx.x == 0) b.cellCnt[(long long)h * m.Cq + a] = 0;
+    return;
+  }
   const int n = b.nK[h];
   int P2 = 1;
   while (P2 < n) P2 <<= 1;
@@ -185,18 +188,18 @@ __global__ void gather_kernel(const void* src, void* dst, const int* perm, int* 
   }
 }
 
-// Squared distance of each query's phi_Q to its group centre (fp32, ascending dims).
+// Squared distance of each query's phi_Q to its group centre (fp64, ascending dims).
 __global__ void probe_dist_kernel(Dims m, Buffers b) {
   const int h = blockIdx.y;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= m.Nq) return;
   const int lab = b.labQ[(long long)h * m.Nq + i];
-  const float* x = b.phiQ + ((long long)h * m.Nq + i) * m.rQ;
-  const float* c = b.centQ + ((long long)h * m.Cq + lab) * m.rQ;
-  float s = 0.0f;
+  const double* x = b.phiQ + ((long long)h * m.Nq + i) * m.rQ;
+  const double* c = b.centQ + ((long long)h * m.Cq + lab) * m.rQ;
+  double s = 0.0;
   for (int k = 0; k < m.rQ; ++k) {
-    const float t = x[k] - c[k];
-    s = fmaf(t, t, s);
+    const double t = x[k] - c[k];
+    s = fma(t, t, s);
   }
   b.dist[(long long)h * m.Nq + i] = s;
 }
@@ -222,15 +225,15 @@ __global__ void __launch_bounds__(32) probe_rank_kernel(Dims m, Buffers b) {
   const int m0 = b.offQ[(long long)h * (m.Cq + 1) + lab], m1 = b.offQ[(long long)h * (m.Cq + 1) + lab + 1];
   const int take = (m1 - m0) < P ? (m1 - m0) : P;
   const int* perm = b.permQ + (long long)h * m.Nq;
-  const float* dist = b.dist + (long long)h * m.Nq;
-  float pd = -INFINITY;
+  const double* dist = b.dist + (long long)h * m.Nq;
+  double pd = -INFINITY;
   int pi = -1;
   for (int t = 0; t < take; ++t) {
-    float bd = INFINITY;
+    double bd = INFINITY;
     int bi = 0x7fffffff;
     for (int mm = m0 + lane; mm < m1; mm += 32) {
       const int row = perm[mm];
-      const float dv = dist[row];
+      const double dv = dist[row];
       const bool after = dv > pd || (dv == pd && row > pi);
       const bool better = dv < bd || (dv == bd && row < bi);
       if (after && better) {
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(32) probe_rank_kernel(Dims m, Buffers b) {
       }
     }
     for (int o = 16; o > 0; o >>= 1) {
-      const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+      const double od = __shfl_xor_sync(0xffffffffu, bd, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (od < bd || (od == bd && oi < bi)) {
         bd = od;

@@ -248,12 +248,12 @@ def _export_layout(p: sparsepr_params, name: str):
         "FACTOR_K": (f64, (H, d, p.r_K)), "FACTOR_Q": (f64, (H, d, p.r_Q)),
         "EIG_K": (f64, (H, p.r_K)), "EIG_Q": (f64, (H, p.r_Q)),
         "METRIC_K": (f64, (H, d, d)), "METRIC_Q": (f64, (H, d, d)),
-        "PHI_K": (f32, (H, p.N_k, p.r_K)), "PHI_Q": (f32, (H, p.N_q, p.r_Q)),
-        "CENTRES_Q": (f32, (H, p.C_q, p.r_Q)), "SCORES": (f64, (H, p.C_q, p.C_k)),
+        "PHI_K": (f64, (H, p.N_k, p.r_K)), "PHI_Q": (f64, (H, p.N_q, p.r_Q)),
+        "CENTRES_Q": (f64, (H, p.C_q, p.r_Q)), "SCORES": (f64, (H, p.C_q, p.C_k)),
         "OSP": (f32, (H, p.N_q, d)), "ODENSE_PROBE": (f32, (H, p.M, d)),
         "FIT_MU_X": (f64, (H, d)), "FIT_MU_R": (f64, (H, d)), "FIT_S": (f64, (H, d)),
         "FIT_B": (f64, (H, d, d)), "FIT_P": (f64, (H, d, d)), "FIT_REFF": (i32, (H,)),
-        "PROBE_DIST": (f32, (H, p.N_q)), "KBAR": (f64, (H, p.C_k, d)),
+        "PROBE_DIST": (f64, (H, p.N_q)), "KBAR": (f64, (H, p.C_k, d)),
         "QBAR": (f64, (H, p.C_q, d)),
     }[name]
 

@@ -221,9 +221,9 @@ typedef enum {
   SPARSEPR_X_EIG_Q = 18,      /* double [H,r_Q]  kept eigenvalues of M_Q */
   SPARSEPR_X_METRIC_K = 19,   /* double [H,d,d]  M_K */
   SPARSEPR_X_METRIC_Q = 20,   /* double [H,d,d]  M_Q */
-  SPARSEPR_X_PHI_K = 21,      /* float [H,N_k,r_K] key coordinates */
-  SPARSEPR_X_PHI_Q = 22,      /* float [H,N_q,r_Q] query coordinates */
-  SPARSEPR_X_CENTRES_Q = 23,  /* float [H,C_q,r_Q] query-group centres in phi_Q space (raw labels) */
+  SPARSEPR_X_PHI_K = 21,      /* double [H,N_k,r_K] key coordinates */
+  SPARSEPR_X_PHI_Q = 22,      /* double [H,N_q,r_Q] query coordinates */
+  SPARSEPR_X_CENTRES_Q = 23,  /* double [H,C_q,r_Q] query-group centres in phi_Q space (raw labels) */
   SPARSEPR_X_SCORES = 24,     /* double [H,C_q,C_k] routing scores (compact ids) */
   SPARSEPR_X_OSP = 25,        /* float [H,N_q,d] sparse output, group-major order */
   SPARSEPR_X_ODENSE_PROBE = 26,/* float [H,M,d]  exact output of the probe rows */
@@ -233,7 +233,7 @@ typedef enum {
   SPARSEPR_X_FIT_B = 30,      /* double [H,d,d] ridge coefficients B_lambda */
   SPARSEPR_X_FIT_P = 31,      /* double [H,d,d] projector Psi_r Psi_r^T */
   SPARSEPR_X_FIT_REFF = 32,   /* int32 [H]      rank kept in the projector */
-  SPARSEPR_X_PROBE_DIST = 33, /* float [H,N_q]  squared phi_Q distance to the group centre */
+  SPARSEPR_X_PROBE_DIST = 33, /* double [H,N_q] squared phi_Q distance to the group centre */
   SPARSEPR_X_KBAR = 34,       /* double [H,C_k,d] K/V group key centroids (compact ids) */
   SPARSEPR_X_QBAR = 35,       /* double [H,C_q,d] query group centroids (compact ids) */
   SPARSEPR_X_COUNT = 36

@@ -141,7 +141,7 @@ def test_tiny_injected_stagewise():
     FK = plan.export("FACTOR_K")[0]
     s = _align_signs(FK, part.F_K)
     assert rel(FK * s, part.F_K) < 1e-8
-    assert rel(plan.export("PHI_K")[0] * s, part.phiK) < 1e-5
+    assert rel(plan.export("PHI_K")[0] * s, part.phiK) < 1e-7
     # centroids, query metric, factor, coordinates
     nk, nq = part.gk.sizes.size, part.gq.sizes.size
     assert rel(plan.export("KBAR")[0][:nk], part.kbar) < 1e-13
@@ -150,10 +150,10 @@ def test_tiny_injected_stagewise():
     FQ = plan.export("FACTOR_Q")[0]
     sq = _align_signs(FQ, part.F_Q)
     assert rel(FQ * sq, part.F_Q) < 1e-8
-    assert rel(plan.export("PHI_Q")[0] * sq, part.phiQ) < 1e-5
+    assert rel(plan.export("PHI_Q")[0] * sq, part.phiQ) < 1e-7
     # routing scores (fp64), then indexing bit-exact and output
     assert rel(plan.export("SCORES")[0][:nq, :nk], res.scores) < 1e-12
-    assert rel(plan.export("PROBE_DIST")[0], res.probe_dist) < 1e-5
+    assert rel(plan.export("PROBE_DIST")[0], res.probe_dist) < 1e-7
     perm = plan.export("PERM_Q")[0]
     osp = plan.export("OSP")[0]
     osp_rows = np.empty_like(osp)
@@ -383,3 +383,17 @@ def test_out_of_range_injected_labels_are_flagged():
     labK[0, 5] = w.C_k + 3
     plan = N.Plan(N.params_from_dict(w.params()), Q, K, V, labels=(labQ, labK))
     assert plan.check() & 16
+
+
+@pytest.mark.parametrize("case", ["mid", "wan2", "ragged"])
+def test_tensor_core_kmeans_equals_full_scan(case):
+    # The tensor-core assignment (bf16 split scores + exact rescoring of near ties) must
+    # give the same labels, objectives and iteration counts as the fp32 full scan.
+    w = {"mid": W.MID.with_(H=3), "wan2": W.WAN.with_(H=2),
+         "ragged": W.TINY.with_(N=1000, grid=(10, 10, 10), C_q=100, C_k=70, M=16)}[case]
+    inputs = W.make_inputs_torch(w, device="cuda")
+    p_tc = N.Plan(N.params_from_dict(w.params()), *inputs)
+    p_ct = N.Plan(N.params_from_dict(w.params(), N.SPARSEPR_ENGINE_SIMT), *inputs)
+    assert p_tc.check() == 0 and p_ct.check() == 0
+    for name in ("LABELS_K", "LABELS_Q", "KMEANS_ITERS", "OBJECTIVE", "PERM_Q", "CELL_COUNT"):
+        assert np.array_equal(p_tc.export(name), p_ct.export(name)), name
