@@ -64,19 +64,22 @@ struct TcArgs {
   int* err;
 };
 
+// Shared memory: two Q tiles, then S stages of K tiles and S stages of V tiles (four
+// stages at d = 64, where the tiles are small; two at d = 128), then bookkeeping.
 template <int D>
 struct Layout {
+  static constexpr int S = D == 64 ? 4 : 2;
   static constexpr uint32_t kTile = kTileRows * D * 2;         // bytes of a Q/K/V tile
   static constexpr uint32_t kPanel = kTileRows * 128;          // one 64-column panel
-  static constexpr uint32_t oQ0 = 0, oQ1 = kTile;
-  static constexpr uint32_t oK0 = 2 * kTile, oK1 = 3 * kTile;
-  static constexpr uint32_t oV0 = 4 * kTile, oV1 = 5 * kTile;
-  static constexpr uint32_t oMisc = 6 * kTile;
+  static constexpr uint32_t oQ0 = 0;
+  static constexpr uint32_t oK0 = 2 * kTile;
+  static constexpr uint32_t oV0 = (2 + S) * kTile;
+  static constexpr uint32_t oMisc = (2 + 2 * S) * kTile;
   static constexpr uint32_t kBytes = oMisc + 14 * 1024;
 };
 
 struct Misc {
-  unsigned long long bars[16];
+  unsigned long long bars[24];
   long long qrow[kItemRows];
   long long krow[2][kTileKeys];
   int csum[kMaxC + 1];
@@ -87,7 +90,7 @@ struct Misc {
 };
 
 enum Bar {
-  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 3, bSFull0 = 5, bPFull0 = 7, bPvDone0 = 9, bDrain = 11, bOReady = 12
+  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 5, bSFull0 = 9, bPFull0 = 11, bPvDone0 = 13, bDrain = 15, bOReady = 16
 };
 
 // Bounded wait; the clock and the abort flag are read once every 32 polls so that
@@ -173,9 +176,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   auto BAR = [&](int i) -> uint32_t { return bars + 8u * i; };
   if (tid == 0) {
     tc::mbar_init(BAR(bQFull), kProducers);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(BAR(bKVFull0 + s), kProducers);
+    for (int s = 0; s < L::S; ++s) {
+      tc::mbar_init(BAR(bKVFull0 + s), kProducers);   // one cp.async completion per producer
       tc::mbar_init(BAR(bKVEmpty0 + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(BAR(bSFull0 + s), 1);
       tc::mbar_init(BAR(bPFull0 + s), 128);
       tc::mbar_init(BAR(bPvDone0 + s), 1);
@@ -222,43 +227,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
     tc::mbar_arrive(BAR(bQFull));
+    // K/V tiles: stage j % S.  Each producer's copies arrive on the stage's barrier when
+    // they complete (cp.async.mbarrier.arrive.noinc), so the producers move on to the next
+    // free stage without waiting for the data; the MMA thread fences the generic-proxy
+    // writes against its tensor-core reads after the barrier.
+    int cur0 = 0, cur1 = 0;             // cells of this thread's two keys (non-decreasing)
     for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
+      const int s = j % L::S, use = j / L::S;
       // every producer thread takes the same decision (they meet at named barriers)
-      const bool got = j < 2 || wait_bar(ms, BAR(bKVEmpty0 + s), ((j >> 1) + 1) & 1, g.err);
+      const bool got = use == 0 || wait_bar(ms, BAR(bKVEmpty0 + s), (use - 1) & 1, g.err);
       if (!tc::named_sync_and(1, kProducers, got)) break;
-      for (int kk = p; kk < kTileKeys; kk += kProducers) {
-      const long long v = (long long)j * kTileKeys + kk;
-      long long kr = -1;
-      if (v < nkeys) {
-        if (g.mode == kModeSparse) {
-          int lo = 0, hi = cnt - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (ms->csum[mid] <= v) lo = mid; else hi = mid - 1;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int kk = p + q * kProducers;
+        if (kk >= kTileKeys) break;
+        const long long v = (long long)j * kTileKeys + kk;
+        long long kr = -1;
+        if (v < nkeys) {
+          if (g.mode == kModeSparse) {
+            int c = q ? cur1 : cur0;
+            while (ms->csum[c + 1] <= v) ++c;     // csum[cnt] = nkeys > v ends the walk
+            if (q) cur1 = c; else cur0 = c;
+            kr = hk + ((long long)ms->cbase[c] + (v - ms->csum[c])) * d;
+          } else if (g.mode == kModeDense) {
+            kr = hk + v * d;
+          } else {
+            kr = hk + ((long long)split * kProbeSplit + v) * d;
           }
-          kr = hk + ((long long)ms->cbase[lo] + (v - ms->csum[lo])) * d;
-        } else if (g.mode == kModeDense) {
-          kr = hk + v * d;
-        } else {
-          kr = hk + ((long long)split * kProbeSplit + v) * d;
         }
-      }
-      ms->krow[s][kk] = kr;
+        ms->krow[j & 1][kk] = kr;
       }
       tc::named_sync(1, kProducers);
       for (int e = p; e < kTileKeys * CPR; e += kProducers) {
         const int row = e / CPR, c = e % CPR;
-        const long long off = ms->krow[s][row];
+        const long long off = ms->krow[j & 1][row];
         const uint32_t o = (c >> 3) * L::kPanel + tc::sw128_offset(row, c & 7);
         const bool ok = off >= 0;
         tc::cp_async16(sK(s) + o, ok ? (const void*)(g.K + off + c * 8) : (const void*)g.K, ok ? 16u : 0u);
         tc::cp_async16(sV(s) + o, ok ? (const void*)(g.V + off + c * 8) : (const void*)g.V, ok ? 16u : 0u);
       }
-      tc::cp_async_commit();
-      tc::cp_async_wait_all();
-      tc::fence_proxy_async();
-      tc::mbar_arrive(BAR(bKVFull0 + s));
+      tc::cp_async_arrive_noinc(BAR(bKVFull0 + s));
     }
     tc::cp_async_wait_all();
   } else if (warp == 11) {
@@ -268,7 +276,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       constexpr uint32_t idPV = tc::idesc_bf16_f32(kTileRows, D, true);
       // S of query tile t against key tile j into S buffer `buf` (TMEM columns 128 buf)
       auto issue_s = [&](int t, int j, int buf) {
-        const int s = j & 1;
+        const int s = j % L::S;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = tc::sw128_desc(sQ(t) + (kk >> 2) * L::kPanel + (kk & 3) * 32, 16, 1024);
@@ -279,7 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       };
       // O_t += P V_j with P in S buffer `buf`
       auto issue_pv = [&](int t, int j, int buf) {
-        const int s = j & 1;
+        const int s = j % L::S;
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk) {
           const uint64_t bd = tc::sw128_desc(sV(s) + kk * 2048, L::kPanel, 1024);
@@ -287,7 +295,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         }
         tc::mma_commit(BAR(bPvDone0 + t));
       };
-      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && wait_bar(ms, BAR(bKVFull0), 0, g.err);
+      // K/V stage j % S, fill j / S; the copies were made by the generic proxy
+      auto kv_ready = [&](int j) -> bool {
+        if (!wait_bar(ms, BAR(bKVFull0 + j % L::S), (j / L::S) & 1, g.err)) return false;
+        tc::fence_proxy_async();
+        return true;
+      };
+      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && kv_ready(0);
       if (hasB) {
         // two query tiles: the softmax of one overlaps the products of the other
         if (ok) {
@@ -301,14 +315,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           issue_pv(0, j, 0);
           const bool more = j + 1 < nt;
           if (more) {
-            if (!wait_bar(ms, BAR(bKVFull0 + ((j + 1) & 1)), ((j + 1) >> 1) & 1, g.err)) { ok = false; break; }
+            if (!kv_ready(j + 1)) { ok = false; break; }
             tc::fence_after_sync();
             issue_s(0, j + 1, 0);
           }
           if (!wait_bar(ms, BAR(bPFull0 + 1), j & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
           issue_pv(1, j, 1);
-          tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
+          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
           if (more) issue_s(1, j + 1, 1);
         }
       } else {
@@ -318,7 +332,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           tc::fence_after_sync();
           issue_s(0, 0, 0);
           if (nt > 1) {
-            ok = wait_bar(ms, BAR(bKVFull0 + 1), 0, g.err);
+            ok = kv_ready(1);
             if (ok) {
               tc::fence_after_sync();
               issue_s(0, 1, 1);
@@ -330,9 +344,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           if (!wait_bar(ms, BAR(bPFull0 + buf), (j >> 1) & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
           issue_pv(0, j, buf);
-          tc::mma_commit(BAR(bKVEmpty0 + (j & 1)));
+          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
           if (j + 2 < nt) {
-            if (!wait_bar(ms, BAR(bKVFull0 + (j & 1)), ((j + 2) >> 1) & 1, g.err)) { ok = false; break; }
+            if (!kv_ready(j + 2)) { ok = false; break; }
             tc::fence_after_sync();
             issue_s(0, j + 2, buf);
           }

@@ -44,21 +44,23 @@ KmView view(const Plan& p, bool query) {
 // Response coordinates in fp64: phi = X F (keys), phi = z / max(rms(z), 1e-6) with
 // z = X F (queries) (paper S4.1, App. B.1-B.2).  X is exact in its dtype; F is the fp64
 // factor; each coordinate is one fp64 dot product over d in ascending order.
-// A block takes 64 rows; thread (row, q) forms coordinates q*R/4 .. (q+1)*R/4 - 1 of its
-// row from the row staged in shared memory and F staged once per block.  When the
-// tensor-core k-means will cluster these coordinates, the block also writes its input:
-// each row split into two bf16 pieces (rows padded to 64 columns, zero rows up to Npad)
-// and |phi|.
+// A block takes 64 rows: X is staged transposed (column j of the tile contiguous), F once
+// per block; thread (tr, tc) forms rows 4tr..4tr+3 x columns tc, tc+16, ... (a register
+// tile, so every shared-memory value feeds several fp64 FMAs and the 16 column threads
+// of a row group read 16 consecutive F values).  When the tensor-core k-means will
+// cluster these coordinates, the block also writes its input: each row split into two
+// bf16 pieces (rows padded to 64 columns, zero rows up to Npad) and |phi|.
 constexpr int kProjRows = 64;
+constexpr int kProjXs = kProjRows + 4;     // transposed tile row stride (floats)
 template <int R, bool RMS>
 __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int N, const double* Fall, int r,
                                                       double* out, __nv_bfloat16* xhi, __nv_bfloat16* xlo,
                                                       float* xn, int Npad) {
-  constexpr int P = R / 4;                 // coordinates per thread
+  constexpr int CPT = R / 16;              // columns per thread
   extern __shared__ double smd[];
   const int d = m.d, h = blockIdx.y;
   double* F = smd;                         // [d][R], zero columns k >= r
-  float* T = reinterpret_cast<float*>(smd + d * R);   // [64][d + 1]
+  float* Xt = reinterpret_cast<float*>(smd + d * R);  // [d][kProjXs]: Xt[j][row]
   const double* Fh = Fall + (long long)h * d * r;
   for (int e = threadIdx.x; e < d * R; e += blockDim.x) {
     const int j = e / R, k = e % R;
@@ -69,67 +71,70 @@ __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int
   for (int e = threadIdx.x; e < kProjRows * d; e += blockDim.x) {
     const int i = e / d, j = e % d;
     const long long row = row0 + i;
-    T[i * (d + 1) + j] = row < N ? load_as_float(X, base + row * d + j, m.dtype) : 0.0f;
+    Xt[j * kProjXs + i] = row < N ? load_as_float(X, base + row * d + j, m.dtype) : 0.0f;
   }
   __syncthreads();
-  const int ri = threadIdx.x >> 2, q = threadIdx.x & 3;
-  const long long row = row0 + ri;
-  double acc[P];
+  const int tr = threadIdx.x >> 4, tc = threadIdx.x & 15;
+  double acc[4][CPT];
 #pragma unroll
-  for (int k = 0; k < P; ++k) acc[k] = 0.0;
-  const float* x = T + ri * (d + 1);
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[a][c] = 0.0;
   for (int j = 0; j < d; ++j) {
-    const double xv = (double)x[j];
-    const double2* f2 = reinterpret_cast<const double2*>(F + j * R + q * P);
+    const float4 x4 = *reinterpret_cast<const float4*>(Xt + j * kProjXs + 4 * tr);
+    const double xv[4] = {(double)x4.x, (double)x4.y, (double)x4.z, (double)x4.w};
+    double fv[CPT];
 #pragma unroll
-    for (int k = 0; k < P / 2; ++k) {
-      const double2 f = f2[k];
-      acc[2 * k] = fma(xv, f.x, acc[2 * k]);
-      acc[2 * k + 1] = fma(xv, f.y, acc[2 * k + 1]);
-    }
+    for (int c = 0; c < CPT; ++c) fv[c] = F[j * R + tc + 16 * c];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) acc[a][c] = fma(xv[a], fv[c], acc[a][c]);
   }
-  // the row's four threads are adjacent lanes: sums over the row by shuffles in a fixed order
+  // the 16 column threads of a row group are one half-warp: row sums by shuffles
   auto row_sum = [](double v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
   };
-  double scale = 1.0;
-  if (RMS) {
-    double ss = 0.0;
 #pragma unroll
-    for (int k = 0; k < P; ++k) ss = fma(acc[k], acc[k], ss);
-    ss = row_sum(ss);
-    scale = 1.0 / fmax(sqrt(ss / (double)r), 1e-6);
-  }
+  for (int a = 0; a < 4; ++a) {
+    const long long row = row0 + 4 * tr + a;
+    if (RMS) {
+      double ss = 0.0;
 #pragma unroll
-  for (int k = 0; k < P; ++k) acc[k] = RMS ? acc[k] * scale : acc[k];
-  if (row < N) {
-    double* o = out + ((long long)h * N + row) * r;
+      for (int c = 0; c < CPT; ++c) ss = fma(acc[a][c], acc[a][c], ss);
+      ss = row_sum(ss);
+      const double scale = 1.0 / fmax(sqrt(ss / (double)r), 1e-6);
 #pragma unroll
-    for (int k = 0; k < P; ++k)
-      if (q * P + k < r) o[q * P + k] = acc[k];
-  }
-  if (xhi) {
-    double ss = 0.0;
+      for (int c = 0; c < CPT; ++c) acc[a][c] *= scale;
+    }
+    if (row < N) {
+      double* o = out + ((long long)h * N + row) * r;
 #pragma unroll
-    for (int k = 0; k < P; ++k) ss = fma(acc[k], acc[k], ss);
-    ss = row_sum(ss);
-    if (row < Npad) {
-      const long long xb = ((long long)h * Npad + row) * 64;
+      for (int c = 0; c < CPT; ++c)
+        if (tc + 16 * c < r) o[tc + 16 * c] = acc[a][c];
+    }
+    if (xhi) {
+      double ss = 0.0;
 #pragma unroll
-      for (int k = 0; k < P; ++k) {
-        const double v = row < N ? acc[k] : 0.0;
-        const __nv_bfloat16 hi = __double2bfloat16(v);
-        xhi[xb + q * P + k] = hi;
-        xlo[xb + q * P + k] = __double2bfloat16(v - (double)__bfloat162float(hi));
-      }
-      if (q == 3)
-        for (int k = R; k < 64; ++k) {
-          xhi[xb + k] = __float2bfloat16_rn(0.0f);
-          xlo[xb + k] = __float2bfloat16_rn(0.0f);
+      for (int c = 0; c < CPT; ++c) ss = fma(acc[a][c], acc[a][c], ss);
+      ss = row_sum(ss);
+      if (row < Npad) {
+        const long long xb = ((long long)h * Npad + row) * 64;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          const double v = row < N ? acc[a][c] : 0.0;
+          const __nv_bfloat16 hi = __double2bfloat16(v);
+          xhi[xb + tc + 16 * c] = hi;
+          xlo[xb + tc + 16 * c] = __double2bfloat16(v - (double)__bfloat162float(hi));
         }
-      if (q == 0 && row < N) xn[(long long)h * N + row] = (float)sqrt(ss);
+        for (int cz = R + tc; cz < 64; cz += 16) {
+          xhi[xb + cz] = __float2bfloat16_rn(0.0f);
+          xlo[xb + cz] = __float2bfloat16_rn(0.0f);
+        }
+        if (tc == 0 && row < N) xn[(long long)h * N + row] = (float)sqrt(ss);
+      }
     }
   }
 }
@@ -141,13 +146,12 @@ sparsepr_status launch_project(const Plan& p, const void* X, int N, const double
   const int rows = xhi ? Npad : N;
   dim3 grid(cdiv(rows, kProjRows), p.dm.H);
   auto run = [&](auto kern, int R) -> sparsepr_status {
-    const size_t smem = (size_t)d * R * sizeof(double) + (size_t)kProjRows * (d + 1) * sizeof(float);
+    const size_t smem = (size_t)d * R * sizeof(double) + (size_t)d * kProjXs * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    kern<<<grid, 4 * kProjRows, smem, st>>>(p.dm, X, N, F, r, out, xhi, xlo, xn, Npad);
+    kern<<<grid, 256, smem, st>>>(p.dm, X, N, F, r, out, xhi, xlo, xn, Npad);
     SPR_LAUNCH_OK();
     return SPARSEPR_OK;
   };
-  if (r <= 8) return run(project_kernel<8, RMS>, 8);
   if (r <= 16) return run(project_kernel<16, RMS>, 16);
   if (r <= 32) return run(project_kernel<32, RMS>, 32);
   if (r <= 48) return run(project_kernel<48, RMS>, 48);

@@ -261,6 +261,20 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
     const float BIG = 3.402823466e38f;
     int J = 0;
     int nfull0 = 0, nfull1 = 0;            // waits done on accFull[0][grp], accFull[1][grp]
+    // per-point values of this group's next tile, loaded one tile ahead of their use
+    ActiveHeads pre{g.km, -1, -1};
+    float nxn = 0.0f, ncm = 0.0f;
+    int nold = 0;
+    auto point_vals = [&](int li2) {
+      const long long t2 = t0 + li2;
+      const int h2 = pre.head((int)(t2 / tph));
+      const int row2 = (int)(t2 % tph) * kRows + r;
+      const long long pi2 = (long long)h2 * g.N + (row2 < g.N ? row2 : 0);
+      nxn = g.xn[pi2];
+      nold = g.lab[pi2];
+      ncm = sqrtf(__int_as_float(g.cmaxb[(g.it & 1) * g.H + h2]));
+    };
+    if (grp < ntiles) point_vals(grp);
     for (int li = 0; li < ntiles; ++li) {
       const long long t = t0 + li;
       const int h = act.head((int)(t / tph));
@@ -269,9 +283,9 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       const int row = (int)(t % tph) * kRows + r;
       const bool live = row < g.N;
       const long long pi = (long long)h * g.N + (live ? row : 0);
-      const float xn = g.xn[pi];
-      const int old = g.lab[pi];
-      const float cm = sqrtf(__int_as_float(g.cmaxb[(g.it & 1) * g.H + h]));
+      const float xn = nxn, cm = ncm;
+      const int old = nold;
+      if (li + 2 < ntiles) point_vals(li + 2);
       const float* cnh = g.cn + (long long)h * g.Cpad;
       float a0 = BIG, a1 = BIG;            // smallest and second smallest score
       int c0 = 0;                           // centre of the smallest (first one on ties)
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
         // rows ambiguous so far: this chunk's centres within T of the running best
         const bool need = live && a1 <= a0 + T;
         if (__any_sync(0xffffffffu, need)) {
-          const float lim = a0 + T;
+          const float lim = need ? a0 + T : -BIG;     // rows that need nothing match nothing
 #pragma unroll 1
           for (int q = 0; q < g.Cw; q += 64) {
             const int cb = c * kChunk + q;
@@ -333,20 +347,30 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
             tc::tmem_ld32(acc + q, *reinterpret_cast<float(*)[32]>(v));
             tc::tmem_ld32(acc + q + 32, *reinterpret_cast<float(*)[32]>(v + 32));
             tc::tmem_wait_ld();
+            // bit i of (m0, m1): column cb + i lies within the bound (branch-free)
+            uint32_t m0 = 0, m1 = 0;
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
               const float cv[4] = {cq[i4].x, cq[i4].y, cq[i4].z, cq[i4].w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const float a = fmaf(-2.0f, v[4 * i4 + e], cv[e]);
-                const int ci = cb + 4 * i4 + e;
-                if (need && a <= lim && ci != c0) {
-                  if (nrec == 0) rk0 = ci;
-                  else if (nrec == 1) rk1 = ci;
-                  else if (nrec == 2) rk2 = ci;
-                  else if (nrec == 3) rk3 = ci;
-                  ++nrec;
-                }
+                const int i = 4 * i4 + e;
+                const uint32_t hit = fmaf(-2.0f, v[i], cv[e]) <= lim ? 1u : 0u;
+                if (i < 32) m0 |= hit << i;
+                else m1 |= hit << (i - 32);
+              }
+            }
+            while (m0 | m1) {                   // a few columns, on the ambiguous rows only
+              int b;
+              if (m0) { b = __ffs(m0) - 1; m0 &= m0 - 1; }
+              else { b = 31 + __ffs(m1); m1 &= m1 - 1; }
+              const int ci = cb + b;
+              if (ci != c0) {
+                if (nrec == 0) rk0 = ci;
+                else if (nrec == 1) rk1 = ci;
+                else if (nrec == 2) rk2 = ci;
+                else if (nrec == 3) rk3 = ci;
+                ++nrec;
               }
             }
           }

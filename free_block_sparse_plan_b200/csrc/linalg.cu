@@ -94,19 +94,23 @@ __device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red,
         if (ia >= ncols || ib >= ncols) continue;     // uniform over the 16 lanes
         double* a = G + (long long)ia * rows;
         double* b = G + (long long)ib * rows;
-        double ga = 0.0;
+        double g0 = 0.0, g1 = 0.0;            // two chains: half the dependent latency
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) {
+        for (int q = 0; q < kPer; q += 2) {
           const int i = sub + 16 * q;
-          if (i < rows) ga += a[i] * b[i];
+          if (i < rows) g0 = fma(a[i], b[i], g0);
+          if (i + 16 < rows) g1 = fma(a[i + 16], b[i + 16], g1);
         }
+        double ga = g0 + g1;
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) ga += __shfl_xor_sync(half, ga, o);
         const double al = nrm[ia], be = nrm[ib];
-        if (ga == 0.0 || fabs(ga) <= 1e-14 * sqrt(al * be) || fabs(ga) <= abs_tol) continue;
-        const double zeta = (be - al) / (2.0 * ga);
-        const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-        const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
+        if (ga == 0.0 || ga * ga <= 1e-28 * (al * be) || fabs(ga) <= abs_tol) continue;
+        // t = tan of the angle that zeroes a.b: with u = |b|^2 - |a|^2 and v = 2 a.b,
+        // t = sign(u) v / (|u| + sqrt(u^2 + v^2)) (the smaller root of t^2 v + 2tu - v = 0)
+        const double u = be - al, v = 2.0 * ga;
+        const double t = copysign(1.0, u) * v / (fabs(u) + sqrt(fma(u, u, v * v)));
+        const double c = rsqrt(fma(t, t, 1.0)), s = c * t;
 #pragma unroll
         for (int q = 0; q < kPer; ++q) {
           const int i = sub + 16 * q;

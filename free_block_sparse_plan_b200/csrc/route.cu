@@ -19,89 +19,143 @@ namespace {
 // Routing score of every (query group a, K/V group b) cell, fp64.  For b other than the
 // largest-mass group, vbar_b - ohat^(-b) = (vbar_b - ohat) / (1 - pi_b) exactly, with
 // 1 - pi_b >= 1/2; for the largest-mass group ohat^(-b) is formed from the others.
+// A block scores kScoreQ query groups, so every K/V centroid row it streams through
+// shared memory (32 rows at a time, rows padded to d + 1 doubles so the 32 rows read by a
+// warp fall in distinct banks) serves all of them: logits, then per query group the two
+// softmax weightings, then the value mixtures, then the distances.
+constexpr int kScoreQ = 8;          // query groups per block (one warp each in phase 2)
+constexpr int kScoreK = 32;         // centroid rows per shared-memory chunk
 __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
-  __shared__ double qa[kMaxD], oh[kMaxD], orest[kMaxD];
-  __shared__ double zz[kMaxC], zr[kMaxC];
-  __shared__ double red[32];
-  __shared__ int redi[32];
-  const int h = blockIdx.y, a = blockIdx.x, d = m.d;
-  if (a >= b.nQ[h]) return;
+  extern __shared__ double ssm[];
+  __shared__ double sZ[kScoreQ], sZr[kScoreQ];
+  __shared__ int sTop[kScoreQ];
+  const int h = blockIdx.y, a0 = blockIdx.x * kScoreQ, d = m.d, ld = d + 1;
+  const int nq = b.nQ[h];
+  if (a0 >= nq) return;
+  const int na = min(kScoreQ, nq - a0);
   const int n = b.nK[h];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double* out0 = b.scores + ((long long)h * m.Cq + a0) * m.Ck;
+  if (n == 1) {
+    if (tid < na) out0[(long long)tid * m.Ck] = 0.0;
+    return;
+  }
+  double* qa = ssm;                       // [kScoreQ][ld] qbar, later ohat
+  double* orr = qa + kScoreQ * ld;        // [kScoreQ][ld] ohat over the others
+  double* kv = orr + kScoreQ * ld;        // [kScoreK][ld] chunk of kbar or vbar rows
+  double* zz = kv + kScoreK * ld;         // [kScoreQ][n] logits, then exp(l - max)
+  double* zr = zz + kScoreQ * n;          // [kScoreQ][n] exp(l - second max), 0 at the top
   const double tau = 1.0 / sqrt((double)d);
   const double* kb = b.kbar + (long long)h * m.Ck * d;
   const double* vb = b.vbar + (long long)h * m.Ck * d;
   const int* sz = b.sizeK + (long long)h * m.Ck;
-  double* out = b.scores + ((long long)h * m.Cq + a) * m.Ck;
-  if (n == 1) {
-    if (threadIdx.x == 0) out[0] = 0.0;
-    return;
+  for (int e = tid; e < kScoreQ * d; e += blockDim.x) {
+    const int a = e / d, j = e % d;
+    qa[a * ld + j] = a < na ? b.qbar[((long long)h * m.Cq + a0 + a) * d + j] : 0.0;
   }
-  for (int j = threadIdx.x; j < d; j += blockDim.x) qa[j] = b.qbar[((long long)h * m.Cq + a) * d + j];
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int k = warp; k < n; k += nw) {      // logits, kept in zr for now
-    double s = 0.0;
-    for (int j = lane; j < d; j += 32) s += qa[j] * kb[(long long)k * d + j];
-    s = warp_sum(s);
-    if (lane == 0) zr[k] = tau * s + log((double)sz[k]);
-  }
-  __syncthreads();
-  // largest logit and its first index; then the largest among the others
-  double mx = -INFINITY;
-  int top = 0x7fffffff;
-  for (int k = threadIdx.x; k < n; k += blockDim.x)
-    if (zr[k] > mx || (zr[k] == mx && k < top)) { mx = zr[k]; top = k; }
-  for (int o = 16; o > 0; o >>= 1) {
-    const double om = __shfl_xor_sync(0xffffffffu, mx, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, top, o);
-    if (om > mx || (om == mx && oi < top)) { mx = om; top = oi; }
-  }
-  if (lane == 0) { red[warp] = mx; redi[warp] = top; }
-  __syncthreads();
-  mx = red[0];
-  top = redi[0];
-  for (int w = 1; w < nw; ++w)
-    if (red[w] > mx || (red[w] == mx && redi[w] < top)) { mx = red[w]; top = redi[w]; }
-  __syncthreads();
-  double m2 = -INFINITY;
-  for (int k = threadIdx.x; k < n; k += blockDim.x)
-    if (k != top) m2 = fmax(m2, zr[k]);
-  for (int o = 16; o > 0; o >>= 1) m2 = fmax(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-  if (lane == 0) red[warp] = m2;
-  __syncthreads();
-  m2 = red[0];
-  for (int w = 1; w < nw; ++w) m2 = fmax(m2, red[w]);
-  __syncthreads();
-  double pz = 0.0, pr = 0.0;
-  for (int k = threadIdx.x; k < n; k += blockDim.x) {
-    const double l = zr[k];
-    zz[k] = exp(l - mx);
-    zr[k] = (k == top) ? 0.0 : exp(l - m2);
-    pz += zz[k];
-    pr += zr[k];
-  }
-  const double Z = block_sum(pz, red);
-  const double Zr = block_sum(pr, red);
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    double s = 0.0, t = 0.0;
-    for (int k = 0; k < n; ++k) {
-      const double v = vb[(long long)k * d + j];
-      s += zz[k] * v;
-      t += zr[k] * v;
+  auto stage = [&](const double* src, int k0) {
+    __syncthreads();
+    for (int e = tid; e < kScoreK * d; e += blockDim.x) {
+      const int kk = e / d, j = e % d;
+      kv[kk * ld + j] = k0 + kk < n ? src[(long long)(k0 + kk) * d + j] : 0.0;
     }
-    oh[j] = s / Z;
-    orest[j] = t / Zr;
+    __syncthreads();
+  };
+  const int ta = tid >> 5, tk = tid & 31;   // phases 1 and 4: thread = (query group, row)
+  // ---- phase 1: logits l_ab = tau qbar_a . kbar_b + ln |G_b|
+  for (int k0 = 0; k0 < n; k0 += kScoreK) {
+    stage(kb, k0);
+    const int k = k0 + tk;
+    if (ta < na && k < n) {
+      double s = 0.0;
+      for (int j = 0; j < d; ++j) s = fma(qa[ta * ld + j], kv[tk * ld + j], s);
+      zz[ta * n + k] = tau * s + log((double)sz[k]);
+    }
   }
   __syncthreads();
-  for (int k = warp; k < n; k += nw) {
-    const double* ref = (k == top) ? orest : oh;
-    double s = 0.0;
-    for (int j = lane; j < d; j += 32) {
-      const double t = vb[(long long)k * d + j] - ref[j];
-      s += t * t;
+  // ---- phase 2 (warp a): largest logit (first index), largest among the others, weights
+  if (warp < na) {
+    double* la = zz + warp * n;
+    double* ra = zr + warp * n;
+    double mx = -INFINITY;
+    int top = 0x7fffffff;
+    for (int k = lane; k < n; k += 32)
+      if (la[k] > mx || (la[k] == mx && k < top)) { mx = la[k]; top = k; }
+    for (int o = 16; o > 0; o >>= 1) {
+      const double om = __shfl_xor_sync(0xffffffffu, mx, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, top, o);
+      if (om > mx || (om == mx && oi < top)) { mx = om; top = oi; }
     }
-    s = warp_sum(s);
-    if (lane == 0) out[k] = (k == top) ? (zz[k] / Z) * sqrt(s) : zz[k] * sqrt(s) / (Z - zz[k]);
+    double m2 = -INFINITY;
+    for (int k = lane; k < n; k += 32)
+      if (k != top) m2 = fmax(m2, la[k]);
+    for (int o = 16; o > 0; o >>= 1) m2 = fmax(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    double pz = 0.0, pr = 0.0;
+    for (int k = lane; k < n; k += 32) {
+      const double l = la[k];
+      const double e1 = exp(l - mx), e2 = (k == top) ? 0.0 : exp(l - m2);
+      la[k] = e1;
+      ra[k] = e2;
+      pz += e1;
+      pr += e2;
+    }
+    pz = warp_sum(pz);
+    pr = warp_sum(pr);
+    if (lane == 0) {
+      sZ[warp] = pz;
+      sZr[warp] = pr;
+      sTop[warp] = top;
+    }
+  }
+  // ---- phase 3: ohat_a = sum_b zz_ab vbar_b / Z_a, and over b != top with zr
+  constexpr int kJ = kMaxD / 32;
+  double acc_h[kJ], acc_r[kJ];
+#pragma unroll
+  for (int i = 0; i < kJ; ++i) acc_h[i] = acc_r[i] = 0.0;
+  for (int k0 = 0; k0 < n; k0 += kScoreK) {
+    stage(vb, k0);
+    if (ta < na) {
+      const int kn = min(kScoreK, n - k0);
+      for (int kk = 0; kk < kn; ++kk) {
+        const double w1 = zz[ta * n + k0 + kk], w2 = zr[ta * n + k0 + kk];
+#pragma unroll
+        for (int i = 0; i < kJ; ++i) {
+          const int j = tk + 32 * i;
+          if (j < d) {
+            const double v = kv[kk * ld + j];
+            acc_h[i] = fma(w1, v, acc_h[i]);
+            acc_r[i] = fma(w2, v, acc_r[i]);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (ta < na) {
+#pragma unroll
+    for (int i = 0; i < kJ; ++i) {
+      const int j = tk + 32 * i;
+      if (j < d) {
+        qa[ta * ld + j] = acc_h[i] / sZ[ta];
+        orr[ta * ld + j] = acc_r[i] / sZr[ta];
+      }
+    }
+  }
+  // ---- phase 4: score_ab = pi_ab ||vbar_b - ohat_a^(-b)||
+  for (int k0 = 0; k0 < n; k0 += kScoreK) {
+    stage(vb, k0);
+    const int k = k0 + tk;
+    if (ta < na && k < n) {
+      const bool istop = k == sTop[ta];
+      const double* ref = istop ? orr + ta * ld : qa + ta * ld;
+      double s = 0.0;
+      for (int j = 0; j < d; ++j) {
+        const double t = kv[tk * ld + j] - ref[j];
+        s = fma(t, t, s);
+      }
+      const double Z = sZ[ta], z = zz[ta * n + k];
+      out0[(long long)ta * m.Ck + k] = istop ? (z / Z) * sqrt(s) : z * sqrt(s) / (Z - z);
+    }
   }
 }
 
@@ -314,7 +368,9 @@ __global__ void __launch_bounds__(1024) probe_pick_kernel(Dims m, Buffers b) {
 
 sparsepr_status launch_route(const Plan& p, cudaStream_t st) {
   const Dims& m = p.dm;
-  score_kernel<<<dim3(m.Cq, m.H), 256, 0, st>>>(m, p.b);
+  const size_t ssmem = (size_t)((2 * kScoreQ + kScoreK) * (m.d + 1) + 2 * kScoreQ * m.Ck) * sizeof(double);
+  SPR_CUDA_OK(cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem));
+  score_kernel<<<dim3(cdiv(m.Cq, kScoreQ), m.H), 256, ssmem, st>>>(m, p.b);
   SPR_LAUNCH_OK();
   select_kernel<<<dim3(m.Cq, m.H), 1024, 0, st>>>(m, p.b);
   SPR_LAUNCH_OK();

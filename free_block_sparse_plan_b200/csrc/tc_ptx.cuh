@@ -63,6 +63,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Arrive on an mbarrier once every cp.async this thread issued so far has completed; the
+// barrier's expected count includes this arrival (no pending-count increment).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 
 // Generic-proxy shared-memory writes made visible to the async proxy (tensor cores).
 __device__ __forceinline__ void fence_proxy_async() {
