@@ -35,18 +35,23 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-def launches_per_call(w, iters_k_run, iters_q_run) -> int:
-    """Kernel launches of one call, in the order the library enqueues them.
+def rank_workload(w, rank: int, world: int):
+    """Weak scaling: every rank runs the whole workload on its own heads (inputs drawn
+    with seed + rank), so the heads of different ranks are independent problems."""
+    return w.with_(seed=w.seed + rank) if world > 1 else w
 
-    plan:   key metric 1, eigen 1, key projection 1, k-means keys (init 1 + max_iter x
-            (assign 1 + update 4)), finalize 4 + groups 1, centroids 1, query metric 1,
-            eigen 1, query projection 1, k-means queries (same), finalize 5, centroids 1,
-            route 2, gather 3, probes 3.   attend: 1.  probe_fit: 2 + fit 1.  correct: 2.
-    Every k-means iteration is launched (converged heads return at once).
-    """
-    km = 1 + w.kmeans_max_iter * 5
-    plan = 3 + km + 5 + 1 + 3 + km + 5 + 1 + 2 + 3 + 3
-    return plan + 1 + 3 + 2
+
+def reduce_over_ranks(ms: float, pairs: float, world: int, device):
+    """Job time = the slowest rank's call time; executed pairs = the sum over ranks."""
+    if world == 1:
+        return ms, pairs
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    tot = torch.tensor([pairs], device=device, dtype=torch.float64)
+    dist.all_reduce(tot)
+    return float(t.item()), float(tot.item())
 
 
 class Clocks:
@@ -198,8 +203,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
-    # every rank takes its own heads: head index offset rank * H (weak scaling)
-    wr = w.with_(seed=w.seed + rank) if world > 1 else w
+    wr = rank_workload(w, rank, world)
     Q, K, V = W.make_inputs_torch(wr, device=dev)
     params = N.params_from_dict(wr.params())
     ws = torch.empty(N.sparsepr_workspace_size(params), dtype=torch.uint8, device=dev)
@@ -240,6 +244,7 @@ def main():
     stage = np.zeros((args.steps, 4))
     with Clocks(local) as clk:
         barrier()
+        launches0 = N.launch_count()                   # the library counts its own launches
         for i in range(args.steps):
             flush.fill_(i & 0xFF)                      # evict L2 between timed calls
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
@@ -249,6 +254,7 @@ def main():
             ev[4].synchronize()
             stage[i] = [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
                         ev[2].elapsed_time(ev[3]), ev[3].elapsed_time(ev[4])]
+        launches = N.launch_count() - launches0
         barrier()
         dense_ms = []
         for i in range(args.steps):
@@ -261,16 +267,7 @@ def main():
             dense_ms.append(e0.elapsed_time(e1))
         barrier()
     call_ms = stage.sum(axis=1)
-    ms = float(np.median(call_ms))
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        tot = torch.tensor([float(st["pairs_exec"])], device=dev, dtype=torch.float64)
-        dist.all_reduce(tot)
-        pairs_exec_all = float(tot.item())
-    else:
-        pairs_exec_all = float(st["pairs_exec"])
+    ms, pairs_exec_all = reduce_over_ranks(float(np.median(call_ms)), float(st["pairs_exec"]), world, dev)
     flops_all = 4.0 * w.d * pairs_exec_all
     value = flops_all / (ms * 1e-3) / 1e12
     attend_ms = float(np.median(stage[:, 1]))
@@ -329,7 +326,7 @@ def main():
                      "frac": attend_tflops / peak, "traffic": None,
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},
         "pct_bf16_peak_call": value / peak,
-        "gpu_launches": launches_per_call(w, 0, 0) * args.steps,
+        "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
     if e2e:

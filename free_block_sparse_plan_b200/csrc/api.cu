@@ -1,4 +1,5 @@
 // C ABI of the SparsePR library: argument validation, workspace layout, stage order.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -7,6 +8,12 @@
 
 using namespace spr;
 
+namespace spr {
+// Kernels launched by this library since it was loaded (all threads, all devices).
+std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace spr
+
 struct sparsepr_plan_s {
   Plan p;
 };
@@ -14,6 +21,9 @@ struct sparsepr_plan_s {
 namespace {
 
 // Bump allocator over the caller's workspace; with base == nullptr it only measures.
+// The kernels read Q, K, V and write Out with 16-byte vector accesses.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 struct Carver {
   char* base;
   size_t off = 0;
@@ -45,6 +55,8 @@ sparsepr_status validate(const sparsepr_params* q) {
     return SPARSEPR_ERR_ARG;
   if (q->kmeans_max_iter < 1 || q->kmeans_max_iter > 1000) return SPARSEPR_ERR_ARG;
   if (q->engine != SPARSEPR_ENGINE_AUTO && q->engine != SPARSEPR_ENGINE_SIMT) return SPARSEPR_ERR_ARG;
+  if (q->estimator < SPARSEPR_EST_RIDGE || q->estimator > SPARSEPR_EST_DIAGONAL || q->reserved != 0)
+    return SPARSEPR_ERR_ARG;
   return SPARSEPR_OK;
 }
 
@@ -54,6 +66,7 @@ Dims make_dims(const sparsepr_params* q) {
   d.Ms = q->M_s; d.rK = q->r_K; d.rQ = q->r_Q; d.Cq = q->C_q; d.Ck = q->C_k;
   d.M = q->M; d.r = q->r; d.lambda = q->lambda; d.rho = q->target_density;
   d.max_iter = q->kmeans_max_iter; d.engine = q->engine; d.seed = q->seed;
+  d.estimator = q->estimator;
   d.nchK = cdiv(q->N_k, kSortChunk);
   d.nchQ = cdiv(q->N_q, kSortChunk);
   d.nsplit = cdiv(q->N_k, kProbeSplit);
@@ -147,6 +160,15 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
     b->kmCmaxb = c.take<int>(2 * H);
     b->kmQueue = c.take<int4>((size_t)km_tc_queue_cap((int)H, (int)Nm));
     b->kmQcnt = c.take<int>(2);
+    b->kmU = c.take<double>(H * Nm);
+    b->kmL = c.take<float>(H * Nm * (size_t)cdiv((int)Cm, 32));
+    b->kmDelta = c.take<double>(H * Cm);
+    b->kmDmax = c.take<unsigned long long>(2 * H * (size_t)cdiv((int)Cm, 32));
+    b->kmAidx = c.take<int>(H * Np);
+    b->kmAcnt = c.take<int>(2 * H);
+    b->kmReassigned = c.take<long long>(2 * H);
+    b->kmShi = c.take<__nv_bfloat16>(H * Np * 64);
+    b->kmSlo = c.take<__nv_bfloat16>(H * Np * 64);
   }
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);
@@ -158,6 +180,7 @@ sparsepr_status make_plan(const sparsepr_params* q, const void* Q, const void* K
   sparsepr_status s = validate(q);
   if (s != SPARSEPR_OK) return s;
   if (!Q || !K || !V || !out) return SPARSEPR_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return SPARSEPR_ERR_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return SPARSEPR_ERR_WORKSPACE;
   plan->dm = make_dims(q);
   const size_t need = carve(plan->dm, nullptr, &plan->b);
@@ -180,6 +203,7 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_CUDA_OK(cudaMemsetAsync(p.b.kmK, 0, m.H * 4 * sizeof(int), st));
   SPR_CUDA_OK(cudaMemsetAsync(p.b.kmQ, 0, m.H * 4 * sizeof(int), st));
   SPR_CUDA_OK(cudaMemsetAsync(p.b.pairs, 0, m.H * sizeof(long long), st));
+  SPR_CUDA_OK(cudaMemsetAsync(p.b.kmReassigned, 0, 2 * m.H * sizeof(long long), st));
   // key side (paper S4.1, App. B.1)
   SPR_TRY(launch_key_metric(p, st));
   SPR_TRY(launch_eigen_factor(p, false, st));
@@ -260,6 +284,7 @@ ExportDesc export_desc(const Plan& p, int what) {
     case SPARSEPR_X_PROBE_DIST: return {b.dist, H * m.Nq * D};
     case SPARSEPR_X_KBAR: return {b.kbar, H * m.Ck * d * D};
     case SPARSEPR_X_QBAR: return {b.qbar, H * m.Cq * d * D};
+    case SPARSEPR_X_KM_REASSIGNED: return {b.kmReassigned, H * 2 * sizeof(long long)};
     default: return {nullptr, 0};
   }
 }
@@ -328,7 +353,7 @@ sparsepr_status sparsepr_probe_fit(sparsepr_plan_t plan, void* stream) {
 }
 
 sparsepr_status sparsepr_correct(sparsepr_plan_t plan, void* Out, void* stream) {
-  if (!plan || !Out) return SPARSEPR_ERR_ARG;
+  if (!plan || !Out || !aligned16(Out)) return SPARSEPR_ERR_ARG;
   if (plan->p.stage < 3) return SPARSEPR_ERR_STATE;
   return launch_correct(plan->p, Out, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -350,6 +375,7 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
                                          const void* K, const void* V, void* Out,
                                          void* stream) {
   if (!params || !Q || !K || !V || !Out) return SPARSEPR_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Out)) return SPARSEPR_ERR_ARG;
   if (params->dtype != SPARSEPR_F32 && params->dtype != SPARSEPR_BF16) return SPARSEPR_ERR_DTYPE;
   if (params->H < 1 || params->N_q < 1 || params->N_k < 1) return SPARSEPR_ERR_SHAPE;
   if (params->d < 8 || params->d > kMaxD || params->d % 8) return SPARSEPR_ERR_SHAPE;
@@ -464,3 +490,5 @@ const char* sparsepr_status_string(sparsepr_status status) {
 }
 
 }  // extern "C"
+
+extern "C" unsigned long long sparsepr_launch_count(void) { return spr::g_launches.load(); }

@@ -29,6 +29,8 @@ struct KmView {         // one k-means instance (keys or queries) for all heads
   int* off;             // [H][C+1]
   int* km;              // [H][4]: done, changed[0], changed[1], iterations
   double* obj;          // [H][C]
+  double* delta;        // [H][C] centre movement of each update, or null
+  unsigned long long* dmax;   // [2][H][G] largest movement per 32-centre group (double bits)
   int N, C, r, nch, stage;
 };
 
@@ -36,21 +38,25 @@ KmView view(const Plan& p, bool query) {
   const Buffers& b = p.b;
   const Dims& m = p.dm;
   if (query)
-    return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, m.Nq, m.Cq, m.rQ, m.nchQ, 1};
-  return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, m.Nk, m.Ck, m.rK, m.nchK, 0};
+    return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, b.kmDelta, b.kmDmax,
+            m.Nq, m.Cq, m.rQ, m.nchQ, 1};
+  return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, b.kmDelta, b.kmDmax,
+          m.Nk, m.Ck, m.rK, m.nchK, 0};
 }
 
 // ---------------------------------------------------------------------------------
 // Response coordinates in fp64: phi = X F (keys), phi = z / max(rms(z), 1e-6) with
 // z = X F (queries) (paper S4.1, App. B.1-B.2).  X is exact in its dtype; F is the fp64
 // factor; each coordinate is one fp64 dot product over d in ascending order.
-// A block takes 64 rows: X is staged transposed (column j of the tile contiguous), F once
-// per block; thread (tr, tc) forms rows 4tr..4tr+3 x columns tc, tc+16, ... (a register
+// A block takes 256 rows in four tiles of 64: F is staged once per block, each X tile
+// transposed (column j of the tile contiguous, 16-byte loads, one row per lane); thread
+// (tr, tc) forms rows 4tr..4tr+3 x columns tc, tc+16, ... (a register
 // tile, so every shared-memory value feeds several fp64 FMAs and the 16 column threads
 // of a row group read 16 consecutive F values).  When the tensor-core k-means will
 // cluster these coordinates, the block also writes its input: each row split into two
 // bf16 pieces (rows padded to 64 columns, zero rows up to Npad) and |phi|.
 constexpr int kProjRows = 64;
+constexpr int kProjTiles = 4;              // 64-row tiles per block
 constexpr int kProjXs = kProjRows + 4;     // transposed tile row stride (floats)
 template <int R, bool RMS>
 __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int N, const double* Fall, int r,
@@ -66,15 +72,41 @@ __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int
     const int j = e / R, k = e % R;
     F[e] = k < r ? Fh[j * r + k] : 0.0;
   }
-  const long long row0 = (long long)blockIdx.x * kProjRows;
   const long long base = ((long long)h * N) * d;
-  for (int e = threadIdx.x; e < kProjRows * d; e += blockDim.x) {
-    const int i = e / d, j = e % d;
+  const int tr = threadIdx.x >> 4, tc = threadIdx.x & 15;
+  for (int tile = 0; tile < kProjTiles; ++tile) {
+  const long long row0 = ((long long)blockIdx.x * kProjTiles + tile) * kProjRows;
+  if (row0 >= (xhi ? Npad : N)) break;
+  __syncthreads();                         // the previous tile's reads of Xt are done
+  // one row per lane, 16 bytes per load: consecutive lanes write consecutive banks
+  const int per = m.dtype == SPARSEPR_BF16 ? 8 : 4;        // elements per 16-byte load
+  const bool vec = (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+  for (int e = threadIdx.x; e < kProjRows * (d / per); e += blockDim.x) {
+    const int i = e % kProjRows, c = e / kProjRows;
     const long long row = row0 + i;
-    Xt[j * kProjXs + i] = row < N ? load_as_float(X, base + row * d + j, m.dtype) : 0.0f;
+    float v[8];
+    if (row < N && !vec) {
+      for (int q = 0; q < per; ++q) v[q] = load_as_float(X, base + row * d + c * per + q, m.dtype);
+    } else if (row < N) {
+      if (m.dtype == SPARSEPR_BF16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(X) + base + row * d + c * 8);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          v[2 * q] = __uint_as_float(w[q] << 16);
+          v[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+        }
+      } else {
+        const float4 f = *reinterpret_cast<const float4*>(static_cast<const float*>(X) + base + row * d + c * 4);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = 0.0f;
+    }
+    for (int q = 0; q < per; ++q) Xt[(c * per + q) * kProjXs + i] = v[q];
   }
   __syncthreads();
-  const int tr = threadIdx.x >> 4, tc = threadIdx.x & 15;
   double acc[4][CPT];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -137,6 +169,7 @@ __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int
       }
     }
   }
+  }
 }
 
 template <bool RMS>
@@ -144,7 +177,7 @@ sparsepr_status launch_project(const Plan& p, const void* X, int N, const double
                                __nv_bfloat16* xhi, __nv_bfloat16* xlo, float* xn, int Npad, cudaStream_t st) {
   const int d = p.dm.d;
   const int rows = xhi ? Npad : N;
-  dim3 grid(cdiv(rows, kProjRows), p.dm.H);
+  dim3 grid(cdiv(rows, kProjRows * kProjTiles), p.dm.H);
   auto run = [&](auto kern, int R) -> sparsepr_status {
     const size_t smem = (size_t)d * R * sizeof(double) + (size_t)d * kProjXs * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -349,6 +382,26 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
     for (int q = 0; q < kMeanSub; ++q) s += part[q][k];
     mean = cnt > 0 ? s / (double)cnt : cent[k];
   }
+  if (!force) {
+    // how far the centre moves (rounded up), for the distance bounds of the next step
+    double dd = 0.0;
+    if (sub == 0 && kk && cnt > 0) {
+      const double t = mean - cent[k];
+      dd = t * t;
+    }
+    dd = warp_sum(dd);
+    if ((threadIdx.x & 31) == 0) opart[threadIdx.x >> 5] = dd;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double s2 = 0.0;
+      for (int q = 0; q < kMeanSub * kMaxR / 32; ++q) s2 += opart[q];
+      const double dl = sqrt(s2) * (1.0 + 1e-12);
+      v.delta[(long long)h * v.C + c] = dl;
+      const int G = (v.C + 31) / 32;              // 32-centre groups of the distance bounds
+      atomicMax(v.dmax + ((long long)(it & 1) * gridDim.y + h) * G + c / 32,
+                (unsigned long long)__double_as_longlong(dl));
+    }
+  }
   __syncthreads();
   if (cnt > 0 && sub == 0 && kk) cent[k] = mean;
   if (!force) return;
@@ -372,10 +425,13 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
 sparsepr_status run_update(const Plan& p, const KmView& v, int it, bool force, cudaStream_t st) {
   const int H = p.dm.H;
   cs_hist_kernel<<<dim3(v.nch, H), kSortChunk, 0, st>>>(v, it, force);
+  SPR_LAUNCH_OK();
   cs_scan_kernel<<<H, 1024, 0, st>>>(v, it, force);
+  SPR_LAUNCH_OK();
   const size_t wsm = (size_t)(kSortChunk / 32) * v.C * sizeof(int);
   SPR_CUDA_OK(cudaFuncSetAttribute(cs_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsm));
   cs_scatter_kernel<<<dim3(v.nch, H), kSortChunk, wsm, st>>>(v, it, force);
+  SPR_LAUNCH_OK();
   cs_mean_kernel<<<dim3(v.C, H), kMeanSub * kMaxR, 0, st>>>(v, it, force);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
@@ -560,21 +616,25 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   // there are enough centres to fill the tiles; the full scan otherwise or on request
   const bool tc = km_uses_tc(p, query);
   const Buffers& b = p.b;
-  const KmTcBuffers kb{b.kmXhi, b.kmXlo, b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt};
+  const KmTcBuffers kb{b.kmXhi, b.kmXlo, b.kmShi, b.kmSlo, b.kmU, b.kmDelta, b.kmL, b.kmDmax, b.kmAidx,
+                       b.kmAcnt, b.kmReassigned + (query ? H : 0), b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt};
   if (tc) {
     SPR_CUDA_OK(cudaMemsetAsync(b.kmCmaxb, 0, sizeof(int) * 2 * H, st));
     SPR_CUDA_OK(cudaMemsetAsync(b.kmQcnt, 0, sizeof(int) * 2, st));
+    SPR_CUDA_OK(cudaMemsetAsync(b.kmAcnt, 0, sizeof(int) * 2 * H, st));
   }
   for (int it = 0; it < p.dm.max_iter; ++it) {
     if (tc) {
       sparsepr_status s = km_tc_assign(kb, v.X, v.cent, H, v.N, v.C, v.r, it, v.lab, v.km, b.err, st);
       if (s != SPARSEPR_OK) return s;
-    } else if (v.r <= 8) assign<8>(v, H, it, st);
-    else if (v.r <= 16) assign<16>(v, H, it, st);
-    else if (v.r <= 32) assign<32>(v, H, it, st);
-    else if (v.r <= 48) assign<48>(v, H, it, st);
-    else assign<64>(v, H, it, st);
-    SPR_LAUNCH_OK();
+    } else {
+      if (v.r <= 8) assign<8>(v, H, it, st);
+      else if (v.r <= 16) assign<16>(v, H, it, st);
+      else if (v.r <= 32) assign<32>(v, H, it, st);
+      else if (v.r <= 48) assign<48>(v, H, it, st);
+      else assign<64>(v, H, it, st);
+      SPR_LAUNCH_OK();
+    }
     sparsepr_status s = run_update(p, v, it, false, st);
     if (s != SPARSEPR_OK) return s;
   }

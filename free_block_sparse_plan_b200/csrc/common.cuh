@@ -34,6 +34,7 @@ struct Dims {
   double lambda, rho;
   int max_iter, engine;
   unsigned long long seed;
+  int estimator;       // sparsepr_estimator
   int nchK, nchQ;      // counting-sort chunks per head
   int nsplit;          // partial blocks of the exact probe attention
   double beta;         // per-query key budget (rho - M/N_q) * N_k
@@ -82,6 +83,13 @@ struct Buffers {
   float *kmCn;               // squared centre norms [H][Cpad]
   int *kmCmaxb;              // largest squared centre norm as float bits [2][H]
   int4 *kmQueue;             // points whose label needs exact rescoring
+  double *kmU;               // distance to the own centre, upper bound [H][Nmax]
+  float *kmL;                // distance to the other centres of each 32-centre group, lower bound [H][G][N]
+  double *kmDelta;           // centre movement of the last update [H][Cmax]
+  unsigned long long *kmDmax;  // largest movement per head and group as double bits [2][H][G]
+  int *kmAidx, *kmAcnt;      // points to re-assign, compacted [H][Npad]; their counts [2][H]
+  long long *kmReassigned;   // points re-assigned, summed over the steps [2 sides][H]
+  __nv_bfloat16 *kmShi, *kmSlo;  // their split coordinates, compacted [H][Npad][64]
   int *kmQcnt;               // queue lengths [2]
   int *err;                  // device error word
 };
@@ -102,8 +110,11 @@ struct Plan {
     if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA;       \
   } while (0)
 
+// After every kernel launch: count it (sparsepr_launch_count) and check it.
+void count_launch();
 #define SPR_LAUNCH_OK()                                    \
   do {                                                     \
+    count_launch();                                        \
     cudaError_t e_ = cudaGetLastError();                   \
     if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA;       \
   } while (0)
@@ -220,6 +231,12 @@ sparsepr_status launch_correct_tc(const Plan& p, void* Out, cudaStream_t st);
 long long km_tc_queue_cap(int H, int N);
 struct KmTcBuffers {
   const __nv_bfloat16 *xhi, *xlo;
+  __nv_bfloat16 *shi, *slo;
+  double *U, *delta;
+  float* L;
+  unsigned long long* dmax;
+  int *aidx, *acnt;
+  long long* reassigned;     // [H] of this side
   const float* xn;
   __nv_bfloat16 *chi, *clo;
   float* cn;

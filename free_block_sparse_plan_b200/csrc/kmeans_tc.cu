@@ -56,7 +56,11 @@ constexpr uint32_t kCBytes = kChunk * kKP * 2;     // 32 KB: one centre chunk (h
 constexpr uint32_t kSmemLimit = 232448;            // opt-in shared memory per block
 
 struct KmArgs {
-  CUtensorMap tm_xhi, tm_xlo, tm_chi, tm_clo;   // [H*Npad][64], [H*Cpad][64] bf16
+  CUtensorMap tm_xhi, tm_xlo, tm_chi, tm_clo;   // [H*Npad][64] (compacted points), [H*Cpad][64] bf16
+  const int* aidx;            // [H][Npad] point of each compacted row
+  const int* acnt;            // [H] compacted rows of this step
+  double* U;                  // [H][N] upper bound: distance to the own centre
+  float* L;                   // [H][G][N] lower bounds: distance to each 32-centre group but the own centre
   const float* xn;            // [H][N] |x|
   const float* cn;            // [H][Cpad] ||c||^2 (+inf for padding centres)
   const int* cmaxb;           // [2][H] max ||c||^2 as float bits, slot it & 1
@@ -68,8 +72,10 @@ struct KmArgs {
   const double* X;            // [H][N][r] fp64 features (fallback when the queue is full)
   const double* cent;         // [H][C][r] fp64 centres
   int* err;
-  int H, N, Npad, C, Cpad, Cw, nch, r, it, slots;
+  int H, N, Npad, C, Cpad, Cw, nch, r, it, slots, G;
 };
+
+constexpr int kGroup = 32;              // centres per lower-bound group
 
 // fp64 direct squared distance in ascending dimensions: the full scan's formula.
 __device__ __forceinline__ double exact_d2(const double* x, const double* c, int r) {
@@ -114,16 +120,25 @@ __device__ __forceinline__ bool km_wait(KmMisc* ms, uint32_t bar, uint32_t parit
   }
 }
 
-// The kk-th head (ascending) that has not converged; queried with non-decreasing kk.
-struct ActiveHeads {
-  const int* km;
-  int k, h;
-  __device__ int head(int kk) {
-    while (k < kk) {
+// A distance no larger than every one whose score is at least `a` (score error below Eb),
+// rounded down to fp32 with a margin.
+__device__ __forceinline__ float dist_floor(float a, double Eb, double x2) {
+  if (!(a < 3.0e38f)) return INFINITY;             // only padding centres in the group
+  return __double2float_rd(sqrt(fmax((double)a - Eb + x2, 0.0)) * (1.0 - 1e-9));
+}
+
+// Global tile index -> (head, tile within the head) over the compacted points of every
+// head (ceil(count / 128) tiles each); queried with non-decreasing tiles.
+struct TileCursor {
+  const int* acnt;
+  int h, base, nt;
+  __device__ int head(long long t, int* lt) {
+    while (t >= base + nt) {
+      base += nt;
       ++h;
-      while (km[4 * h]) ++h;
-      ++k;
+      nt = (acnt[h] + kRows - 1) / kRows;
     }
+    *lt = (int)(t - base);
     return h;
   }
 };
@@ -136,11 +151,9 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
   KmMisc* ms = reinterpret_cast<KmMisc*>(smem_raw + (base - raw) + oX + g.slots * 2 * kXBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // tiles of the heads still iterating, split evenly over the CTAs
-  int nact = 0;
-  for (int h = 0; h < g.H; ++h) nact += g.km[4 * h] == 0;
-  const int tph = g.Npad / kRows;
-  const long long T = (long long)nact * tph;
+  // tiles of the points to re-assign (converged heads have none), split evenly over CTAs
+  long long T = 0;
+  for (int h = 0; h < g.H; ++h) T += (g.acnt[h] + kRows - 1) / kRows;
   const long long t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
   const int ntiles = (int)(t1 - t0);
   if (blockIdx.x == 0 && tid == 0) {
@@ -176,7 +189,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = ms->tmem_base;
-  ActiveHeads act{g.km, -1, -1};
+  TileCursor act{g.acnt, -1, 0, 0};
 
   if (warp == 8) {
     // ============================================================ TMA producer
@@ -184,7 +197,8 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       int loaded = -1, nload = 0;
       for (int li = 0; li < ntiles; ++li) {
         const long long t = t0 + li;
-        const int h = act.head((int)(t / tph));
+        int lt;
+        const int h = act.head(t, &lt);
         if (h != loaded) {
           if (nload > 0 && !km_wait(ms, BAR(kbCEmpty), (nload - 1) & 1, g.err)) break;
           tc::mbar_expect_tx(BAR(kbCFull), 2u * g.nch * g.Cw * kKP * 2);
@@ -199,7 +213,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
         const int slot = li % g.slots, use = li / g.slots;
         if (use > 0 && !km_wait(ms, BAR(kbXEmpty0 + slot), (use - 1) & 1, g.err)) break;
         tc::mbar_expect_tx(BAR(kbXFull0 + slot), 2u * kXBytes);
-        const int row = h * g.Npad + (int)(t % tph) * kRows;
+        const int row = h * g.Npad + lt * kRows;          // compacted rows of the head
         const uint32_t xs = base + oX + slot * 2 * kXBytes;
         tc::tma_load_2d(xs, &g.tm_xhi, 0, row, BAR(kbXFull0 + slot));
         tc::tma_load_2d(xs + kXBytes, &g.tm_xlo, 0, row, BAR(kbXFull0 + slot));
@@ -214,7 +228,8 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       bool ok = true;
       for (int li = 0; ok && li < ntiles; ++li) {
         const long long t = t0 + li;
-        const int h = act.head((int)(t / tph));
+        int lt;
+        const int h = act.head(t, &lt);
         if (h != cur) {
           if (nload > 0) tc::mma_commit(BAR(kbCEmpty));     // old centres free once done
           if (!km_wait(ms, BAR(kbCFull), nload & 1, g.err)) { ok = false; break; }
@@ -262,14 +277,15 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
     int J = 0;
     int nfull0 = 0, nfull1 = 0;            // waits done on accFull[0][grp], accFull[1][grp]
     // per-point values of this group's next tile, loaded one tile ahead of their use
-    ActiveHeads pre{g.km, -1, -1};
+    TileCursor pre{g.acnt, -1, 0, 0};
     float nxn = 0.0f, ncm = 0.0f;
-    int nold = 0;
+    int nold = 0, nn = 0;
     auto point_vals = [&](int li2) {
-      const long long t2 = t0 + li2;
-      const int h2 = pre.head((int)(t2 / tph));
-      const int row2 = (int)(t2 % tph) * kRows + r;
-      const long long pi2 = (long long)h2 * g.N + (row2 < g.N ? row2 : 0);
+      int lt2;
+      const int h2 = pre.head(t0 + li2, &lt2);
+      const int j2 = lt2 * kRows + r;
+      nn = j2 < g.acnt[h2] ? g.aidx[(long long)h2 * g.Npad + j2] : -1;
+      const long long pi2 = (long long)h2 * g.N + (nn >= 0 ? nn : 0);
       nxn = g.xn[pi2];
       nold = g.lab[pi2];
       ncm = sqrtf(__int_as_float(g.cmaxb[(g.it & 1) * g.H + h2]));
@@ -277,15 +293,17 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
     if (grp < ntiles) point_vals(grp);
     for (int li = 0; li < ntiles; ++li) {
       const long long t = t0 + li;
-      const int h = act.head((int)(t / tph));
+      int lt;
+      const int h = act.head(t, &lt);
       if ((li & 1) != grp) { J += g.nch; continue; }
-      // per-point values first: their loads overlap the wait for the scores
-      const int row = (int)(t % tph) * kRows + r;
-      const bool live = row < g.N;
-      const long long pi = (long long)h * g.N + (live ? row : 0);
+      const bool live = nn >= 0;          // this row holds a point to re-assign
+      const long long pi = (long long)h * g.N + (live ? nn : 0);
       const float xn = nxn, cm = ncm;
       const int old = nold;
       if (li + 2 < ntiles) point_vals(li + 2);
+      // score error bound: a lower bound on a distance from a score is sqrt(a - Eb + |x|^2)
+      const double x2 = (double)xn * xn;
+      const double Eb = 2e-4 * xn * cm + 5e-6 * (double)cm * cm + 1e-6 * x2;
       const float* cnh = g.cn + (long long)h * g.Cpad;
       float a0 = BIG, a1 = BIG;            // smallest and second smallest score
       int c0 = 0;                           // centre of the smallest (first one on ties)
@@ -315,6 +333,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
           tc::tmem_ld32(acc + q, *reinterpret_cast<float(*)[32]>(v));
           tc::tmem_ld32(acc + q + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
+          float gm[2] = {BIG, BIG};         // smallest score of each 32-centre group
 #pragma unroll
           for (int i4 = 0; i4 < 16; ++i4) {
             const float cv[4] = {cq[i4].x, cq[i4].y, cq[i4].z, cq[i4].w};
@@ -324,6 +343,14 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
               a1 = fminf(a1, fmaxf(a0, a));
               c0 = a < a0 ? cb + 4 * i4 + e : c0;
               a0 = fminf(a0, a);
+              gm[i4 >> 3] = fminf(gm[i4 >> 3], a);
+            }
+          }
+          if (live) {
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+              const int gi = cb / kGroup + s2;
+              if (gi < g.G) g.L[((long long)h * g.G + gi) * g.N + (pi - (long long)h * g.N)] = dist_floor(gm[s2], Eb, x2);
             }
           }
         }
@@ -383,6 +410,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       const float T = 4e-4f * xn * cm + 1e-5f * (xn + cm) * (xn + cm) + 1e-30f;
       int best = c0;
       if (!(a1 > a0 + T)) {
+        g.U[pi] = INFINITY;                          // near a tie: re-assign at the next step
         const int full = nrec > 4 ? 1 : 0;
         const int slot = atomicAdd(g.qcnt + (g.it & 1), 1);
         if (slot < g.qcap) {
@@ -398,6 +426,11 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
           const double d2 = exact_d2(x, cent + (long long)ci * g.r, g.r);
           if (d2 < bd) { bd = d2; best = ci; }
         }
+      } else {
+        // the own centre is nearer than u; in its group every other centre scores at
+        // least the runner-up a1 (the other groups' bounds were written above)
+        g.U[pi] = sqrt(fmax((double)a0 + Eb + x2, 0.0)) * (1.0 + 1e-9);
+        g.L[((long long)h * g.G + c0 / kGroup) * g.N + (pi - (long long)h * g.N)] = dist_floor(a1, Eb, x2);
       }
       if (old != best) {
         g.lab[pi] = best;
@@ -410,6 +443,97 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
   if (warp == 9) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// Which points can change label at this step (exact; Hamerly's bounds refined per group
+// of 32 centres as in Yinyang k-means): u bounds the distance to the point's own centre
+// from above, l_g the distance to every centre of group g except the own one from below.
+// After an update that moved centre c by delta_c (group g by at most dmax_g),
+// u + delta_own and l_g - dmax_g still bound them; if u < min_g l_g the own centre stays
+// strictly the nearest and the label cannot change.  Every other point is listed in its
+// head's compacted index (warp-aggregated slots; the order inside a head does not affect
+// any result).  Step 0 re-assigns every point.
+struct KmFilter {
+  const int* km;
+  const int* lab;
+  const double* delta;
+  unsigned long long* dmax;
+  double* U;
+  float* L;
+  int *aidx, *acnt;
+  long long* reassigned;
+  const __nv_bfloat16 *xhi, *xlo;
+  __nv_bfloat16 *shi, *slo;
+  int H, N, Npad, C, G, it;
+};
+
+__global__ void __launch_bounds__(256) km_filter_kernel(const KmFilter f) {
+  const int h = blockIdx.y, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0) f.acnt[((f.it + 1) & 1) * f.H + h] = 0;    // the next step's count
+    if (threadIdx.x < f.G)                                           // this step's update
+      f.dmax[((long long)(f.it & 1) * f.H + h) * f.G + threadIdx.x] = 0ull;
+  }
+  if (f.km[4 * h]) return;                         // converged head
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  bool act = false;
+  if (n < f.N) {
+    const long long pi = (long long)h * f.N + n;
+    if (f.it == 0) {
+      act = true;
+    } else {
+      const double u = f.U[pi] + f.delta[(long long)h * f.C + f.lab[pi]];
+      const unsigned long long* dm = f.dmax + ((long long)((f.it - 1) & 1) * f.H + h) * f.G;
+      float* lp = f.L + (long long)h * f.G * f.N + n;          // [g] at lp[g * N]
+      // every bound loaded before any is stored back, so the loads are all in flight
+      constexpr int kMaxG = kMaxChunks * kChunk / kGroup;
+      float lv[kMaxG];
+#pragma unroll
+      for (int gi = 0; gi < kMaxG; ++gi)
+        if (gi < f.G) lv[gi] = lp[(long long)gi * f.N];
+      double lmin = INFINITY;
+#pragma unroll
+      for (int gi = 0; gi < kMaxG; ++gi)
+        if (gi < f.G) {
+          const double l = (double)lv[gi] - __longlong_as_double((long long)dm[gi]);
+          lp[(long long)gi * f.N] = __double2float_rd(l);
+          lmin = fmin(lmin, l);
+        }
+      f.U[pi] = u;
+      act = !(u < lmin);
+    }
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, act);
+  int base = 0;
+  if (lane == 0 && m) {
+    base = atomicAdd(f.acnt + (f.it & 1) * f.H + h, __popc(m));
+    atomicAdd(reinterpret_cast<unsigned long long*>(f.reassigned + h), (unsigned long long)__popc(m));
+  }
+  base = __shfl_sync(0xffffffffu, base, 0);
+  if (act) f.aidx[(long long)h * f.Npad + base + __popc(m & ((1u << lane) - 1u))] = n;
+  // the listed points' split rows into their compacted rows: 16 lanes per point, one
+  // 16-byte chunk each (8 of the hi row, 8 of the lo row), two points per pass
+  unsigned mm = m;
+  while (mm) {
+    const int l0 = __ffs(mm) - 1;
+    mm &= mm - 1;
+    int l1 = -1;
+    if (mm) {
+      l1 = __ffs(mm) - 1;
+      mm &= mm - 1;
+    }
+    const int src = lane < 16 ? l0 : l1;
+    const int sl = src < 0 ? 0 : src;
+    const int pn = __shfl_sync(0xffffffffu, n, sl);
+    if (src >= 0) {
+      const int slot = base + __popc(m & ((1u << sl) - 1u));
+      const int c = lane & 7;
+      const bool lo = (lane & 8) != 0;
+      const uint4* s4 = reinterpret_cast<const uint4*>((lo ? f.xlo : f.xhi) + ((long long)h * f.Npad + pn) * kKP);
+      uint4* d4 = reinterpret_cast<uint4*>((lo ? f.slo : f.shi) + ((long long)h * f.Npad + slot) * kKP);
+      d4[c] = s4[c];
+    }
   }
 }
 
@@ -536,12 +660,18 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   const int Npad = km_tc_npad(N), Cpad = km_tc_cpad(C);
   const int nch = cdiv(C, kChunk);
   const int Cw = nch > 1 ? kChunk : cdiv(C, 64) * 64;
+  const int G = cdiv(C, kGroup);
+  const KmFilter f{kmstate, lab, kb.delta, kb.dmax, kb.U, kb.L, kb.aidx, kb.acnt, kb.reassigned, kb.xhi, kb.xlo,
+                   kb.shi, kb.slo, H, N, Npad, C, G, it};
+  km_filter_kernel<<<dim3(cdiv(N, 256), H), 256, 0, st>>>(f);
+  SPR_LAUNCH_OK();
   km_split_c_kernel<<<dim3(Cpad / 8, H), 256, 0, st>>>(cent, H, C, Cpad, r, it, kmstate, kb.chi, kb.clo,
                                                        kb.cn, kb.cmaxb);
   SPR_LAUNCH_OK();
   KmArgs g;
-  if (!make_map(&g.tm_xhi, kb.xhi, (long long)H * Npad, kRows) ||
-      !make_map(&g.tm_xlo, kb.xlo, (long long)H * Npad, kRows) ||
+  g.G = G;
+  if (!make_map(&g.tm_xhi, kb.shi, (long long)H * Npad, kRows) ||
+      !make_map(&g.tm_xlo, kb.slo, (long long)H * Npad, kRows) ||
       !make_map(&g.tm_chi, kb.chi, (long long)H * Cpad, Cw) ||
       !make_map(&g.tm_clo, kb.clo, (long long)H * Cpad, Cw))
     return SPARSEPR_ERR_CUDA;
@@ -550,6 +680,7 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   slots = slots > kMaxSlots ? kMaxSlots : slots;
   if (slots < 1) return SPARSEPR_ERR_ARG;
   const uint32_t smem = fixed + (uint32_t)slots * 2 * kXBytes;
+  g.aidx = kb.aidx; g.acnt = kb.acnt + (it & 1) * H; g.U = kb.U; g.L = kb.L;
   g.xn = kb.xn; g.cn = kb.cn; g.cmaxb = kb.cmaxb; g.lab = lab; g.km = kmstate;
   g.queue = kb.queue; g.qcnt = kb.qcnt; g.qcap = (int)km_tc_queue_cap(H, N);
   g.X = X; g.cent = cent; g.err = err;

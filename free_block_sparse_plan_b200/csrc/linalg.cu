@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const v
 // remove.  Bounded sweeps.  `nrm` is shared scratch of at least ncols doubles.
 __device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red, double* nrm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  // sixteen lanes per column pair (two pairs per warp)
   const int sub = lane & 15, grp = 2 * warp + (lane >> 4), ngrp = 2 * nwarps;
-  const unsigned half = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
+  const unsigned gmask = 0xffffu << (lane & 16);
   double f = 0.0;
   for (int e = threadIdx.x; e < rows * ncols; e += blockDim.x) f += G[e] * G[e];
   const double abs_tol = 1e-15 * block_sum(f, red);
@@ -89,8 +90,17 @@ __device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red,
       for (int k = grp; k < npairs; k += ngrp) {
         // circle method: position 0 fixed, the others rotate by `round`
         const int pa = k, pb = nn - 1 - k;
-        const int ia = pa == 0 ? 0 : 1 + (pa - 1 + round) % (nn - 1);
-        const int ib = pb == 0 ? 0 : 1 + (pb - 1 + round) % (nn - 1);
+        int ia = 0, ib = 0;
+        if (pa != 0) {
+          int v = pa - 1 + round;
+          if (v >= nn - 1) v -= nn - 1;
+          ia = 1 + v;
+        }
+        if (pb != 0) {
+          int v = pb - 1 + round;
+          if (v >= nn - 1) v -= nn - 1;
+          ib = 1 + v;
+        }
         if (ia >= ncols || ib >= ncols) continue;     // uniform over the 16 lanes
         double* a = G + (long long)ia * rows;
         double* b = G + (long long)ib * rows;
@@ -103,7 +113,7 @@ __device__ void hestenes(double* G, int rows, int ncols, int* flag, double* red,
         }
         double ga = g0 + g1;
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) ga += __shfl_xor_sync(half, ga, o);
+        for (int o = 8; o > 0; o >>= 1) ga += __shfl_xor_sync(gmask, ga, o);
         const double al = nrm[ia], be = nrm[ib];
         if (ga == 0.0 || ga * ga <= 1e-28 * (al * be) || fabs(ga) <= abs_tol) continue;
         // t = tan of the angle that zeroes a.b: with u = |b|^2 - |a|^2 and v = 2 a.b,
@@ -573,8 +583,88 @@ sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st) 
   return SPARSEPR_OK;
 }
 
+// Restricted estimators (paper App. D.3, Table 4), one CTA per head: the statistics of
+// the full fit, then B = 0 (mean only), B = a I with
+// a = sum_pj w_p xb_pj Rb_pj / (sum_pj w_p xb_pj^2 + lambda d) (scalar), or B = diag(b) with
+// b_j = sum_p w_p xb_pj Rb_pj / (sum_p w_p xb_pj^2 + lambda) (diagonal); omega-weighted
+// sums over the probes, no projection (P = I), folded as B' = diag(b / s), c = mu_R - mu_x b / s.
+__global__ void __launch_bounds__(kLinThreads) fit_simple_kernel(Dims m, Buffers b) {
+  __shared__ double num[kMaxD], den[kMaxD], red[32];
+  const int h = blockIdx.x, d = m.d, M = m.M;
+  const long long hd = (long long)h * d;
+  const int* probes = b.probes + (long long)h * M;
+  const double* w = b.wP + (long long)h * M;
+  double wsum = 0.0;
+  for (int p = 0; p < M; ++p) wsum += w[p];
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    double mx = 0.0, mr = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const int pos = b.invQ[(long long)h * m.Nq + probes[p]];
+      const double x = (double)b.Osp[((long long)h * m.Nq + pos) * d + j];
+      const double dn = (double)b.Odense[((long long)h * M + p) * d + j];
+      if (!isfinite(x) || !isfinite(dn)) atomicOr(b.err, kErrNonFinite);
+      mx += (w[p] / wsum) * x;
+      mr += (w[p] / wsum) * (dn - x);
+    }
+    double var = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const int pos = b.invQ[(long long)h * m.Nq + probes[p]];
+      const double t = (double)b.Osp[((long long)h * m.Nq + pos) * d + j] - mx;
+      var += (w[p] / wsum) * t * t;
+    }
+    const double sd = sqrt(var + 1e-6);
+    double nu = 0.0, de = 0.0;
+    for (int p = 0; p < M; ++p) {
+      const int pos = b.invQ[(long long)h * m.Nq + probes[p]];
+      const double x = (double)b.Osp[((long long)h * m.Nq + pos) * d + j];
+      const double dn = (double)b.Odense[((long long)h * M + p) * d + j];
+      const double om = (double)M * w[p] / wsum;
+      const double xb = (x - mx) / sd, rb = (dn - x) - mr;
+      nu += om * xb * rb;
+      de += om * xb * xb;
+    }
+    num[j] = nu;
+    den[j] = de;
+    b.muX[hd + j] = mx;
+    b.muR[hd + j] = mr;
+    b.sX[hd + j] = sd;
+  }
+  __syncthreads();
+  double pn = 0.0, pd = 0.0;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    pn += num[j];
+    pd += den[j];
+  }
+  const double snum = block_sum(pn, red), sden = block_sum(pd, red);
+  const double a = snum / (sden + m.lambda * d);
+  double* Bh = b.Bm + (long long)h * d * d;
+  double* Ph = b.Pm + (long long)h * d * d;
+  float* Bp = b.Bp + (long long)h * d * d;
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const int i = e / d, j = e % d;
+    double v = 0.0;
+    if (i == j)
+      v = m.estimator == SPARSEPR_EST_SCALAR ? a
+        : m.estimator == SPARSEPR_EST_DIAGONAL ? num[j] / (den[j] + m.lambda) : 0.0;
+    Bh[e] = v;
+    Ph[e] = i == j ? 1.0 : 0.0;
+    Bp[e] = (float)(v / b.sX[hd + i]);
+  }
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const double bj = m.estimator == SPARSEPR_EST_SCALAR ? a
+                    : m.estimator == SPARSEPR_EST_DIAGONAL ? num[j] / (den[j] + m.lambda) : 0.0;
+    b.cvec[hd + j] = (float)(b.muR[hd + j] - b.muX[hd + j] / b.sX[hd + j] * bj);
+  }
+  if (threadIdx.x == 0) b.reff[h] = d;
+}
+
 sparsepr_status launch_fit(const Plan& p, cudaStream_t st) {
   const int d = p.dm.d, M = p.dm.M;
+  if (p.dm.estimator != SPARSEPR_EST_RIDGE) {
+    fit_simple_kernel<<<p.dm.H, kLinThreads, 0, st>>>(p.dm, p.b);
+    SPR_LAUNCH_OK();
+    return SPARSEPR_OK;
+  }
   // shared-memory path when the dual form applies and A, Y, S (M x d each) and the
   // M x M Gram fit next to the kernel's static arrays
   const size_t fast_smem = (size_t)(3 * M * d + M * M) * sizeof(double);

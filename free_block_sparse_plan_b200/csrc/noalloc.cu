@@ -90,6 +90,8 @@ extern "C" sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* pa
                                                        const int32_t* rows, int32_t nrows,
                                                        void* Out, void* stream) {
   if (!params || !Q || !K || !V || !rows || !Out) return SPARSEPR_ERR_ARG;
+  if (((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V)) & 15) != 0)
+    return SPARSEPR_ERR_ARG;              // the kernels read Q, K, V with 16-byte copies
   if (params->dtype != SPARSEPR_F32 && params->dtype != SPARSEPR_BF16) return SPARSEPR_ERR_DTYPE;
   if (params->H < 1 || params->N_q < 1 || params->N_k < 1) return SPARSEPR_ERR_SHAPE;
   if (params->d < 8 || params->d > kMaxD || params->d % 8) return SPARSEPR_ERR_SHAPE;

@@ -383,7 +383,9 @@ sparsepr_status launch_permute(const Plan& p, cudaStream_t st) {
   const int chunks = m.d * es / 16;
   const int blocks = 148 * 8;
   gather_kernel<<<blocks, 256, 0, st>>>(p.Q, p.b.Qp, p.b.permQ, p.b.invQ, m.H, m.Nq, chunks);
+  SPR_LAUNCH_OK();
   gather_kernel<<<blocks, 256, 0, st>>>(p.K, p.b.Kp, p.b.permK, nullptr, m.H, m.Nk, chunks);
+  SPR_LAUNCH_OK();
   gather_kernel<<<blocks, 256, 0, st>>>(p.V, p.b.Vp, p.b.permK, nullptr, m.H, m.Nk, chunks);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;

@@ -27,6 +27,7 @@ SPARSEPR_ERR_STATE = 7
 SPARSEPR_F32 = 0
 SPARSEPR_BF16 = 1
 SPARSEPR_ENGINE_AUTO = 0
+SPARSEPR_EST_RIDGE, SPARSEPR_EST_MEAN, SPARSEPR_EST_SCALAR, SPARSEPR_EST_DIAGONAL = 0, 1, 2, 3
 SPARSEPR_ENGINE_SIMT = 1
 
 EXPORTS = [
@@ -34,7 +35,7 @@ EXPORTS = [
     "CELL_COUNT", "CELL_IDS", "PROBES", "PROBE_COUNT", "KMEANS_ITERS", "OBJECTIVE", "PAIRS",
     "FACTOR_K", "FACTOR_Q", "EIG_K", "EIG_Q", "METRIC_K", "METRIC_Q", "PHI_K", "PHI_Q",
     "CENTRES_Q", "SCORES", "OSP", "ODENSE_PROBE", "FIT_MU_X", "FIT_MU_R", "FIT_S", "FIT_B",
-    "FIT_P", "FIT_REFF", "PROBE_DIST", "KBAR", "QBAR",
+    "FIT_P", "FIT_REFF", "PROBE_DIST", "KBAR", "QBAR", "KM_REASSIGNED",
 ]
 EXPORT_ID = {name: i for i, name in enumerate(EXPORTS)}
 
@@ -44,6 +45,7 @@ SYMBOLS = [
     "sparsepr_probe_fit", "sparsepr_correct", "sparsepr_forward", "sparsepr_dense_attention",
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
     "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
+    "sparsepr_launch_count",
 ]
 
 
@@ -52,7 +54,8 @@ class sparsepr_params(ctypes.Structure):
                 ("dtype", c_int32), ("M_s", c_int32), ("r_K", c_int32), ("r_Q", c_int32),
                 ("C_q", c_int32), ("C_k", c_int32), ("M", c_int32), ("r", c_int32),
                 ("lam", c_double), ("target_density", c_double),
-                ("kmeans_max_iter", c_int32), ("engine", c_int32), ("seed", c_uint64)]
+                ("kmeans_max_iter", c_int32), ("engine", c_int32), ("seed", c_uint64),
+                ("estimator", c_int32), ("reserved", c_int32)]
 
 
 class sparsepr_stats(ctypes.Structure):
@@ -102,6 +105,7 @@ def lib():
             "sparsepr_dense_rows_noalloc": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p,
                                                       c_int32, c_void_p, c_void_p]),
             "sparsepr_status_string": (c_char_p, [c_int32]),
+            "sparsepr_launch_count": (ctypes.c_ulonglong, []),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -109,6 +113,11 @@ def lib():
             fn.argtypes = args
         _lib = L
     return _lib
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(lib().sparsepr_launch_count())
 
 
 def status_string(status: int) -> str:
@@ -121,18 +130,20 @@ def _check(status: int, where: str):
 
 
 def make_params(H, N_q, N_k, d, dtype, M_s, r_K, r_Q, C_q, C_k, M, r, lam, target_density,
-                kmeans_max_iter=25, seed=0, engine=SPARSEPR_ENGINE_AUTO) -> sparsepr_params:
+                kmeans_max_iter=25, seed=0, engine=SPARSEPR_ENGINE_AUTO, estimator=0) -> sparsepr_params:
     if isinstance(dtype, str):
         dtype = {"f32": SPARSEPR_F32, "bf16": SPARSEPR_BF16}[dtype]
     return sparsepr_params(H=H, N_q=N_q, N_k=N_k, d=d, dtype=dtype, M_s=M_s, r_K=r_K, r_Q=r_Q,
                            C_q=C_q, C_k=C_k, M=M, r=r, lam=lam, target_density=target_density,
-                           kmeans_max_iter=kmeans_max_iter, engine=engine, seed=seed)
+                           kmeans_max_iter=kmeans_max_iter, engine=engine, seed=seed,
+                           estimator=estimator, reserved=0)
 
 
 def params_from_dict(p: dict, engine=SPARSEPR_ENGINE_AUTO) -> sparsepr_params:
     return make_params(p["H"], p["N_q"], p["N_k"], p["d"], p["dtype"], p["M_s"], p["r_K"],
                        p["r_Q"], p["C_q"], p["C_k"], p["M"], p["r"], p["lam"],
-                       p["target_density"], p["kmeans_max_iter"], p["seed"], engine)
+                       p["target_density"], p["kmeans_max_iter"], p["seed"], engine,
+                       p.get("estimator", 0))
 
 
 # ----------------------------------------------------------------------------------
@@ -255,6 +266,7 @@ def _export_layout(p: sparsepr_params, name: str):
         "FIT_B": (f64, (H, d, d)), "FIT_P": (f64, (H, d, d)), "FIT_REFF": (i32, (H,)),
         "PROBE_DIST": (f64, (H, p.N_q)), "KBAR": (f64, (H, p.C_k, d)),
         "QBAR": (f64, (H, p.C_q, d)),
+        "KM_REASSIGNED": (i64, (H, 2)),
     }[name]
 
 

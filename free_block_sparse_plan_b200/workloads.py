@@ -60,6 +60,7 @@ class Workload:
     rho: float
     kmeans_max_iter: int = 25
     seed: int = 0
+    estimator: int = 0          # 0 ridge, 1 mean-only, 2 scalar affine, 3 diagonal affine
 
     @property
     def centres(self) -> int:
@@ -75,7 +76,7 @@ class Workload:
                     M_s=self.M_s, r_K=self.r_K, r_Q=self.r_Q, C_q=self.C_q,
                     C_k=self.C_k, M=self.M, r=self.r, lam=self.lam,
                     target_density=self.rho, kmeans_max_iter=self.kmeans_max_iter,
-                    seed=self.seed)
+                    seed=self.seed, estimator=self.estimator)
 
 
 TINY = Workload("tiny-f32-1x1024x64", H=1, N=1024, d=64, dtype="f32",

@@ -30,6 +30,7 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *     Every call except sparsepr_get_stats, sparsepr_export and sparsepr_check only
  *     enqueues work on it and never synchronises the host.
+ *   - Q, K, V and Out must be 16-byte aligned (SPARSEPR_ERR_ARG otherwise).
  *   - The caller owns Q, K, V, Out and the workspace (device memory of at least
  *     sparsepr_workspace_size bytes, 256-byte aligned).  A plan handle is host memory
  *     owned by the library until sparsepr_destroy; it refers to, but does not own, the
@@ -72,6 +73,14 @@ typedef enum {
   SPARSEPR_ENGINE_SIMT = 1    /* fp32 CUDA-core engine for every dtype (reference path) */
 } sparsepr_engine;
 
+/* Residual estimator of sparsepr_probe_fit (paper S4.2; App. D.3, Table 4). */
+typedef enum {
+  SPARSEPR_EST_RIDGE = 0,     /* full weighted ridge B, projected on Psi_r (the method) */
+  SPARSEPR_EST_MEAN = 1,      /* weighted mean residual only (B = 0) */
+  SPARSEPR_EST_SCALAR = 2,    /* B = a I, penalty lambda d a^2, no projection */
+  SPARSEPR_EST_DIAGONAL = 3   /* B = diag(b), penalty lambda |b|^2, no projection */
+} sparsepr_estimator;
+
 /*
  * Problem and hyper-parameters of one call (paper S2, S4; values of the review page's
  * hyper-parameter table: r_K=48, r_Q=64, M=64, r=16, lambda=0.1).
@@ -89,6 +98,7 @@ typedef enum {
  *   kmeans_max_iter   Lloyd assignment steps at most (1..1000; the paper uses 25)
  *   engine            sparsepr_engine
  *   seed              seed of the SplitMix64 stream that draws the k-means initial rows
+ *   estimator         sparsepr_estimator (0, the method's weighted ridge, unless comparing)
  */
 typedef struct {
   int32_t H, N_q, N_k, d;
@@ -99,6 +109,8 @@ typedef struct {
   int32_t kmeans_max_iter;
   int32_t engine;
   uint64_t seed;
+  int32_t estimator;
+  int32_t reserved;          /* must be 0 */
 } sparsepr_params;
 
 typedef struct sparsepr_plan_s* sparsepr_plan_t;
@@ -236,7 +248,10 @@ typedef enum {
   SPARSEPR_X_PROBE_DIST = 33, /* double [H,N_q] squared phi_Q distance to the group centre */
   SPARSEPR_X_KBAR = 34,       /* double [H,C_k,d] K/V group key centroids (compact ids) */
   SPARSEPR_X_QBAR = 35,       /* double [H,C_q,d] query group centroids (compact ids) */
-  SPARSEPR_X_COUNT = 36
+  SPARSEPR_X_KM_REASSIGNED = 36,/* int64 [H,2] points the tensor-core k-means re-assigned,
+                                   summed over its steps (keys, queries); the others kept
+                                   their label by the distance bounds */
+  SPARSEPR_X_COUNT = 37
 } sparsepr_export_what;
 
 /* Size in bytes of an exported array for this plan. Host only. */
@@ -252,6 +267,12 @@ void sparsepr_destroy(sparsepr_plan_t plan);
 
 /* Static text for a status code. */
 const char* sparsepr_status_string(sparsepr_status status);
+
+/* Number of CUDA kernels this library has enqueued since it was loaded, over all threads
+ * and devices (a relaxed atomic counter; the difference of two readings around a region
+ * counts that region's launches when no other thread calls the library meanwhile).
+ * The paper has no counterpart: it serves measurement.  Never fails. */
+unsigned long long sparsepr_launch_count(void);
 
 #ifdef __cplusplus
 }

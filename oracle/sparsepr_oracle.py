@@ -379,7 +379,11 @@ class Fit:
     sigma: np.ndarray      # singular values of Omega^{1/2} R_bar
 
 
-def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int) -> Fit:
+ESTIMATORS = ("ridge", "mean", "scalar", "diagonal")   # codes 0..3 of the C ABI
+
+
+def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int,
+                 estimator: str = "ridge") -> Fit:
     """Coverage-weighted ridge fit of the residual on the sparse output.
 
     [P] App. A.3: weights normalised to unit sum give mu_x, mu_R and the elementwise
@@ -389,6 +393,12 @@ def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int
     minimiser is (X^T Omega X + lambda I)^-1 X^T Omega R.  [P] App. D.2 / [R] step 4: the
     centred prediction is projected on the leading r right singular vectors of
     Omega^{1/2} R_bar.
+
+    `estimator` selects the restricted corrections of [P] App. D.3 (Table 4), which
+    minimise the same weighted objective over a smaller family, with the same lambda, no
+    penalty on the mean and no projection (P = I): "mean" (B = 0, predict mu_R),
+    "scalar" (B = a I, penalty lambda d a^2), "diagonal" (B = diag(b), penalty
+    lambda sum_j b_j^2).
     """
     M, d = x.shape
     wt = w / w.sum()
@@ -398,6 +408,20 @@ def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int
     xb = (x - mu_x) / s
     Rb = R - mu_R
     omega = M * w / w.sum()
+    if estimator != "ridge":
+        if estimator == "mean":
+            B = np.zeros((d, d))
+        elif estimator == "scalar":
+            # d/da [sum_p omega_p ||Rb_p - a xb_p||^2 + lam d a^2] = 0
+            a = float(np.sum(omega[:, None] * xb * Rb)) / (float(np.sum(omega[:, None] * xb * xb)) + lam * d)
+            B = a * np.eye(d)
+        elif estimator == "diagonal":
+            # one column at a time: sum_p omega_p (Rb_pj - b_j xb_pj)^2 + lam b_j^2
+            b = (omega @ (xb * Rb)) / (omega @ (xb * xb) + lam)
+            B = np.diag(b)
+        else:
+            raise ValueError(estimator)
+        return Fit(mu_x, mu_R, s, B, np.eye(d), d, np.zeros(0))
     lhs = xb.T @ (omega[:, None] * xb) + lam * np.eye(d)
     rhs = xb.T @ (omega[:, None] * Rb)
     B = np.linalg.solve(lhs, rhs)
@@ -433,13 +457,14 @@ class Params:
     rho: float
     kmeans_max_iter: int = 25
     seed: int = 0
+    estimator: str = "ridge"
 
     @classmethod
     def from_dict(cls, p: Dict) -> "Params":
         return cls(d=p["d"], M_s=p["M_s"], r_K=p["r_K"], r_Q=p["r_Q"], C_q=p["C_q"],
                    C_k=p["C_k"], M=p["M"], r=p["r"], lam=p["lam"],
                    rho=p["target_density"], kmeans_max_iter=p["kmeans_max_iter"],
-                   seed=p["seed"])
+                   seed=p["seed"], estimator=ESTIMATORS[int(p.get("estimator", 0))])
 
 
 @dataclass
@@ -535,7 +560,7 @@ def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] 
     w = gq.sizes[a_of].astype(np.float64) / m_a[a_of]  # [R] step 4: w_p = |G_a^Q| / m_a
     x_probe = sparse_attention(Q, K, V, gq, gk, sel, probes)
     dense_probe = dense_attention(Q, K, V, probes)
-    fit = fit_residual(x_probe, dense_probe - x_probe, w, p.lam, p.r)
+    fit = fit_residual(x_probe, dense_probe - x_probe, w, p.lam, p.r, p.estimator)
     rows = np.arange(N_q) if rows is None else np.asarray(rows)
     osp = sparse_attention(Q, K, V, gq, gk, sel, rows)
     out = correct_rows(osp, fit)

@@ -166,6 +166,26 @@ def test_tiny_injected_stagewise():
     check_injected_head(plan, out[0].double().cpu().numpy(), res, 0, w)
 
 
+@pytest.mark.parametrize("est", [N.SPARSEPR_EST_MEAN, N.SPARSEPR_EST_SCALAR, N.SPARSEPR_EST_DIAGONAL])
+def test_restricted_estimators_match_oracle(est):
+    # App. D.3's mean-only, scalar and diagonal corrections, oracle labels injected
+    for w in (W.TINY.with_(estimator=est), W.MID.with_(H=2, estimator=est)):
+        inputs = W.make_inputs_torch(w, device="cuda")
+        ref = [oracle_head(w, h)[3] for h in range(w.H)]
+        labQ = torch.tensor(np.stack([r.part.km_Q.labels for r in ref]), dtype=torch.int32, device="cuda")
+        labK = torch.tensor(np.stack([r.part.km_K.labels for r in ref]), dtype=torch.int32, device="cuda")
+        plan, out, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK))
+        assert plan.check() == 0
+        B = plan.export("FIT_B")
+        for h, res in enumerate(ref):
+            if est == N.SPARSEPR_EST_MEAN:
+                assert np.all(B[h] == 0.0)
+            elif np.array_equal(plan.export("PROBES")[h], res.probes):
+                assert rel(B[h], res.fit.B) < 1e-4, h
+            assert np.array_equal(plan.export("FIT_P")[h], np.eye(w.d))
+            check_injected_head(plan, out[h].double().cpu().numpy(), res, h, w)
+
+
 def test_tiny_simt_engine_equals_auto():
     w = W.TINY
     _, out_a, inputs = gpu_call(w)

@@ -19,8 +19,8 @@ def built():
 
 def _declared_functions():
     text = open(os.path.join(ROOT, "include", "sparsepr.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:sparsepr_status|void|const char\*)\s+(sparsepr_\w+)\s*\(",
-                                 text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:sparsepr_status|void|const char\*|unsigned long long)\s+"
+                                 r"(sparsepr_\w+)\s*\(", text, re.M)))
 
 
 def test_every_declared_symbol_is_exported():
@@ -33,7 +33,8 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_struct_layout_matches_header():
-    assert ctypes.sizeof(N.sparsepr_params) == 80
+    assert ctypes.sizeof(N.sparsepr_params) == 88
+    assert N.sparsepr_params.estimator.offset == 80
     assert N.sparsepr_params.lam.offset == 48
     assert N.sparsepr_params.seed.offset == 72
 

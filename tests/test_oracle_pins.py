@@ -500,3 +500,69 @@ def test_full_call_correction_reduces_error():
         unprobed = np.setdiff1d(np.arange(Q.shape[0]), res.probes)
         err = lambda A: np.linalg.norm(A[unprobed] - dense[unprobed]) / np.linalg.norm(dense[unprobed])
         assert err(res.out) < 0.9 * err(res.osp)
+
+
+# ----------------------------------------------------------------------------------
+# Restricted estimators ([P] App. D.3, Table 4): each is the minimiser of the weighted
+# objective over its family, pinned against an augmented least-squares solve.
+
+def _fit_inputs(seed=3, M=12, d=5):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(M, d))
+    R = 0.3 * x @ rng.normal(size=(d, d)) + 0.05 * rng.normal(size=(M, d)) + 0.2
+    w = rng.uniform(0.5, 2.0, size=M)
+    return x, R, w
+
+
+def _standardised(x, R, w):
+    wt = w / w.sum()
+    mu_x, mu_R = wt @ x, wt @ R
+    s = np.sqrt(wt @ ((x - mu_x) ** 2) + O.STD_EPS)
+    return (x - mu_x) / s, R - mu_R, x.shape[0] * w / w.sum()
+
+
+def test_mean_only_estimator_predicts_the_weighted_mean_residual():
+    x, R, w = _fit_inputs()
+    f = O.fit_residual(x, R, w, 0.1, 4, "mean")
+    assert np.all(f.B == 0) and np.array_equal(f.P, np.eye(x.shape[1]))
+    xs = np.random.default_rng(9).normal(size=(7, x.shape[1]))
+    np.testing.assert_allclose(O.correct_rows(xs, f), xs + (w / w.sum()) @ R, rtol=1e-13)
+
+
+def test_scalar_estimator_matches_augmented_least_squares():
+    x, R, w = _fit_inputs()
+    lam, d = 0.7, x.shape[1]
+    xb, Rb, om = _standardised(x, R, w)
+    A = np.concatenate([(np.sqrt(om)[:, None] * xb).ravel(), [np.sqrt(lam * d)]])[:, None]
+    y = np.concatenate([(np.sqrt(om)[:, None] * Rb).ravel(), [0.0]])
+    a = np.linalg.lstsq(A, y, rcond=None)[0][0]
+    f = O.fit_residual(x, R, w, lam, 4, "scalar")
+    np.testing.assert_allclose(f.B, a * np.eye(d), rtol=1e-12, atol=1e-14)
+    assert np.array_equal(f.P, np.eye(d))
+
+
+def test_diagonal_estimator_matches_augmented_least_squares():
+    x, R, w = _fit_inputs(seed=5)
+    lam, d = 0.4, x.shape[1]
+    xb, Rb, om = _standardised(x, R, w)
+    b = np.empty(d)
+    for j in range(d):
+        A = np.concatenate([np.sqrt(om) * xb[:, j], [np.sqrt(lam)]])[:, None]
+        y = np.concatenate([np.sqrt(om) * Rb[:, j], [0.0]])
+        b[j] = np.linalg.lstsq(A, y, rcond=None)[0][0]
+    f = O.fit_residual(x, R, w, lam, 4, "diagonal")
+    np.testing.assert_allclose(f.B, np.diag(b), rtol=1e-12, atol=1e-14)
+
+
+def test_restricted_estimators_never_beat_ridge_on_the_weighted_objective():
+    # ridge minimises over all B, so its penalised objective is the smallest (r = d, P = I)
+    x, R, w = _fit_inputs(seed=11, M=20, d=4)
+    lam = 0.3
+    xb, Rb, om = _standardised(x, R, w)
+
+    def obj(B):
+        return float(np.sum(om[:, None] * (Rb - xb @ B) ** 2) + lam * np.sum(B * B))
+
+    ridge = O.fit_residual(x, R, w, lam, 4, "ridge")
+    for est in ("mean", "scalar", "diagonal"):
+        assert obj(ridge.B) <= obj(O.fit_residual(x, R, w, lam, 4, est).B) + 1e-12
