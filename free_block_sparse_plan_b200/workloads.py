@@ -20,6 +20,9 @@ Recipe (one head; every head draws from its own child seed):
     e_n = [sin(pi t/T), cos(pi t/T), sin(2 pi y/GH), cos(2 pi y/GH), sin(2 pi x/GW),
     cos(2 pi x/GW)] and G ~ N(0,1) of shape [6, d];
   * V ~ N(0, 1);
+  * call `step` s > 0 of a sequence (denoising steps) adds s * drift * (dmu_c(n) +
+    sigma * e_n) to K and Q and s * drift * e_n to V, with dmu ~ N(0, I_d) per centre and
+    e_n ~ N(0, I_d) drawn from the head's second seed stream (step 0 is unchanged);
   * logit-std calibration: sigma_hat = std(q_i . k_j / sqrt(d)) over 65536 random
     (i, j) pairs (all pairs when N*N <= 65536 * 16), then Q and K are each multiplied
     by sqrt(target / sigma_hat);
@@ -61,6 +64,9 @@ class Workload:
     kmeans_max_iter: int = 25
     seed: int = 0
     estimator: int = 0          # 0 ridge, 1 mean-only, 2 scalar affine, 3 diagonal affine
+    # position in a sequence of calls (denoising steps) and the drift per step
+    step: int = 0
+    drift: float = 0.05
 
     @property
     def centres(self) -> int:
@@ -176,6 +182,14 @@ def make_head(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
         Q += bias
         K += bias
     V = rng.standard_normal((N, d))
+    if w.step > 0:
+        # drift along a sequence of calls: the mixture centres and the token noise move
+        # by drift * step along fixed directions drawn from the head's second stream
+        drng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(w.seed, spawn_key=(h, 1))))
+        a = w.drift * w.step
+        K += a * (drng.standard_normal((w.centres, d))[cid] + w.sigma_k * drng.standard_normal((N, d)))
+        Q += a * (drng.standard_normal((w.centres, d))[cid] + w.sigma_q * drng.standard_normal((N, d)))
+        V += a * drng.standard_normal((N, d))
     if N * N <= 65536 * 16:
         logits = (Q @ K.T) / math.sqrt(d)
         sigma_hat = float(np.std(logits))

@@ -37,6 +37,14 @@ Readings where the pages are silent (each is listed in the design doc):
   S16 probe distance d_i is the squared distance to the group centre in phi_Q space
   S20 r = 0 means no subspace projection (P = I)
   S21 singular values <= 1e-10 * sigma_max are dropped before taking the leading r
+  W1  a warm factor update is F <- Z L^-T with Z = M F and L L^T = F^T Z (a Cholesky
+      factor), twice, then scaled to unit mean eigenvalue: F F^T = M F (F^T M F)^-1 F^T M,
+      which depends only on span(F); if F^T M F is not positive definite the call takes
+      the full eigendecomposition instead
+  W2  warm k-means starts label c at the previous call's original-space centroid of
+      label c mapped into the current coordinates (phi_K linear, phi_Q with its RMS
+      step); a label that was empty in the previous call has no centroid and takes the
+      fresh draw c of the counter-based init stream
 
 Parity status: every function here is pinned by tests in ``tests/test_oracle_*.py``
 except ``route_scores``, whose formula is a reading (S11) of a score the pages only
@@ -120,6 +128,35 @@ def eigen_factor(Msym: np.ndarray, r: int):
     return Ur * np.sqrt(lam / mean)[None, :], lam, Ur
 
 
+def subspace_factor(Msym: np.ndarray, F_prev: np.ndarray, steps: int = 2):
+    """Warm update of an eigenvalue-weighted factor ([P] App. C: later calls refresh the
+    metric factors with two subspace iterations started from the previous factors, using
+    a Cholesky factorisation).
+
+    Reading W1: each iteration multiplies by the metric, Z = M F, factors the projected
+    metric F^T M F = F^T Z = L L^T and takes F <- Z L^-T, so that
+    F F^T = M F (F^T M F)^-1 F^T M.  That product depends only on the subspace spanned
+    by F, and equals U_r Lambda_r U_r^T when the subspace is the leading eigenspace, i.e.
+    the eigen-weighted factor of `eigen_factor` up to a rotation of its columns (which
+    leaves every distance in the coordinates unchanged).  The result is scaled so its
+    eigenvalues, those of F^T F, have unit mean (S3).  Returns None when F^T M F is not
+    positive definite (the caller falls back to the full eigendecomposition).
+    """
+    F = np.array(F_prev, dtype=np.float64)
+    for _ in range(steps):
+        Z = Msym @ F
+        try:
+            L = np.linalg.cholesky(F.T @ Z)
+        except np.linalg.LinAlgError:
+            return None
+        F = np.linalg.solve(L, Z.T).T
+    r = F.shape[1]
+    mean = float(np.trace(F.T @ F)) / r
+    if not mean > 0.0:
+        return None
+    return F / math.sqrt(mean)
+
+
 # ----------------------------------------------------------------------------------
 # k-means ([P] S4.1, App. C: Lloyd iterations, fresh centres, at most 25 iterations)
 
@@ -154,13 +191,15 @@ def objective(X: np.ndarray, labels: np.ndarray, centres: np.ndarray) -> float:
     return float((diff * diff).sum())
 
 
-def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int) -> KMeansResult:
+def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int,
+           centres0: Optional[np.ndarray] = None) -> KMeansResult:
     """Lloyd's algorithm: assign to the nearest centre, move centres to member means.
 
+    Starts from the feature rows `init_idx`, or from `centres0` when given (warm start).
     S7: stop after `max_iter` assignment steps or as soon as an assignment step leaves
     every label unchanged.  The returned centres are the means of the returned labels.
     """
-    centres = X[init_idx].copy()
+    centres = X[init_idx].copy() if centres0 is None else np.array(centres0, dtype=np.float64)
     labels = None
     it = 0
     history = []
@@ -489,21 +528,65 @@ class Partition:
     qbar: np.ndarray
 
 
-def partition(Q, K, V, p: Params, head: int) -> Partition:
+@dataclass
+class WarmState:
+    """What one call of a sequence hands to the next ([P] App. C warm start), per head."""
+    F_K: np.ndarray          # d x r_K key factor
+    F_Q: np.ndarray          # d x r_Q query factor
+    kbar: np.ndarray         # C_k x d original-space key centroid of each label
+    k_used: np.ndarray       # bool C_k: label non-empty (rows of empty labels are unused)
+    qbar: np.ndarray         # C_q x d original-space query centroid of each label
+    q_used: np.ndarray       # bool C_q
+
+
+def warm_state(part: Partition, p: Params) -> WarmState:
+    """The state a finished partition leaves for the next call of the sequence."""
+    d = part.F_K.shape[0]
+    kb = np.zeros((p.C_k, d))
+    qb = np.zeros((p.C_q, d))
+    ku = np.zeros(p.C_k, dtype=bool)
+    qu = np.zeros(p.C_q, dtype=bool)
+    kb[part.gk.labels_used] = part.kbar
+    qb[part.gq.labels_used] = part.qbar
+    ku[part.gk.labels_used] = True
+    qu[part.gq.labels_used] = True
+    return WarmState(part.F_K.copy(), part.F_Q.copy(), kb, ku, qb, qu)
+
+
+def warm_centres(X: np.ndarray, fresh_idx: np.ndarray, used: np.ndarray,
+                 mapped: np.ndarray) -> np.ndarray:
+    """W2: label c starts at `mapped[c]` (the previous original-space centroid in the
+    current coordinates) when it was non-empty, else at the fresh draw X[fresh_idx[c]]."""
+    return np.where(used[:, None], mapped, X[fresh_idx])
+
+
+def partition(Q, K, V, p: Params, head: int, warm: Optional[WarmState] = None) -> Partition:
     N_q, N_k = Q.shape[0], K.shape[0]
     rows = sample_rows(N_q, p.M_s)
     M_K = key_metric(Q, rows)
-    F_K, lam_K, _ = eigen_factor(M_K, p.r_K)
+    F_K = subspace_factor(M_K, warm.F_K) if warm is not None else None
+    if F_K is None:
+        F_K, lam_K, _ = eigen_factor(M_K, p.r_K)
+    else:
+        lam_K = np.sort(np.linalg.eigvalsh(F_K.T @ F_K))[::-1]
     phiK = K @ F_K
-    km_K = kmeans(phiK, kmeans_init_indices(p.seed, head, 0, p.C_k, N_k), p.kmeans_max_iter)
+    idxK = kmeans_init_indices(p.seed, head, 0, p.C_k, N_k)
+    c0K = None if warm is None else warm_centres(phiK, idxK, warm.k_used, warm.kbar @ F_K)
+    km_K = kmeans(phiK, idxK, p.kmeans_max_iter, c0K)
     gk = compact_groups(km_K.labels, p.C_k)
     kbar = group_means(K, gk)
     vbar = group_means(V, gk)
     Ktil = centred_key_centroids(kbar)
     M_Q = query_metric(Ktil)
-    F_Q, lam_Q, _ = eigen_factor(M_Q, p.r_Q)
+    F_Q = subspace_factor(M_Q, warm.F_Q) if warm is not None else None
+    if F_Q is None:
+        F_Q, lam_Q, _ = eigen_factor(M_Q, p.r_Q)
+    else:
+        lam_Q = np.sort(np.linalg.eigvalsh(F_Q.T @ F_Q))[::-1]
     phiQ = query_coords(Q, F_Q)
-    km_Q = kmeans(phiQ, kmeans_init_indices(p.seed, head, 1, p.C_q, N_q), p.kmeans_max_iter)
+    idxQ = kmeans_init_indices(p.seed, head, 1, p.C_q, N_q)
+    c0Q = None if warm is None else warm_centres(phiQ, idxQ, warm.q_used, query_coords(warm.qbar, F_Q))
+    km_Q = kmeans(phiQ, idxQ, p.kmeans_max_iter, c0Q)
     gq = compact_groups(km_Q.labels, p.C_q)
     qbar = group_means(Q, gq)
     return Partition(rows, M_K, F_K, lam_K, phiK, km_K, gk, kbar, vbar, Ktil, M_Q, F_Q,
@@ -537,14 +620,16 @@ class CallResult:
 
 
 def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] = None,
-                  part: Optional[Partition] = None) -> CallResult:
+                  part: Optional[Partition] = None,
+                  warm: Optional[WarmState] = None) -> CallResult:
     """One SparsePR attention call for one head, in the pages' order.
 
     `rows` limits the rows whose sparse and corrected outputs are formed (the fit only
-    needs the probe rows); `part` reuses a partition computed earlier for this head.
+    needs the probe rows); `part` reuses a partition computed earlier for this head;
+    `warm` is the previous call's state in a sequence ([P] App. C warm start).
     """
     N_q, N_k = Q.shape[0], K.shape[0]
-    part = partition(Q, K, V, p, head) if part is None else part
+    part = partition(Q, K, V, p, head, warm) if part is None else part
     gq, gk = part.gq, part.gk
     S = route_scores(part.qbar, part.kbar, part.vbar, gk.sizes, p.d)
     beta = route_budget(p.rho, p.M, N_q, N_k)

@@ -566,3 +566,89 @@ def test_restricted_estimators_never_beat_ridge_on_the_weighted_objective():
     ridge = O.fit_residual(x, R, w, lam, 4, "ridge")
     for est in ("mean", "scalar", "diagonal"):
         assert obj(ridge.B) <= obj(O.fit_residual(x, R, w, lam, 4, est).B) + 1e-12
+
+
+# ---------------------------------------------------------------- warm start ([P] App. C)
+def _spd_with_spectrum(seed, lam):
+    rng = _rng(seed)
+    U, _ = np.linalg.qr(rng.standard_normal((lam.size, lam.size)))
+    return U @ np.diag(lam) @ U.T, U
+
+
+def test_subspace_factor_from_the_leading_eigenspace_is_the_eigen_factor():
+    # started anywhere inside the leading r-dimensional eigenspace (any basis), the
+    # update returns U_r diag(lam_r / mean lam_r) U_r^T, built here from the spectrum
+    lam = np.array([9.0, 7.0, 5.5, 4.0, 1.0, 0.5, 0.25, 0.1, 0.05, 0.01])
+    M, U = _spd_with_spectrum(21, lam)
+    r = 4
+    T = _rng(22).standard_normal((r, r)) + 3.0 * np.eye(r)
+    F = O.subspace_factor(M, U[:, :r] @ T)
+    want = U[:, :r] @ np.diag(lam[:r] / lam[:r].mean()) @ U[:, :r].T
+    assert np.abs(F @ F.T - want).max() < 1e-12 * np.abs(want).max()
+    assert abs(np.trace(F.T @ F) - r) < 1e-12
+
+
+def test_subspace_factor_at_full_rank_reproduces_the_metric():
+    # r = d: M F (F^T M F)^-1 F^T M = M for any invertible F, scaled to unit mean
+    lam = np.array([3.0, 2.0, 1.5, 0.7, 0.2, 0.1])
+    M, _ = _spd_with_spectrum(23, lam)
+    F = O.subspace_factor(M, _rng(24).standard_normal((6, 6)))
+    assert np.abs(F @ F.T - M / lam.mean()).max() < 1e-11
+
+
+def test_subspace_factor_iterated_converges_to_the_leading_eigenspace():
+    lam = np.array([10.0, 8.0, 6.0, 1.0, 0.8, 0.5, 0.3, 0.1])
+    M, U = _spd_with_spectrum(25, lam)
+    r = 3
+    F = O.subspace_factor(M, _rng(26).standard_normal((8, r)), steps=60)
+    want = U[:, :r] @ np.diag(lam[:r] / lam[:r].mean()) @ U[:, :r].T
+    assert np.abs(F @ F.T - want).max() < 1e-10
+
+
+def test_subspace_factor_depends_only_on_the_span_of_its_start():
+    lam = np.linspace(5.0, 0.1, 9)
+    M, _ = _spd_with_spectrum(27, lam)
+    F0 = _rng(28).standard_normal((9, 4))
+    T = _rng(29).standard_normal((4, 4)) + 2.0 * np.eye(4)
+    A = O.subspace_factor(M, F0)
+    B = O.subspace_factor(M, F0 @ T)
+    assert np.abs(A @ A.T - B @ B.T).max() < 1e-11
+
+
+def test_subspace_factor_reports_a_singular_projected_metric():
+    M = np.diag([1.0, 0.0, 2.0])
+    assert O.subspace_factor(M, np.array([[0.0], [1.0], [0.0]])) is None
+
+
+def test_warm_key_kmeans_restarts_at_its_fixed_point():
+    # the same inputs again: the previous key centroids in the original space, mapped by
+    # the (same) factor, are the converged centres, so the first assignment reproduces
+    # the converged labels and the second one confirms them
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY
+    p = O.Params.from_dict(w.params())
+    Q, K, V = W.make_head(w, 0)
+    cold = O.partition(Q, K, V, p, 0)
+    assert cold.km_K.iterations < p.kmeans_max_iter        # converged
+    warm = O.partition(Q, K, V, p, 0, O.warm_state(cold, p))
+    assert np.array_equal(warm.km_K.labels, cold.km_K.labels)
+    assert warm.km_K.iterations == 2
+    assert np.abs(warm.F_K @ warm.F_K.T - cold.F_K @ cold.F_K.T).max() < 1e-10
+
+
+def test_warm_kmeans_objective_is_monotone_and_empty_labels_redraw():
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY
+    p = O.Params.from_dict(w.params())
+    Q, K, V = W.make_head(w, 0)
+    st = O.warm_state(O.partition(Q, K, V, p, 0), p)
+    st.k_used[3] = False                                   # label 3 had no members
+    Q1, K1, V1 = W.make_head(w.with_(step=1), 0)
+    part = O.partition(Q1, K1, V1, p, 0, st)
+    h = part.km_K.history
+    assert all(b <= a * (1 + 1e-12) for a, b in zip(h, h[1:]))
+    idx = O.kmeans_init_indices(p.seed, 0, 0, p.C_k, w.N)
+    c0 = O.warm_centres(part.phiK, idx, st.k_used, st.kbar @ part.F_K)
+    assert np.array_equal(c0[3], part.phiK[idx[3]])
+    c = int(np.flatnonzero(st.k_used)[0])
+    assert np.allclose(c0[c], st.kbar[c] @ part.F_K, rtol=1e-13, atol=1e-13)
