@@ -170,6 +170,7 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
     b->kmShi = c.take<__nv_bfloat16>(H * Np * 64);
     b->kmSlo = c.take<__nv_bfloat16>(H * Np * 64);
   }
+  b->warmCold = c.take<int>(2 * H);
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);
 }
@@ -187,6 +188,7 @@ sparsepr_status make_plan(const sparsepr_params* q, const void* Q, const void* K
   if (ws_bytes < need) return SPARSEPR_ERR_WORKSPACE;
   carve(plan->dm, reinterpret_cast<char*>(ws), &plan->b);
   plan->Q = Q; plan->K = K; plan->V = V;
+  plan->warm = nullptr;
   plan->stage = 0;
   return SPARSEPR_OK;
 }
@@ -206,7 +208,7 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_CUDA_OK(cudaMemsetAsync(p.b.kmReassigned, 0, 2 * m.H * sizeof(long long), st));
   // key side (paper S4.1, App. B.1)
   SPR_TRY(launch_key_metric(p, st));
-  SPR_TRY(launch_eigen_factor(p, false, st));
+  SPR_TRY(p.warm ? launch_warm_factor(p, false, st) : launch_eigen_factor(p, false, st));
   SPR_TRY(launch_project_keys(p, st));
   if (labK) {
     SPR_CUDA_OK(cudaMemcpyAsync(p.b.labK, labK, sizeof(int) * m.H * m.Nk,
@@ -219,7 +221,7 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_TRY(launch_centroids(p, false, st));
   // query side (paper S4.1, App. B.2)
   SPR_TRY(launch_query_metric(p, st));
-  SPR_TRY(launch_eigen_factor(p, true, st));
+  SPR_TRY(p.warm ? launch_warm_factor(p, true, st) : launch_eigen_factor(p, true, st));
   SPR_TRY(launch_project_queries(p, st));
   if (labQ) {
     SPR_CUDA_OK(cudaMemcpyAsync(p.b.labQ, labQ, sizeof(int) * m.H * m.Nq,
@@ -304,12 +306,13 @@ sparsepr_status sparsepr_workspace_size(const sparsepr_params* params, size_t* b
 
 static sparsepr_status plan_common(const sparsepr_params* params, const void* Q, const void* K,
                                    const void* V, const int32_t* labQ, const int32_t* labK,
-                                   void* ws, size_t ws_bytes, void* stream,
+                                   const void* warm, void* ws, size_t ws_bytes, void* stream,
                                    sparsepr_plan_t* out) {
   if (out) *out = nullptr;
   sparsepr_plan_s* h = new (std::nothrow) sparsepr_plan_s();
   if (!h) return SPARSEPR_ERR_ARG;
   sparsepr_status s = make_plan(params, Q, K, V, ws, ws_bytes, out, &h->p);
+  h->p.warm = warm;
   if (s == SPARSEPR_OK) s = run_plan(h->p, labQ, labK, reinterpret_cast<cudaStream_t>(stream));
   if (s != SPARSEPR_OK) {
     delete h;
@@ -322,7 +325,28 @@ static sparsepr_status plan_common(const sparsepr_params* params, const void* Q,
 sparsepr_status sparsepr_plan(const sparsepr_params* params, const void* Q, const void* K,
                               const void* V, void* workspace, size_t workspace_bytes,
                               void* stream, sparsepr_plan_t* out) {
-  return plan_common(params, Q, K, V, nullptr, nullptr, workspace, workspace_bytes, stream, out);
+  return plan_common(params, Q, K, V, nullptr, nullptr, nullptr, workspace, workspace_bytes, stream, out);
+}
+
+sparsepr_status sparsepr_state_size(const sparsepr_params* params, size_t* bytes) {
+  sparsepr_status s = validate(params);
+  if (s != SPARSEPR_OK) return s;
+  if (!bytes) return SPARSEPR_ERR_ARG;
+  *bytes = state_layout(make_dims(params)).total;
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_plan_warm(const sparsepr_params* params, const void* Q, const void* K,
+                                   const void* V, const void* state, void* workspace,
+                                   size_t workspace_bytes, void* stream, sparsepr_plan_t* out) {
+  if (!state || (reinterpret_cast<uintptr_t>(state) & 255)) return SPARSEPR_ERR_ARG;
+  return plan_common(params, Q, K, V, nullptr, nullptr, state, workspace, workspace_bytes, stream, out);
+}
+
+sparsepr_status sparsepr_save_state(sparsepr_plan_t plan, void* state, void* stream) {
+  if (!plan || !state || (reinterpret_cast<uintptr_t>(state) & 255)) return SPARSEPR_ERR_ARG;
+  if (plan->p.stage < 1) return SPARSEPR_ERR_STATE;
+  return launch_save_state(plan->p, state, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sparsepr_status sparsepr_plan_from_labels(const sparsepr_params* params, const void* Q,
@@ -331,7 +355,7 @@ sparsepr_status sparsepr_plan_from_labels(const sparsepr_params* params, const v
                                           void* workspace, size_t workspace_bytes,
                                           void* stream, sparsepr_plan_t* out) {
   if (!labQ || !labK) return SPARSEPR_ERR_ARG;
-  return plan_common(params, Q, K, V, labQ, labK, workspace, workspace_bytes, stream, out);
+  return plan_common(params, Q, K, V, labQ, labK, nullptr, workspace, workspace_bytes, stream, out);
 }
 
 sparsepr_status sparsepr_attend(sparsepr_plan_t plan, void* stream) {

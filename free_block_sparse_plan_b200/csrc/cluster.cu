@@ -205,6 +205,72 @@ __global__ void km_init_kernel(KmView v, unsigned long long seed) {
   }
 }
 
+// Warm initialisation (paper App. C: later calls start from the previous centroids in
+// the original space, mapped into the current response coordinates): label c starts at
+// phi(cbar_c), phi(x) = x F for keys and (x F) / max(rms(x F), 1e-6) for queries, when
+// label c was non-empty in the previous call; otherwise at the fresh draw c of the
+// init stream.  A state that does not match the plan starts every label fresh.  One
+// warp per label, lanes over the coordinates.
+__global__ void __launch_bounds__(256) km_warm_init_kernel(KmView v, unsigned long long seed, Dims m,
+                                                           const int* hdr, const double* cprev,
+                                                           const int* used, const double* F) {
+  const int h = blockIdx.y, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (c >= v.C) return;
+  const int d = m.d, r = v.r;
+  double* out = v.cent + ((long long)h * v.C + c) * r;
+  if (state_matches(hdr, m) && used[(long long)h * v.C + c]) {
+    const double* cb = cprev + ((long long)h * v.C + c) * d;
+    const double* Fh = F + (long long)h * d * r;
+    double z0 = 0.0, z1 = 0.0;
+    for (int j = 0; j < d; ++j) {
+      const double x = cb[j];
+      if (lane < r) z0 += x * Fh[j * r + lane];
+      if (lane + 32 < r) z1 += x * Fh[j * r + lane + 32];
+    }
+    double sc = 1.0;
+    if (v.stage == 1) {
+      const double rms = sqrt(warp_sum(z0 * z0 + z1 * z1) / (double)r);
+      sc = 1.0 / (rms > 1e-6 ? rms : 1e-6);
+    }
+    if (lane < r) out[lane] = v.stage == 1 ? z0 * sc : z0;
+    if (lane + 32 < r) out[lane + 32] = v.stage == 1 ? z1 * sc : z1;
+  } else {
+    const unsigned long long key = sm64_mix(seed + (unsigned long long)(2 * h + v.stage + 1) * kGamma);
+    const unsigned long long z = sm64_mix(key + (unsigned long long)(c + 1) * kGamma);
+    const long long idx = (long long)(((z >> 32) * (unsigned long long)v.N) >> 32);
+    for (int k = lane; k < r; k += 32) out[k] = v.X[((long long)h * v.N + idx) * r + k];
+  }
+}
+
+// The state a finished plan leaves for the next call: header, factors, and per label
+// the original-space centroid (zero for an empty label) with its non-empty flag.
+__global__ void __launch_bounds__(1024) save_state_kernel(Dims m, Buffers b, char* state) {
+  const StateLayout L = state_layout(m);
+  const int h = blockIdx.x, d = m.d;
+  if (h == 0 && threadIdx.x < 16) {
+    const int vals[8] = {kStateMagic, m.H, m.d, m.rK, m.rQ, m.Ck, m.Cq, 1};
+    reinterpret_cast<int*>(state)[threadIdx.x] = threadIdx.x < 8 ? vals[threadIdx.x] : 0;
+  }
+  double* FK = reinterpret_cast<double*>(state + L.FK) + (long long)h * d * m.rK;
+  double* FQ = reinterpret_cast<double*>(state + L.FQ) + (long long)h * d * m.rQ;
+  for (int e = threadIdx.x; e < d * m.rK; e += blockDim.x) FK[e] = b.FK64[(long long)h * d * m.rK + e];
+  for (int e = threadIdx.x; e < d * m.rQ; e += blockDim.x) FQ[e] = b.FQ64[(long long)h * d * m.rQ + e];
+  for (int side = 0; side < 2; ++side) {
+    const int C = side ? m.Cq : m.Ck;
+    const int* comp = (side ? b.compQ : b.compK) + (long long)h * C;
+    const double* bar = (side ? b.qbar : b.kbar) + (long long)h * C * d;
+    double* cs = reinterpret_cast<double*>(state + (side ? L.QC : L.KC)) + (long long)h * C * d;
+    int* us = reinterpret_cast<int*>(state + (side ? L.qu : L.ku)) + (long long)h * C;
+    for (int e = threadIdx.x; e < C * d; e += blockDim.x) {
+      const int c = e / d, j = e % d;
+      const int g = comp[c];
+      cs[e] = g >= 0 ? bar[(long long)g * d + j] : 0.0;
+      if (j == 0) us[c] = g >= 0 ? 1 : 0;
+    }
+  }
+}
+
 // Assignment: label = argmin_c ||x - c||^2 (direct sum of squared differences in fp64,
 // dimensions in ascending order; ties to the lowest index).
 template <int R>
@@ -610,7 +676,16 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   const int H = p.dm.H;
   SPR_CUDA_OK(cudaMemsetAsync(v.km, 0, sizeof(int) * 4 * H, st));
   SPR_CUDA_OK(cudaMemsetAsync(v.lab, 0xFF, sizeof(int) * (size_t)H * v.N, st));  // labels = -1
-  km_init_kernel<<<H, 256, 0, st>>>(v, p.dm.seed);
+  if (p.warm) {
+    const StateLayout L = state_layout(p.dm);
+    const char* base = static_cast<const char*>(p.warm);
+    km_warm_init_kernel<<<dim3(cdiv(v.C, 8), H), 256, 0, st>>>(
+        v, p.dm.seed, p.dm, reinterpret_cast<const int*>(base),
+        reinterpret_cast<const double*>(base + (query ? L.QC : L.KC)),
+        reinterpret_cast<const int*>(base + (query ? L.qu : L.ku)), query ? p.b.FQ64 : p.b.FK64);
+  } else {
+    km_init_kernel<<<H, 256, 0, st>>>(v, p.dm.seed);
+  }
   SPR_LAUNCH_OK();
   // tensor-core scores with exact rescoring (labels identical to the fp32 full scan) when
   // there are enough centres to fill the tiles; the full scan otherwise or on request
@@ -625,7 +700,10 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   }
   for (int it = 0; it < p.dm.max_iter; ++it) {
     if (tc) {
-      sparsepr_status s = km_tc_assign(kb, v.X, v.cent, H, v.N, v.C, v.r, it, v.lab, v.km, b.err, st);
+      // the distance bounds pay where few points can move: a warm start begins near a
+      // fixed point; from fresh centres about half of the points stay undecided by them
+      sparsepr_status s = km_tc_assign(kb, v.X, v.cent, H, v.N, v.C, v.r, it, v.lab, v.km, b.err,
+                                       p.warm != nullptr, st);
       if (s != SPARSEPR_OK) return s;
     } else {
       if (v.r <= 8) assign<8>(v, H, it, st);
@@ -659,6 +737,12 @@ sparsepr_status launch_centroids(const Plan& p, bool query, cudaStream_t st) {
     centroid_kernel<<<dim3(m.Cq, m.H), kCentSub * kMaxD, 0, st>>>(m, p.Q, nullptr, m.Nq, m.Cq, b.permQ, b.offQ, b.usedQ, b.nQ, b.qbar, nullptr);
   else
     centroid_kernel<<<dim3(m.Ck, m.H), kCentSub * kMaxD, 0, st>>>(m, p.K, p.V, m.Nk, m.Ck, b.permK, b.offK, b.usedK, b.nK, b.kbar, b.vbar);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
+
+sparsepr_status launch_save_state(const Plan& p, void* state, cudaStream_t st) {
+  save_state_kernel<<<p.dm.H, 1024, 0, st>>>(p.dm, p.b, static_cast<char*>(state));
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

@@ -25,6 +25,7 @@ enum : int {
   kErrProbe = 8,       // probe selection could not find M rows
   kErrLabels = 16,     // an injected label was outside [0, C)
   kErrHang = 32,       // a pipeline wait timed out (the kernel abandoned its work)
+  kErrWarmState = 64,  // a warm state did not match the plan's dimensions (started cold)
 };
 
 // Problem dimensions, passed by value to kernels.
@@ -91,14 +92,41 @@ struct Buffers {
   long long *kmReassigned;   // points re-assigned, summed over the steps [2 sides][H]
   __nv_bfloat16 *kmShi, *kmSlo;  // their split coordinates, compacted [H][Npad][64]
   int *kmQcnt;               // queue lengths [2]
+  int *warmCold;             // heads whose warm factor update fell back to the eigensolve [2][H]
   int *err;                  // device error word
 };
+
+// Warm state handed from one call of a sequence to the next (paper App. C): a header,
+// the fp64 metric factors, and the original-space centroid of every label with a
+// non-empty flag.  Offsets in bytes from the state base; every block 256-byte aligned.
+constexpr int kStateMagic = 0x57525053;
+struct StateLayout {
+  size_t FK, FQ, KC, QC, ku, qu, total;
+};
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+__device__ inline bool state_matches(const int* hdr, const Dims& m) {
+  return hdr[0] == kStateMagic && hdr[1] == m.H && hdr[2] == m.d && hdr[3] == m.rK &&
+         hdr[4] == m.rQ && hdr[5] == m.Ck && hdr[6] == m.Cq && hdr[7] == 1;
+}
+__host__ __device__ inline StateLayout state_layout(const Dims& m) {
+  const size_t H = m.H, d = m.d;
+  StateLayout L;
+  L.FK = 256;                                          // header: 16 int32
+  L.FQ = L.FK + align256(H * d * m.rK * sizeof(double));
+  L.KC = L.FQ + align256(H * d * m.rQ * sizeof(double));
+  L.QC = L.KC + align256(H * (size_t)m.Ck * d * sizeof(double));
+  L.ku = L.QC + align256(H * (size_t)m.Cq * d * sizeof(double));
+  L.qu = L.ku + align256(H * (size_t)m.Ck * sizeof(int));
+  L.total = L.qu + align256(H * (size_t)m.Cq * sizeof(int));
+  return L;
+}
 
 // Host-side plan handle.
 struct Plan {
   Dims dm;
   Buffers b;
   const void *Q, *K, *V;
+  const void* warm;          // previous call's state (warm start), or null
   int stage;                 // 1 planned, 2 attended, 3 fitted
 };
 
@@ -198,6 +226,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
 // Stage launchers (defined in the .cu files; all enqueue on `st`, return a status).
 sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st);
 sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_warm_factor(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_save_state(const Plan& p, void* state, cudaStream_t st);
 sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st);
 sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st);
 sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st);
@@ -245,7 +275,7 @@ struct KmTcBuffers {
   int* qcnt;
 };
 sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const double* cent, int H, int N, int C,
-                             int r, int it, int* lab, int* kmstate, int* err, cudaStream_t st);
+                             int r, int it, int* lab, int* kmstate, int* err, bool bounds, cudaStream_t st);
 sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void* K,
                                        const void* V, void* Out, cudaStream_t st);
 

@@ -127,22 +127,34 @@ __device__ __forceinline__ float dist_floor(float a, double Eb, double x2) {
   return __double2float_rd(sqrt(fmax((double)a - Eb + x2, 0.0)) * (1.0 - 1e-9));
 }
 
-// Global tile index -> (head, tile within the head) over the compacted points of every
+// Points to assign in head h at this step: the compacted list when the distance bounds
+// are in use, else every point of a head that has not converged.
+template <bool B>
+__device__ __forceinline__ int step_count(const KmArgs& g, int h) {
+  return B ? g.acnt[h] : (g.km[4 * h] ? 0 : g.N);
+}
+
+// Global tile index -> (head, tile within the head) over the points to assign of every
 // head (ceil(count / 128) tiles each); queried with non-decreasing tiles.
+template <bool B>
 struct TileCursor {
-  const int* acnt;
+  const KmArgs* g;
   int h, base, nt;
   __device__ int head(long long t, int* lt) {
     while (t >= base + nt) {
       base += nt;
       ++h;
-      nt = (acnt[h] + kRows - 1) / kRows;
+      nt = (step_count<B>(*g, h) + kRows - 1) / kRows;
     }
     *lt = (int)(t - base);
     return h;
   }
 };
 
+// B: distance bounds in use (points listed by the filter, their rows compacted, bounds
+// written for the next step); without them every point of an unconverged head is
+// assigned from its own row and no bound is kept.
+template <bool B>
 __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __grid_constant__ KmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
@@ -153,7 +165,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
 
   // tiles of the points to re-assign (converged heads have none), split evenly over CTAs
   long long T = 0;
-  for (int h = 0; h < g.H; ++h) T += (g.acnt[h] + kRows - 1) / kRows;
+  for (int h = 0; h < g.H; ++h) T += (step_count<B>(g, h) + kRows - 1) / kRows;
   const long long t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
   const int ntiles = (int)(t1 - t0);
   if (blockIdx.x == 0 && tid == 0) {
@@ -189,7 +201,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = ms->tmem_base;
-  TileCursor act{g.acnt, -1, 0, 0};
+  TileCursor<B> act{&g, -1, 0, 0};
 
   if (warp == 8) {
     // ============================================================ TMA producer
@@ -277,14 +289,15 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
     int J = 0;
     int nfull0 = 0, nfull1 = 0;            // waits done on accFull[0][grp], accFull[1][grp]
     // per-point values of this group's next tile, loaded one tile ahead of their use
-    TileCursor pre{g.acnt, -1, 0, 0};
+    TileCursor<B> pre{&g, -1, 0, 0};
     float nxn = 0.0f, ncm = 0.0f;
     int nold = 0, nn = 0;
     auto point_vals = [&](int li2) {
       int lt2;
       const int h2 = pre.head(t0 + li2, &lt2);
       const int j2 = lt2 * kRows + r;
-      nn = j2 < g.acnt[h2] ? g.aidx[(long long)h2 * g.Npad + j2] : -1;
+      if (B) nn = j2 < g.acnt[h2] ? g.aidx[(long long)h2 * g.Npad + j2] : -1;
+      else nn = j2 < g.N ? j2 : -1;
       const long long pi2 = (long long)h2 * g.N + (nn >= 0 ? nn : 0);
       nxn = g.xn[pi2];
       nold = g.lab[pi2];
@@ -343,10 +356,10 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
               a1 = fminf(a1, fmaxf(a0, a));
               c0 = a < a0 ? cb + 4 * i4 + e : c0;
               a0 = fminf(a0, a);
-              gm[i4 >> 3] = fminf(gm[i4 >> 3], a);
+              if (B) gm[i4 >> 3] = fminf(gm[i4 >> 3], a);
             }
           }
-          if (live) {
+          if (B && live) {
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
               const int gi = cb / kGroup + s2;
@@ -410,7 +423,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       const float T = 4e-4f * xn * cm + 1e-5f * (xn + cm) * (xn + cm) + 1e-30f;
       int best = c0;
       if (!(a1 > a0 + T)) {
-        g.U[pi] = INFINITY;                          // near a tie: re-assign at the next step
+        if (B) g.U[pi] = INFINITY;                   // near a tie: re-assign at the next step
         const int full = nrec > 4 ? 1 : 0;
         const int slot = atomicAdd(g.qcnt + (g.it & 1), 1);
         if (slot < g.qcap) {
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
           const double d2 = exact_d2(x, cent + (long long)ci * g.r, g.r);
           if (d2 < bd) { bd = d2; best = ci; }
         }
-      } else {
+      } else if (B) {
         // the own centre is nearer than u; in its group every other centre scores at
         // least the runner-up a1 (the other groups' bounds were written above)
         g.U[pi] = sqrt(fmax((double)a0 + Eb + x2, 0.0)) * (1.0 + 1e-9);
@@ -655,23 +668,25 @@ bool km_tc_supported(int C) { return C >= 64 && C <= kMaxChunks * kChunk; }
 long long km_tc_queue_cap(int H, int N) { return (long long)H * N / 16 + 1024; }
 
 sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const double* cent, int H, int N, int C,
-                             int r, int it, int* lab, int* kmstate, int* err, cudaStream_t st) {
+                             int r, int it, int* lab, int* kmstate, int* err, bool bounds, cudaStream_t st) {
   if (!km_tc_supported(C)) return SPARSEPR_ERR_ARG;
   const int Npad = km_tc_npad(N), Cpad = km_tc_cpad(C);
   const int nch = cdiv(C, kChunk);
   const int Cw = nch > 1 ? kChunk : cdiv(C, 64) * 64;
   const int G = cdiv(C, kGroup);
-  const KmFilter f{kmstate, lab, kb.delta, kb.dmax, kb.U, kb.L, kb.aidx, kb.acnt, kb.reassigned, kb.xhi, kb.xlo,
-                   kb.shi, kb.slo, H, N, Npad, C, G, it};
-  km_filter_kernel<<<dim3(cdiv(N, 256), H), 256, 0, st>>>(f);
-  SPR_LAUNCH_OK();
+  if (bounds) {
+    const KmFilter f{kmstate, lab, kb.delta, kb.dmax, kb.U, kb.L, kb.aidx, kb.acnt, kb.reassigned, kb.xhi, kb.xlo,
+                     kb.shi, kb.slo, H, N, Npad, C, G, it};
+    km_filter_kernel<<<dim3(cdiv(N, 256), H), 256, 0, st>>>(f);
+    SPR_LAUNCH_OK();
+  }
   km_split_c_kernel<<<dim3(Cpad / 8, H), 256, 0, st>>>(cent, H, C, Cpad, r, it, kmstate, kb.chi, kb.clo,
                                                        kb.cn, kb.cmaxb);
   SPR_LAUNCH_OK();
   KmArgs g;
   g.G = G;
-  if (!make_map(&g.tm_xhi, kb.shi, (long long)H * Npad, kRows) ||
-      !make_map(&g.tm_xlo, kb.slo, (long long)H * Npad, kRows) ||
+  if (!make_map(&g.tm_xhi, bounds ? kb.shi : kb.xhi, (long long)H * Npad, kRows) ||
+      !make_map(&g.tm_xlo, bounds ? kb.slo : kb.xlo, (long long)H * Npad, kRows) ||
       !make_map(&g.tm_chi, kb.chi, (long long)H * Cpad, Cw) ||
       !make_map(&g.tm_clo, kb.clo, (long long)H * Cpad, Cw))
     return SPARSEPR_ERR_CUDA;
@@ -686,10 +701,11 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   g.X = X; g.cent = cent; g.err = err;
   g.H = H; g.N = N; g.Npad = Npad; g.C = C; g.Cpad = Cpad; g.Cw = Cw; g.nch = nch; g.r = r; g.it = it;
   g.slots = slots;
-  SPR_CUDA_OK(cudaFuncSetAttribute(km_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  auto kern = bounds ? km_assign_tc_kernel<true> : km_assign_tc_kernel<false>;
+  SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const long long tiles = (long long)H * (Npad / kRows);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  km_assign_tc_kernel<<<grid, kKmThreads, smem, st>>>(g);
+  kern<<<grid, kKmThreads, smem, st>>>(g);
   SPR_LAUNCH_OK();
   km_rescore_kernel<<<4 * sm_count(), 256, 0, st>>>(kb.queue, kb.qcnt, g.qcap, X, cent, lab, kmstate, N, C, r,
                                                     it);

@@ -157,12 +157,14 @@ __device__ __forceinline__ int desc_rank(const double* key, int n, int j) {
 __global__ void __launch_bounds__(kLinThreads) eigen_factor_kernel(Dims m, const double* Mall,
                                                                    int r, double* lam_out,
                                                                    double* F64, float* F32,
-                                                                   int* err, int err_bit) {
+                                                                   int* err, int err_bit,
+                                                                   const int* only) {
   extern __shared__ double G[];          // [d][d] column-major
   __shared__ double norm[kMaxD], lam[kMaxD], red[32], hnrm[kMaxD];
   __shared__ int rank[kMaxD];
   __shared__ int flag;
   const int h = blockIdx.x, d = m.d;
+  if (only && only[h] == 0) return;      // warm plan: this head's factor is already updated
   const double* Mh = Mall + (long long)h * d * d;
   for (int e = threadIdx.x; e < d * d; e += blockDim.x) G[e] = Mh[e];  // symmetric
   __syncthreads();
@@ -251,6 +253,89 @@ __device__ void cholesky_solve(const double* L, int n, double* Z, int ldz, int n
     }
   }
   __syncthreads();
+}
+
+// ---------------------------------------------------------------------------------
+// Warm update of an eigenvalue-weighted factor (paper App. C: later calls refresh the
+// metric factors by two subspace iterations started from the previous factors, with a
+// Cholesky factorisation).  Each iteration: Z = M F, L L^T = F^T Z, F <- Z L^-T, so that
+// F F^T = M F (F^T M F)^-1 F^T M, a function of span(F) alone that equals the
+// eigen-weighted U_r Lambda_r U_r^T when the span is the leading eigenspace.  The result
+// is scaled to unit mean eigenvalue (trace F^T F = r).  F and Z live in shared memory
+// with rows padded to r + 1 doubles; M is read from global memory (L2-resident).  A head
+// whose saved state does not match the plan, or whose F^T M F is not positive definite,
+// is flagged in `cold` and left to the full eigendecomposition.
+__global__ void __launch_bounds__(kLinThreads) subspace_factor_kernel(
+    Dims m, const double* Mall, const int* hdr, const double* Fprev, int r, double* lam_out,
+    double* F64, float* F32, int* cold, int* err) {
+  extern __shared__ double sm[];
+  __shared__ double red[32];
+  __shared__ int bad;
+  const int h = blockIdx.x, d = m.d, rs = r + 1;
+  double* Fs = sm;                 // [d][rs]
+  double* Zs = Fs + d * rs;        // [d][rs]
+  double* G = Zs + d * rs;         // [r][r]
+  if (!state_matches(hdr, m)) {
+    if (threadIdx.x == 0) {
+      cold[h] = 1;
+      atomicOr(err, kErrWarmState);
+    }
+    return;
+  }
+  const double* Mh = Mall + (long long)h * d * d;
+  const double* Fp = Fprev + (long long)h * d * r;
+  for (int e = threadIdx.x; e < d * r; e += blockDim.x) Fs[(e / r) * rs + e % r] = Fp[e];
+  for (int step = 0; step < 2; ++step) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < d * r; e += blockDim.x) {      // Z = M F
+      const int i = e / r, k = e % r;
+      double v = 0.0;
+      for (int j = 0; j < d; ++j) v += Mh[i * d + j] * Fs[j * rs + k];
+      Zs[i * rs + k] = v;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < r * r; e += blockDim.x) {      // G = F^T Z
+      const int a = e / r, c = e % r;
+      double v = 0.0;
+      for (int i = 0; i < d; ++i) v += Fs[i * rs + a] * Zs[i * rs + c];
+      G[e] = v;
+    }
+    __syncthreads();
+    if (!cholesky(G, r, &bad)) {                                  // uniform across the block
+      if (threadIdx.x == 0) cold[h] = 1;
+      return;
+    }
+    // F L^T = Z, column by column: F_k = Z_k / L_kk, then Z_c -= F_k L_ck for c > k
+    for (int k = 0; k < r; ++k) {
+      const double piv = G[k * r + k];
+      for (int i = threadIdx.x; i < d; i += blockDim.x) Fs[i * rs + k] = Zs[i * rs + k] / piv;
+      __syncthreads();
+      const int rem = r - k - 1;
+      for (int e = threadIdx.x; e < d * rem; e += blockDim.x) {
+        const int i = e / rem, c = k + 1 + e % rem;
+        Zs[i * rs + c] -= Fs[i * rs + k] * G[c * r + k];
+      }
+      __syncthreads();
+    }
+  }
+  double part = 0.0;
+  for (int e = threadIdx.x; e < d * r; e += blockDim.x) {
+    const double f = Fs[(e / r) * rs + e % r];
+    part += f * f;
+  }
+  const double mean = block_sum(part, red) / (double)r;
+  if (!(mean > 0.0) || !isfinite(mean)) {
+    if (threadIdx.x == 0) cold[h] = 1;
+    return;
+  }
+  const double sc = 1.0 / sqrt(mean);
+  for (int e = threadIdx.x; e < d * r; e += blockDim.x) {
+    const double v = Fs[(e / r) * rs + e % r] * sc;
+    F64[(long long)h * d * r + e] = v;
+    F32[(long long)h * d * r + e] = (float)v;
+  }
+  // the columns are not eigenvectors: the eigenvalue export is left at zero
+  for (int k = threadIdx.x; k < r; k += blockDim.x) lam_out[(long long)h * r + k] = 0.0;
 }
 
 __global__ void __launch_bounds__(kLinThreads) fit_kernel(Dims m, Buffers b) {
@@ -575,12 +660,32 @@ sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st) {
 sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st) {
   const size_t smem = (size_t)p.dm.d * p.dm.d * sizeof(double);
   SPR_CUDA_OK(cudaFuncSetAttribute(eigen_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int* only = p.warm ? p.b.warmCold + (query ? p.dm.H : 0) : nullptr;
   if (query)
-    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MQ, p.dm.rQ, p.b.lamQ, p.b.FQ64, p.b.FQ, p.b.err, kErrEigQ);
+    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MQ, p.dm.rQ, p.b.lamQ, p.b.FQ64, p.b.FQ, p.b.err, kErrEigQ, only);
   else
-    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MK, p.dm.rK, p.b.lamK, p.b.FK64, p.b.FK, p.b.err, kErrEigK);
+    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MK, p.dm.rK, p.b.lamK, p.b.FK64, p.b.FK, p.b.err, kErrEigK, only);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
+}
+
+// Warm plans: the subspace update from the saved factor, then the full eigendecomposition
+// for the heads it flagged (a launch whose other blocks return at once).
+sparsepr_status launch_warm_factor(const Plan& p, bool query, cudaStream_t st) {
+  const Dims& m = p.dm;
+  const int r = query ? m.rQ : m.rK;
+  const StateLayout L = state_layout(m);
+  const char* base = static_cast<const char*>(p.warm);
+  const size_t smem = (size_t)(2 * m.d * (r + 1) + r * r) * sizeof(double);
+  SPR_CUDA_OK(cudaFuncSetAttribute(subspace_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int* cold = p.b.warmCold + (query ? m.H : 0);
+  SPR_CUDA_OK(cudaMemsetAsync(cold, 0, sizeof(int) * m.H, st));
+  subspace_factor_kernel<<<m.H, kLinThreads, smem, st>>>(
+      m, query ? p.b.MQ : p.b.MK, reinterpret_cast<const int*>(base),
+      reinterpret_cast<const double*>(base + (query ? L.FQ : L.FK)), r,
+      query ? p.b.lamQ : p.b.lamK, query ? p.b.FQ64 : p.b.FK64, query ? p.b.FQ : p.b.FK, cold, p.b.err);
+  SPR_LAUNCH_OK();
+  return launch_eigen_factor(p, query, st);
 }
 
 // Restricted estimators (paper App. D.3, Table 4), one CTA per head: the statistics of

@@ -43,7 +43,6 @@ sparsepr_status scratch_address(void** out) {
   return SPARSEPR_OK;
 }
 
-size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 // Copies the requested rows into the scratch array once per head (the partial-attention
 // kernels read a [H][nrows] row list), clamped to [0, N_q) so that no later kernel can

@@ -45,7 +45,7 @@ SYMBOLS = [
     "sparsepr_probe_fit", "sparsepr_correct", "sparsepr_forward", "sparsepr_dense_attention",
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
     "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
-    "sparsepr_launch_count",
+    "sparsepr_launch_count", "sparsepr_state_size", "sparsepr_save_state", "sparsepr_plan_warm",
 ]
 
 
@@ -106,6 +106,10 @@ def lib():
                                                       c_int32, c_void_p, c_void_p]),
             "sparsepr_status_string": (c_char_p, [c_int32]),
             "sparsepr_launch_count": (ctypes.c_ulonglong, []),
+            "sparsepr_state_size": (c_int32, [P, POINTER(c_size_t)]),
+            "sparsepr_save_state": (c_int32, [c_void_p, c_void_p, c_void_p]),
+            "sparsepr_plan_warm": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_size_t, c_void_p, POINTER(c_void_p)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -168,6 +172,23 @@ def sparsepr_plan_from_labels(params, Q, K, V, labQ, labK, workspace, workspace_
     _check(lib().sparsepr_plan_from_labels(ctypes.byref(params), Q, K, V, labQ, labK, workspace,
                                            workspace_bytes, stream, ctypes.byref(h)),
            "sparsepr_plan_from_labels")
+    return h
+
+
+def sparsepr_state_size(params: sparsepr_params) -> int:
+    n = c_size_t()
+    _check(lib().sparsepr_state_size(ctypes.byref(params), ctypes.byref(n)), "sparsepr_state_size")
+    return n.value
+
+
+def sparsepr_save_state(plan, state, stream):
+    _check(lib().sparsepr_save_state(plan, state, stream), "sparsepr_save_state")
+
+
+def sparsepr_plan_warm(params, Q, K, V, state, workspace, workspace_bytes, stream):
+    h = c_void_p()
+    _check(lib().sparsepr_plan_warm(ctypes.byref(params), Q, K, V, state, workspace,
+                                    workspace_bytes, stream, ctypes.byref(h)), "sparsepr_plan_warm")
     return h
 
 
@@ -273,7 +294,10 @@ def _export_layout(p: sparsepr_params, name: str):
 class Plan:
     """A planned SparsePR call over device tensors Q, K, V [H, N, d] (fp32 or bf16)."""
 
-    def __init__(self, params: sparsepr_params, Q, K, V, workspace=None, labels=None, stream=None):
+    def __init__(self, params: sparsepr_params, Q, K, V, workspace=None, labels=None, stream=None,
+                 warm=None):
+        """`warm`: a state tensor written by `save_state` of the previous call of a sequence
+        (cross-call warm start); `labels`: injected k-means labels (testing)."""
         import torch
         self.params = params
         self.inputs = (Q, K, V)          # keep alive until the plan is destroyed
@@ -282,7 +306,11 @@ class Plan:
             workspace = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
         self.workspace = workspace
         st = _stream(stream)
-        if labels is None:
+        if warm is not None:
+            self._warm = warm
+            self.handle = sparsepr_plan_warm(params, _ptr(Q), _ptr(K), _ptr(V), _ptr(warm),
+                                             _ptr(workspace), workspace.numel(), st)
+        elif labels is None:
             self.handle = sparsepr_plan(params, _ptr(Q), _ptr(K), _ptr(V), _ptr(workspace),
                                         workspace.numel(), st)
         else:
@@ -294,6 +322,14 @@ class Plan:
 
     def attend(self, stream=None):
         sparsepr_attend(self.handle, _stream(stream))
+
+    def save_state(self, state=None, stream=None):
+        """Writes this call's warm state into `state` (a device uint8 tensor of
+        `state_size(params)` bytes, allocated when None) and returns it."""
+        if state is None:
+            state = new_state(self.params, self.inputs[0].device)
+        sparsepr_save_state(self.handle, _ptr(state), _stream(stream))
+        return state
 
     def probe_fit(self, stream=None):
         sparsepr_probe_fit(self.handle, _stream(stream))
@@ -330,6 +366,12 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def new_state(params: sparsepr_params, device):
+    """An uninitialised warm-state buffer (torch allocations are 256-byte aligned)."""
+    import torch
+    return torch.empty(sparsepr_state_size(params), dtype=torch.uint8, device=device)
 
 
 def forward(params: sparsepr_params, Q, K, V, out=None, workspace=None, stream=None):

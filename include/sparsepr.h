@@ -154,6 +154,37 @@ sparsepr_status sparsepr_plan_from_labels(const sparsepr_params* params, const v
                                           void* workspace, size_t workspace_bytes,
                                           void* stream, sparsepr_plan_t* out);
 
+/*
+ * Cross-call warm start ("Partition the Support, Reconstruct the Residual", App. C:
+ * later calls of a denoising sequence start the k-means from the previous centroids in
+ * the original space, mapped into the current response coordinates, and refresh the
+ * metric factors by two subspace iterations with a Cholesky factorisation instead of a
+ * full eigendecomposition).
+ *
+ * The state is caller-owned DEVICE memory of sparsepr_state_size bytes, 256-byte
+ * aligned.  It holds a header (the dimensions it was saved for), the fp64 factors F_K
+ * [H,d,r_K] and F_Q [H,d,r_Q], and for every k-means label its original-space centroid
+ * (fp64 [H,C_k,d] and [H,C_q,d]) with a non-empty flag; the layout is internal.
+ *
+ * sparsepr_save_state writes a planned call's state (asynchronous, any time after
+ * sparsepr_plan*; the plan keeps its own copies).  sparsepr_plan_warm is sparsepr_plan
+ * started from a saved state: per head, the factor update is
+ * F <- Z L^-T with Z = M F, L L^T = F^T Z, twice, then scaled to unit mean eigenvalue;
+ * label c of each k-means starts at phi(cbar_c) when it was non-empty, else at the fresh
+ * draw c.  A head whose F^T M F is not positive definite takes the full
+ * eigendecomposition.  A state saved for other dimensions (or never saved) makes every
+ * head start cold and sets the device error word (SPARSEPR_ERR_DEVICE_CHECK from
+ * sparsepr_check).  The state is read by work enqueued on `stream`; saving the new
+ * plan's state into the same buffer later on the same stream is allowed.  After a warm
+ * plan, the EIG_K / EIG_Q exports are zero for the heads updated this way.
+ * Errors: SPARSEPR_ERR_ARG for a null or misaligned state; otherwise as sparsepr_plan.
+ */
+sparsepr_status sparsepr_state_size(const sparsepr_params* params, size_t* bytes);
+sparsepr_status sparsepr_save_state(sparsepr_plan_t plan, void* state, void* stream);
+sparsepr_status sparsepr_plan_warm(const sparsepr_params* params, const void* Q, const void* K,
+                                   const void* V, const void* state, void* workspace,
+                                   size_t workspace_bytes, void* stream, sparsepr_plan_t* out);
+
 /* Renormalised hard-drop attention over the selected cells; the sparse output stays in
  * the workspace (group-major, fp32).  Requires a plan.  Asynchronous. */
 sparsepr_status sparsepr_attend(sparsepr_plan_t plan, void* stream);

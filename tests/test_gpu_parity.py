@@ -181,9 +181,90 @@ def test_restricted_estimators_match_oracle(est):
             if est == N.SPARSEPR_EST_MEAN:
                 assert np.all(B[h] == 0.0)
             elif np.array_equal(plan.export("PROBES")[h], res.probes):
-                assert rel(B[h], res.fit.B) < 1e-4, h
+                # B is a least-squares coefficient of the residuals R = dense - sparse on the
+                # standardised features; where the two barely correlate B is near zero and
+                # its relative error means nothing.  Its error is measured on what it
+                # predicts, x_bar (B - B_ref), against what it fits, R_bar (both weighted by
+                # omega).  To first order a weighted least-squares fit moves by at most the
+                # perturbation of its targets plus twice that of its features, so the bound
+                # is taken from the GPU's own residuals and features against the oracle's.
+                om = np.sqrt(w.M * res.weights / res.weights.sum())[:, None]
+                osp = plan.export("OSP")[h]
+                rows = np.empty_like(osp)
+                rows[plan.export("PERM_Q")[h]] = osp
+                x_gpu = rows[res.probes]
+                R_gpu = plan.export("ODENSE_PROBE")[h] - x_gpu
+                x, R = res.x_probe, res.dense_probe - res.x_probe
+                xb = (x - res.fit.mu_x) / res.fit.s
+                Rb_n = np.linalg.norm(om * (R - res.fit.mu_R))
+                err = np.linalg.norm(om * (xb @ (B[h] - res.fit.B))) / Rb_n
+                eps_R = np.linalg.norm(om * (R_gpu - R)) / Rb_n
+                eps_x = np.linalg.norm(x_gpu - x) / np.linalg.norm(x - res.fit.mu_x)
+                # on the bf16 path the residual (0.35% of the output at the mid shape) is
+                # as small as the rounding of the bf16 probabilities, so eps_R is large
+                # there and only the bound below (and the output check) apply
+                if w.dtype == "f32":
+                    assert eps_R < 1e-3, (h, eps_R)
+                assert err < 3.0 * (eps_R + eps_x) + 1e-4, (h, err, eps_R, eps_x)
             assert np.array_equal(plan.export("FIT_P")[h], np.eye(w.d))
             check_injected_head(plan, out[h].double().cpu().numpy(), res, h, w)
+
+
+def _ff(F):
+    return F @ F.T
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_warm_start_sequence_matches_oracle(name):
+    # App. C warm start: call 0 cold, call 1 on drifted inputs from call 0's saved state
+    # (factors by two Cholesky subspace iterations, k-means from the previous centroids)
+    w0 = W.TINY if name == "tiny" else W.MID.with_(H=2)
+    w1 = w0.with_(step=1)
+    params = N.params_from_dict(w0.params())
+    P = O.Params.from_dict(w0.params())
+    plan0 = N.Plan(params, *W.make_inputs_torch(w0, device="cuda"))
+    state = plan0.save_state()
+    plan1 = N.Plan(params, *W.make_inputs_torch(w1, device="cuda"), warm=state)
+    plan1.attend()
+    plan1.probe_fit()
+    out = plan1.correct()
+    torch.cuda.synchronize()
+    assert plan1.check() == 0
+    FK, FQ = plan1.export("FACTOR_K"), plan1.export("FACTOR_Q")
+    labK, labQ = plan1.export("LABELS_K"), plan1.export("LABELS_Q")
+    iters, obj = plan1.export("KMEANS_ITERS"), plan1.export("OBJECTIVE")
+    rows = None if w0.N <= 4096 else (np.arange(2048) * w0.N) // 2048
+    for h in range(w0.H):
+        q0, k0, v0 = W.make_head(w0, h)
+        st = O.warm_state(O.partition(q0, k0, v0, P, h), P)
+        res = O.sparsepr_call(*W.make_head(w1, h), P, head=h, rows=rows, warm=st)
+        part = res.part
+        assert rel(_ff(FK[h]), _ff(part.F_K)) < 1e-10
+        assert rel(_ff(FQ[h]), _ff(part.F_Q)) < 1e-10
+        assert np.mean(labK[h] == part.km_K.labels) >= 0.999
+        assert np.mean(labQ[h] == part.km_Q.labels) >= 0.999
+        assert abs(obj[h][0] - part.km_K.objective) <= 1e-4 * part.km_K.objective
+        assert abs(obj[h][1] - part.km_Q.objective) <= 1e-4 * part.km_Q.objective
+        if np.array_equal(labK[h], part.km_K.labels) and np.array_equal(labQ[h], part.km_Q.labels):
+            assert tuple(iters[h]) == (part.km_K.iterations, part.km_Q.iterations)
+            assert rel(out[h].double().cpu().numpy()[res.rows], res.out) < TOL[w0.dtype]
+
+
+def test_warm_state_that_was_never_saved_starts_cold_and_is_flagged():
+    w = W.TINY
+    inputs = W.make_inputs_torch(w, device="cuda")
+    params = N.params_from_dict(w.params())
+    cold, out_c, _ = gpu_call(w, inputs=inputs)
+    state = torch.zeros(N.sparsepr_state_size(params), dtype=torch.uint8, device="cuda")
+    plan = N.Plan(params, *inputs, warm=state)
+    plan.attend()
+    plan.probe_fit()
+    out = plan.correct()
+    torch.cuda.synchronize()
+    assert plan.check() == 64                                  # the warm-state bit alone
+    assert np.array_equal(plan.export("LABELS_K"), cold.export("LABELS_K"))
+    assert np.array_equal(plan.export("LABELS_Q"), cold.export("LABELS_Q"))
+    assert torch.equal(out, out_c)
 
 
 def test_tiny_simt_engine_equals_auto():
