@@ -381,14 +381,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       const bool whole = valid == kTileKeys;           // uniform: no key column masked
       float mx = -INFINITY;
       if (whole) {
+        // two 32-column loads per wait, four independent max chains
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(tS + 32 * c, v);
+        for (int c = 0; c < 4; c += 2) {
+          float v[64];
+          tc::tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(v));
+          tc::tmem_ld32(tS + 32 * c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
+          for (int i = 0; i < 64; ++i) m4[i & 3] = fmaxf(m4[i & 3], v[i]);
         }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       } else {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -426,24 +430,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       }
       float rs = 0.0f;
       if (whole) {
+        // two 32-column loads per wait; four independent partial sums
+        float r4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(tS + 32 * c, v);
+        for (int c = 0; c < 4; c += 2) {
+          float v[64];
+          tc::tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(v));
+          tc::tmem_ld32(tS + 32 * c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 32; ++i) {
             const float x0 = fmaf(v[2 * i], sl2, -m_run), x1 = fmaf(v[2 * i + 1], sl2, -m_run);
             // a quarter of the exponentials on the FMA pipe, the rest on the SFU
-            const float p0 = i >= 16 - kPolyPairs ? tc::exp2_poly(x0) : tc::ex2(x0);
-            const float p1 = i >= 16 - kPolyPairs ? tc::exp2_poly(x1) : tc::ex2(x1);
-            rs += p0 + p1;
+            const bool poly = (i & 15) >= 16 - kPolyPairs;
+            const float p0 = poly ? tc::exp2_poly(x0) : tc::ex2(x0);
+            const float p1 = poly ? tc::exp2_poly(x1) : tc::ex2(x1);
+            r4[i & 3] += p0 + p1;
             pk[i] = tc::pack_bf16x2(p0, p1);
           }
-          // P columns 16c..16c+15 lie inside S columns already read (chunks 0..c)
-          tc::tmem_st16(tS + 16 * c, pk);
+          // P columns 16c..16c+31 lie inside S columns already read (chunks 0..c+1)
+          tc::tmem_st16(tS + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
+          tc::tmem_st16(tS + 16 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
         }
+        rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
       } else {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
