@@ -67,6 +67,12 @@ class Workload:
     # position in a sequence of calls (denoising steps) and the drift per step
     step: int = 0
     drift: float = 0.05
+    # grouped-query attention: G query heads share each K/V head (H/G K/V heads)
+    G: int = 1
+
+    @property
+    def H_kv(self) -> int:
+        return self.H // self.G
 
     @property
     def centres(self) -> int:
@@ -82,7 +88,7 @@ class Workload:
                     M_s=self.M_s, r_K=self.r_K, r_Q=self.r_Q, C_q=self.C_q,
                     C_k=self.C_k, M=self.M, r=self.r, lam=self.lam,
                     target_density=self.rho, kmeans_max_iter=self.kmeans_max_iter,
-                    seed=self.seed, estimator=self.estimator)
+                    seed=self.seed, estimator=self.estimator, G=self.G)
 
 
 TINY = Workload("tiny-f32-1x1024x64", H=1, N=1024, d=64, dtype="f32",
@@ -167,7 +173,25 @@ def _round_storage(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def make_head(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Q, K, V of head ``h`` as fp64 arrays holding exactly the stored (rounded) values."""
+    """Q of query head ``h`` and K, V of its K/V head (``h // G``) as fp64 arrays holding
+    exactly the stored (rounded) values."""
+    if w.G > 1:
+        qs, k, v = make_kv_group(w, h // w.G)
+        return qs[h % w.G], k, v
+    return _make_kv_head(w, h, 0)
+
+
+def make_kv_group(w: Workload, hk: int):
+    """GQA: the G query heads of K/V head ``hk`` (a list) and its K, V.  Query head 0 of
+    the group is drawn exactly as a head of the G = 1 recipe; query head j > 0 draws its
+    own noise (and nothing else) from the stream (hk, 2, j) and shares the group's
+    mixture centres, positional bias and logit scale."""
+    assert w.step == 0, "drifting sequences are drawn for G = 1 only"
+    q0, k, v, extra = _make_kv_head(w, hk, w.G - 1)
+    return [q0] + extra, k, v
+
+
+def _make_kv_head(w: Workload, h: int, n_extra: int):
     N, d = w.N, w.d
     assert N == w.grid[0] * w.grid[1] * w.grid[2]
     rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(w.seed, spawn_key=(h,))))
@@ -200,11 +224,27 @@ def make_head(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     scale = math.sqrt(w.logit_std / sigma_hat)
     Q *= scale
     K *= scale
-    return (_round_storage(Q, w.dtype), _round_storage(K, w.dtype), _round_storage(V, w.dtype))
+    out = (_round_storage(Q, w.dtype), _round_storage(K, w.dtype), _round_storage(V, w.dtype))
+    if n_extra == 0:
+        return out
+    extra = []
+    for j in range(1, n_extra + 1):
+        erng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(w.seed, spawn_key=(h, 2, j))))
+        Qj = base + w.sigma_q * erng.standard_normal((N, d))
+        if w.spatial_bias:
+            Qj += bias
+        extra.append(_round_storage(Qj * scale, w.dtype))
+    return out + (extra,)
 
 
 def make_inputs_np(w: Workload, heads: Optional[list] = None):
-    """Stacked fp64 [len(heads), N, d] arrays of the stored values (small workloads)."""
+    """Stacked fp64 [len(heads), N, d] arrays of the stored values (small workloads); with
+    G > 1 (all heads only) Q is [H, N, d] and K, V are [H/G, N, d]."""
+    if w.G > 1:
+        assert heads is None
+        groups = [make_kv_group(w, hk) for hk in range(w.H_kv)]
+        return (np.stack([q for g in groups for q in g[0]]), np.stack([g[1] for g in groups]),
+                np.stack([g[2] for g in groups]))
     heads = list(range(w.H)) if heads is None else list(heads)
     qs, ks, vs = zip(*(make_head(w, h) for h in heads))
     return np.stack(qs), np.stack(ks), np.stack(vs)
@@ -220,13 +260,22 @@ def make_inputs_torch(w: Workload, device="cpu", pin: bool = False):
     import torch
     td = torch_dtype(w.dtype)
     out = []
-    for _ in range(3):
-        t = torch.empty((w.H, w.N, w.d), dtype=td, pin_memory=pin and device == "cpu")
+    for i in range(3):
+        t = torch.empty((w.H if i == 0 else w.H_kv, w.N, w.d), dtype=td, pin_memory=pin and device == "cpu")
         out.append(t)
-    for h in range(w.H):
-        for t, a in zip(out, make_head(w, h)):
-            # the fp64 values are exactly representable in the storage dtype
-            t[h].copy_(torch.from_numpy(a.astype(np.float32)).to(td))
+    # the fp64 values are exactly representable in the storage dtype
+    conv = lambda a: torch.from_numpy(a.astype(np.float32)).to(td)
+    if w.G > 1:
+        for hk in range(w.H_kv):
+            qs, k, v = make_kv_group(w, hk)
+            for j, q in enumerate(qs):
+                out[0][hk * w.G + j].copy_(conv(q))
+            out[1][hk].copy_(conv(k))
+            out[2][hk].copy_(conv(v))
+    else:
+        for h in range(w.H):
+            for t, a in zip(out, make_head(w, h)):
+                t[h].copy_(conv(a))
     if device != "cpu":
         out = [t.to(device) for t in out]
     return tuple(out)

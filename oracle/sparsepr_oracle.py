@@ -41,6 +41,11 @@ Readings where the pages are silent (each is listed in the design doc):
       factor), twice, then scaled to unit mean eigenvalue: F F^T = M F (F^T M F)^-1 F^T M,
       which depends only on span(F); if F^T M F is not positive definite the call takes
       the full eigendecomposition instead
+  G1  GQA: the key metric of a K/V head is built from the concatenation (head-major) of
+      the query rows of its G query heads, sampled by S1 with G*M_s rows out of G*N_q;
+      the K/V partition, its centroids, the query metric and F_Q are shared by the G
+      heads; query coordinates, query k-means (init stream of the query head), routing,
+      probes and fit stay per query head
   W2  warm k-means starts label c at the previous call's original-space centroid of
       label c mapped into the current coordinates (phi_K linear, phi_Q with its RMS
       step); a label that was empty in the previous call has no centroid and takes the
@@ -560,17 +565,29 @@ def warm_centres(X: np.ndarray, fresh_idx: np.ndarray, used: np.ndarray,
     return np.where(used[:, None], mapped, X[fresh_idx])
 
 
-def partition(Q, K, V, p: Params, head: int, warm: Optional[WarmState] = None) -> Partition:
+def partition(Q, K, V, p: Params, head: int, warm: Optional[WarmState] = None,
+              Qgroup: Optional[List[np.ndarray]] = None, kv_head: Optional[int] = None) -> Partition:
+    """Response-Coupled Partitioning of query head `head`.
+
+    GQA ([P] App. C, reading G1): `Qgroup` holds the query rows of the G heads sharing
+    this K/V head (in head order) and `kv_head` its index; the key metric is built from
+    G*M_s evenly spaced rows of their concatenation and the key k-means draws its initial
+    rows from the K/V head's stream.  Without them (G = 1) both are this head's own.
+    """
     N_q, N_k = Q.shape[0], K.shape[0]
-    rows = sample_rows(N_q, p.M_s)
-    M_K = key_metric(Q, rows)
+    if Qgroup is None:
+        Qcat, M_s, kv_head = Q, p.M_s, head if kv_head is None else kv_head
+    else:
+        Qcat, M_s = np.concatenate(Qgroup, axis=0), p.M_s * len(Qgroup)
+    rows = sample_rows(Qcat.shape[0], M_s)
+    M_K = key_metric(Qcat, rows)
     F_K = subspace_factor(M_K, warm.F_K) if warm is not None else None
     if F_K is None:
         F_K, lam_K, _ = eigen_factor(M_K, p.r_K)
     else:
         lam_K = np.sort(np.linalg.eigvalsh(F_K.T @ F_K))[::-1]
     phiK = K @ F_K
-    idxK = kmeans_init_indices(p.seed, head, 0, p.C_k, N_k)
+    idxK = kmeans_init_indices(p.seed, kv_head, 0, p.C_k, N_k)
     c0K = None if warm is None else warm_centres(phiK, idxK, warm.k_used, warm.kbar @ F_K)
     km_K = kmeans(phiK, idxK, p.kmeans_max_iter, c0K)
     gk = compact_groups(km_K.labels, p.C_k)

@@ -652,3 +652,42 @@ def test_warm_kmeans_objective_is_monotone_and_empty_labels_redraw():
     assert np.array_equal(c0[3], part.phiK[idx[3]])
     c = int(np.flatnonzero(st.k_used)[0])
     assert np.allclose(c0[c], st.kbar[c] @ part.F_K, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- GQA ([P] App. C)
+def test_gqa_key_metric_is_the_mean_of_the_heads_metrics():
+    # G * M_s evenly spaced rows of the head-major concatenation take, when M_s divides
+    # N_q, exactly each head's own M_s sample rows, so the shared metric is the mean of
+    # the G per-head metrics
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY.with_(H=3, G=3)
+    p = O.Params.from_dict(w.params())
+    qs, K, V = W.make_kv_group(w, 0)
+    part = O.partition(qs[1], K, V, p, 1, Qgroup=qs, kv_head=0)
+    want = sum(O.key_metric(q, O.sample_rows(w.N, p.M_s)) for q in qs) / 3.0
+    assert np.abs(part.M_K - want).max() < 1e-13 * np.abs(want).max()
+
+
+def test_gqa_with_identical_query_heads_reproduces_the_single_head_partition():
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY
+    p = O.Params.from_dict(w.params())
+    Q, K, V = W.make_head(w, 0)
+    single = O.partition(Q, K, V, p, 0)
+    shared = O.partition(Q, K, V, p, 0, Qgroup=[Q, Q], kv_head=0)
+    assert np.abs(shared.M_K - single.M_K).max() < 1e-13 * np.abs(single.M_K).max()
+    assert np.array_equal(shared.km_K.labels, single.km_K.labels)
+    assert np.array_equal(shared.km_Q.labels, single.km_Q.labels)
+
+
+def test_gqa_query_heads_share_the_key_partition_and_keep_their_own_query_groups():
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY.with_(H=2, G=2)
+    p = O.Params.from_dict(w.params())
+    qs, K, V = W.make_kv_group(w, 0)
+    a = O.partition(qs[0], K, V, p, 0, Qgroup=qs, kv_head=0)
+    b = O.partition(qs[1], K, V, p, 1, Qgroup=qs, kv_head=0)
+    assert np.array_equal(a.km_K.labels, b.km_K.labels)
+    assert np.array_equal(a.F_Q, b.F_Q)                    # M_Q comes from the K/V groups
+    assert not np.array_equal(a.km_Q.labels, b.km_Q.labels)
+    assert not np.array_equal(qs[0], qs[1])
