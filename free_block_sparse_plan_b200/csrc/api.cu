@@ -55,8 +55,8 @@ sparsepr_status validate(const sparsepr_params* q) {
     return SPARSEPR_ERR_ARG;
   if (q->kmeans_max_iter < 1 || q->kmeans_max_iter > 1000) return SPARSEPR_ERR_ARG;
   if (q->engine != SPARSEPR_ENGINE_AUTO && q->engine != SPARSEPR_ENGINE_SIMT) return SPARSEPR_ERR_ARG;
-  if (q->estimator < SPARSEPR_EST_RIDGE || q->estimator > SPARSEPR_EST_DIAGONAL || q->reserved != 0)
-    return SPARSEPR_ERR_ARG;
+  if (q->estimator < SPARSEPR_EST_RIDGE || q->estimator > SPARSEPR_EST_DIAGONAL) return SPARSEPR_ERR_ARG;
+  if (q->G < 0 || (q->G > 1 && q->H % q->G != 0)) return SPARSEPR_ERR_SHAPE;
   return SPARSEPR_OK;
 }
 
@@ -67,6 +67,8 @@ Dims make_dims(const sparsepr_params* q) {
   d.M = q->M; d.r = q->r; d.lambda = q->lambda; d.rho = q->target_density;
   d.max_iter = q->kmeans_max_iter; d.engine = q->engine; d.seed = q->seed;
   d.estimator = q->estimator;
+  d.G = q->G > 1 ? q->G : 1;
+  d.Hk = d.H / d.G;
   d.nchK = cdiv(q->N_k, kSortChunk);
   d.nchQ = cdiv(q->N_q, kSortChunk);
   d.nsplit = cdiv(q->N_k, kProbeSplit);
@@ -211,7 +213,7 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_TRY(p.warm ? launch_warm_factor(p, false, st) : launch_eigen_factor(p, false, st));
   SPR_TRY(launch_project_keys(p, st));
   if (labK) {
-    SPR_CUDA_OK(cudaMemcpyAsync(p.b.labK, labK, sizeof(int) * m.H * m.Nk,
+    SPR_CUDA_OK(cudaMemcpyAsync(p.b.labK, labK, sizeof(int) * m.Hk * m.Nk,
                                 cudaMemcpyDeviceToDevice, st));
     SPR_TRY(launch_check_labels(p, false, st));
   } else {
@@ -248,30 +250,30 @@ struct ExportDesc {
 ExportDesc export_desc(const Plan& p, int what) {
   const Dims& m = p.dm;
   const Buffers& b = p.b;
-  const size_t H = m.H, d = m.d, I = sizeof(int), D = sizeof(double), F = sizeof(float);
+  const size_t H = m.H, Hk = m.Hk, d = m.d, I = sizeof(int), D = sizeof(double), F = sizeof(float);
   switch (what) {
-    case SPARSEPR_X_LABELS_K: return {b.labK, H * m.Nk * I};
+    case SPARSEPR_X_LABELS_K: return {b.labK, Hk * m.Nk * I};
     case SPARSEPR_X_LABELS_Q: return {b.labQ, H * m.Nq * I};
-    case SPARSEPR_X_PERM_K: return {b.permK, H * m.Nk * I};
+    case SPARSEPR_X_PERM_K: return {b.permK, Hk * m.Nk * I};
     case SPARSEPR_X_PERM_Q: return {b.permQ, H * m.Nq * I};
-    case SPARSEPR_X_GROUPS_K: return {b.nK, H * I};
+    case SPARSEPR_X_GROUPS_K: return {b.nK, Hk * I};
     case SPARSEPR_X_GROUPS_Q: return {b.nQ, H * I};
-    case SPARSEPR_X_SIZES_K: return {b.sizeK, H * m.Ck * I};
+    case SPARSEPR_X_SIZES_K: return {b.sizeK, Hk * m.Ck * I};
     case SPARSEPR_X_SIZES_Q: return {b.sizeQ, H * m.Cq * I};
     case SPARSEPR_X_CELL_COUNT: return {b.cellCnt, H * m.Cq * I};
     case SPARSEPR_X_CELL_IDS: return {b.cellIds, H * m.Cq * m.Ck * I};
     case SPARSEPR_X_PROBES: return {b.probes, H * m.M * I};
     case SPARSEPR_X_PROBE_COUNT: return {b.mA, H * m.Cq * I};
     case SPARSEPR_X_KMEANS_ITERS: return {nullptr, H * 2 * I};   // gathered specially
-    case SPARSEPR_X_OBJECTIVE: return {b.objH, H * 2 * D};
+    case SPARSEPR_X_OBJECTIVE: return {nullptr, H * 2 * D};      // gathered specially
     case SPARSEPR_X_PAIRS: return {b.pairs, H * sizeof(long long)};
-    case SPARSEPR_X_FACTOR_K: return {b.FK64, H * d * m.rK * D};
-    case SPARSEPR_X_FACTOR_Q: return {b.FQ64, H * d * m.rQ * D};
-    case SPARSEPR_X_EIG_K: return {b.lamK, H * m.rK * D};
-    case SPARSEPR_X_EIG_Q: return {b.lamQ, H * m.rQ * D};
-    case SPARSEPR_X_METRIC_K: return {b.MK, H * d * d * D};
-    case SPARSEPR_X_METRIC_Q: return {b.MQ, H * d * d * D};
-    case SPARSEPR_X_PHI_K: return {b.phiK, H * m.Nk * m.rK * D};
+    case SPARSEPR_X_FACTOR_K: return {b.FK64, Hk * d * m.rK * D};
+    case SPARSEPR_X_FACTOR_Q: return {b.FQ64, Hk * d * m.rQ * D};
+    case SPARSEPR_X_EIG_K: return {b.lamK, Hk * m.rK * D};
+    case SPARSEPR_X_EIG_Q: return {b.lamQ, Hk * m.rQ * D};
+    case SPARSEPR_X_METRIC_K: return {b.MK, Hk * d * d * D};
+    case SPARSEPR_X_METRIC_Q: return {b.MQ, Hk * d * d * D};
+    case SPARSEPR_X_PHI_K: return {b.phiK, Hk * m.Nk * m.rK * D};
     case SPARSEPR_X_PHI_Q: return {b.phiQ, H * m.Nq * m.rQ * D};
     case SPARSEPR_X_CENTRES_Q: return {b.centQ, H * m.Cq * m.rQ * D};
     case SPARSEPR_X_SCORES: return {b.scores, H * m.Cq * m.Ck * D};
@@ -284,7 +286,7 @@ ExportDesc export_desc(const Plan& p, int what) {
     case SPARSEPR_X_FIT_P: return {b.Pm, H * d * d * D};
     case SPARSEPR_X_FIT_REFF: return {b.reff, H * I};
     case SPARSEPR_X_PROBE_DIST: return {b.dist, H * m.Nq * D};
-    case SPARSEPR_X_KBAR: return {b.kbar, H * m.Ck * d * D};
+    case SPARSEPR_X_KBAR: return {b.kbar, Hk * m.Ck * d * D};
     case SPARSEPR_X_QBAR: return {b.qbar, H * m.Cq * d * D};
     case SPARSEPR_X_KM_REASSIGNED: return {b.kmReassigned, H * 2 * sizeof(long long)};
     default: return {nullptr, 0};
@@ -340,6 +342,7 @@ sparsepr_status sparsepr_plan_warm(const sparsepr_params* params, const void* Q,
                                    const void* V, const void* state, void* workspace,
                                    size_t workspace_bytes, void* stream, sparsepr_plan_t* out) {
   if (!state || (reinterpret_cast<uintptr_t>(state) & 255)) return SPARSEPR_ERR_ARG;
+  if (params && params->G > 1) return SPARSEPR_ERR_ARG;
   return plan_common(params, Q, K, V, nullptr, nullptr, state, workspace, workspace_bytes, stream, out);
 }
 
@@ -405,9 +408,12 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
   if (params->d < 8 || params->d > kMaxD || params->d % 8) return SPARSEPR_ERR_SHAPE;
   if (params->engine != SPARSEPR_ENGINE_AUTO && params->engine != SPARSEPR_ENGINE_SIMT)
     return SPARSEPR_ERR_ARG;
+  if (params->G < 0 || (params->G > 1 && params->H % params->G != 0)) return SPARSEPR_ERR_SHAPE;
   Dims m{};
   m.H = params->H; m.Nq = params->N_q; m.Nk = params->N_k; m.d = params->d;
   m.dtype = params->dtype; m.engine = params->engine;
+  m.G = params->G > 1 ? params->G : 1;
+  m.Hk = m.H / m.G;
   return launch_dense_attention(m, Q, K, V, Out, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -447,10 +453,12 @@ sparsepr_status sparsepr_get_stats(sparsepr_plan_t plan, void* stream, sparsepr_
   s.groups_q_min = 1 << 30;
   for (int h = 0; h < H; ++h) {
     s.pairs_route += pairs[h];
-    s.kmeans_iters_k_max = kmK[4 * h + 3] > s.kmeans_iters_k_max ? kmK[4 * h + 3] : s.kmeans_iters_k_max;
     s.kmeans_iters_q_max = kmQ[4 * h + 3] > s.kmeans_iters_q_max ? kmQ[4 * h + 3] : s.kmeans_iters_q_max;
-    s.groups_k_min = nK[h] < s.groups_k_min ? nK[h] : s.groups_k_min;
     s.groups_q_min = nQ[h] < s.groups_q_min ? nQ[h] : s.groups_q_min;
+  }
+  for (int hk = 0; hk < p.dm.Hk; ++hk) {          // K/V heads
+    s.kmeans_iters_k_max = kmK[4 * hk + 3] > s.kmeans_iters_k_max ? kmK[4 * hk + 3] : s.kmeans_iters_k_max;
+    s.groups_k_min = nK[hk] < s.groups_k_min ? nK[hk] : s.groups_k_min;
   }
   const double total = (double)H * p.dm.Nq * p.dm.Nk;
   s.pairs_exec = s.pairs_route + (long long)H * p.dm.M * p.dm.Nk;
@@ -476,8 +484,9 @@ sparsepr_status sparsepr_export(sparsepr_plan_t plan, int32_t what, void* dst, s
   ExportDesc x = export_desc(p, what);
   if (bytes != x.bytes) return SPARSEPR_ERR_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // row h: key side of its K/V head h / G, query side of h
   if (what == SPARSEPR_X_KMEANS_ITERS) {
-    const int H = p.dm.H;
+    const int H = p.dm.H, G = p.dm.G;
     int* km = new int[8 * H];
     cudaError_t e = cudaMemcpyAsync(km, p.b.kmK, 4 * H * sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(km + 4 * H, p.b.kmQ, 4 * H * sizeof(int), cudaMemcpyDeviceToHost, st);
@@ -485,11 +494,26 @@ sparsepr_status sparsepr_export(sparsepr_plan_t plan, int32_t what, void* dst, s
     if (e == cudaSuccess) {
       int* o = reinterpret_cast<int*>(dst);
       for (int h = 0; h < H; ++h) {
-        o[2 * h] = km[4 * h + 3];
+        o[2 * h] = km[4 * (h / G) + 3];
         o[2 * h + 1] = km[4 * H + 4 * h + 3];
       }
     }
     delete[] km;
+    return e == cudaSuccess ? SPARSEPR_OK : SPARSEPR_ERR_CUDA;
+  }
+  if (what == SPARSEPR_X_OBJECTIVE) {
+    const int H = p.dm.H, G = p.dm.G;
+    double* ob = new double[2 * H];
+    cudaError_t e = cudaMemcpyAsync(ob, p.b.objH, 2 * H * sizeof(double), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) {
+      double* o = reinterpret_cast<double*>(dst);
+      for (int h = 0; h < H; ++h) {
+        o[2 * h] = ob[2 * (h / G)];
+        o[2 * h + 1] = ob[2 * h + 1];
+      }
+    }
+    delete[] ob;
     return e == cudaSuccess ? SPARSEPR_OK : SPARSEPR_ERR_CUDA;
   }
   SPR_CUDA_OK(cudaMemcpyAsync(dst, x.ptr, x.bytes, cudaMemcpyDeviceToHost, st));

@@ -128,9 +128,9 @@ __global__ void __launch_bounds__(kThreads) sparse_simt_kernel(Dims m, Buffers b
     int sz = 0, start = 0;
     if (i < cnt) {
       const int kb = ids[i];
-      const int labk = b.usedK[(long long)h * m.Ck + kb];
-      start = b.offK[(long long)h * (m.Ck + 1) + labk];
-      sz = b.offK[(long long)h * (m.Ck + 1) + labk + 1] - start;
+      const int labk = b.usedK[(long long)(h / m.G) * m.Ck + kb];
+      start = b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk];
+      sz = b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk + 1] - start;
     }
     int tot;
     const int ex = block_exclusive_scan(sz, sh, &tot);
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) sparse_simt_kernel(Dims m, Buffers b
     __syncthreads();
   }
   const long long nkeys = cnt > 0 ? csum[cnt] : 0;
-  const long long kbase = (long long)h * m.Nk * d;
+  const long long kbase = (long long)(h / m.G) * m.Nk * d;   // K/V head h / G
   auto key_row = [&](long long v) -> long long {
     int lo = 0, hi = cnt - 1;      // last i with csum[i] <= v
     while (lo < hi) {
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(kThreads) probe_simt_kernel(Dims m, Buffers b,
   __syncthreads();
   const long long k0 = (long long)s * kProbeSplit;
   const long long k1 = (k0 + kProbeSplit < m.Nk) ? k0 + kProbeSplit : m.Nk;
-  const long long kbase = (long long)h * m.Nk * d;
+  const long long kbase = (long long)(h / m.G) * m.Nk * d;   // K/V head h / G
   auto key_row = [&](long long v) -> long long { return kbase + (k0 + v) * d; };
   float mrow, lrow, o[D / 4];
   attend_core<D>(m, Q, qrow, K, V, k1 - k0, key_row, ks, vs, krow, mrow, lrow, o);
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThreads) dense_simt_kernel(Dims m, const void
     qrow[threadIdx.x] = row < m.Nq ? ((long long)h * m.Nq + row) * d : -1;
   }
   __syncthreads();
-  const long long kbase = (long long)h * m.Nk * d;
+  const long long kbase = (long long)(h / m.G) * m.Nk * d;   // K/V head h / G
   auto key_row = [&](long long v) -> long long { return kbase + v * d; };
   float mrow, lrow, o[D / 4];
   attend_core<D>(m, Q, qrow, K, V, m.Nk, key_row, ks, vs, krow, mrow, lrow, o);

@@ -141,9 +141,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       const int i = base_i + tid;
       int sz = 0, start = 0;
       if (i < cnt) {
-        const int labk = g.b.usedK[(long long)h * m.Ck + ids[i]];
-        start = g.b.offK[(long long)h * (m.Ck + 1) + labk];
-        sz = g.b.offK[(long long)h * (m.Ck + 1) + labk + 1] - start;
+        const int labk = g.b.usedK[(long long)(h / m.G) * m.Ck + ids[i]];
+        start = g.b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk];
+        sz = g.b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk + 1] - start;
       }
       int tot;
       const int ex = block_exclusive_scan(sz, ms->sh, &tot);
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   if (warp >= 8 && warp < 11) {
     // ============================================================ producers
     const int p = tid - 256;
-    const long long hq = (long long)h * m.Nq * d, hk = (long long)h * m.Nk * d;
+    const long long hq = (long long)h * m.Nq * d, hk = (long long)(h / m.G) * m.Nk * d;   // K/V head h / G
     for (int row = p; row < kItemRows; row += kProducers) {
       long long qr = -1;
       if (row < nrows) {

@@ -32,6 +32,7 @@ struct KmView {         // one k-means instance (keys or queries) for all heads
   double* delta;        // [H][C] centre movement of each update, or null
   unsigned long long* dmax;   // [2][H][G] largest movement per 32-centre group (double bits)
   int N, C, r, nch, stage;
+  int H;                // instances: query heads, or K/V heads for the key side
 };
 
 KmView view(const Plan& p, bool query) {
@@ -39,9 +40,9 @@ KmView view(const Plan& p, bool query) {
   const Dims& m = p.dm;
   if (query)
     return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, b.kmDelta, b.kmDmax,
-            m.Nq, m.Cq, m.rQ, m.nchQ, 1};
+            m.Nq, m.Cq, m.rQ, m.nchQ, 1, m.H};
   return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, b.kmDelta, b.kmDmax,
-          m.Nk, m.Ck, m.rK, m.nchK, 0};
+          m.Nk, m.Ck, m.rK, m.nchK, 0, m.Hk};
 }
 
 // ---------------------------------------------------------------------------------
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int
   const int d = m.d, h = blockIdx.y;
   double* F = smd;                         // [d][R], zero columns k >= r
   float* Xt = reinterpret_cast<float*>(smd + d * R);  // [d][kProjXs]: Xt[j][row]
-  const double* Fh = Fall + (long long)h * d * r;
+  const double* Fh = Fall + (long long)(RMS ? h / m.G : h) * d * r;   // queries: their K/V head's F_Q
   for (int e = threadIdx.x; e < d * R; e += blockDim.x) {
     const int j = e / R, k = e % R;
     F[e] = k < r ? Fh[j * r + k] : 0.0;
@@ -177,7 +178,7 @@ sparsepr_status launch_project(const Plan& p, const void* X, int N, const double
                                __nv_bfloat16* xhi, __nv_bfloat16* xlo, float* xn, int Npad, cudaStream_t st) {
   const int d = p.dm.d;
   const int rows = xhi ? Npad : N;
-  dim3 grid(cdiv(rows, kProjRows * kProjTiles), p.dm.H);
+  dim3 grid(cdiv(rows, kProjRows * kProjTiles), RMS ? p.dm.H : p.dm.Hk);
   auto run = [&](auto kern, int R) -> sparsepr_status {
     const size_t smem = (size_t)d * R * sizeof(double) + (size_t)d * kProjXs * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(256) km_warm_init_kernel(KmView v, unsigned lo
   double* out = v.cent + ((long long)h * v.C + c) * r;
   if (state_matches(hdr, m) && used[(long long)h * v.C + c]) {
     const double* cb = cprev + ((long long)h * v.C + c) * d;
-    const double* Fh = F + (long long)h * d * r;
+    const double* Fh = F + (long long)(v.stage == 1 ? h / m.G : h) * d * r;
     double z0 = 0.0, z1 = 0.0;
     for (int j = 0; j < d; ++j) {
       const double x = cb[j];
@@ -489,7 +490,7 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
 }
 
 sparsepr_status run_update(const Plan& p, const KmView& v, int it, bool force, cudaStream_t st) {
-  const int H = p.dm.H;
+  const int H = v.H;
   cs_hist_kernel<<<dim3(v.nch, H), kSortChunk, 0, st>>>(v, it, force);
   SPR_LAUNCH_OK();
   cs_scan_kernel<<<H, 1024, 0, st>>>(v, it, force);
@@ -638,7 +639,7 @@ __global__ void check_labels_kernel(int* lab, long long n, int C, int* err) {
 
 sparsepr_status launch_check_labels(const Plan& p, bool query, cudaStream_t st) {
   const KmView v = view(p, query);
-  check_labels_kernel<<<148 * 4, 256, 0, st>>>(v.lab, (long long)p.dm.H * v.N, v.C, p.b.err);
+  check_labels_kernel<<<148 * 4, 256, 0, st>>>(v.lab, (long long)v.H * v.N, v.C, p.b.err);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -646,7 +647,7 @@ sparsepr_status launch_check_labels(const Plan& p, bool query, cudaStream_t st) 
 // The tensor-core k-means serves a side when the engine allows it and C fits its tiles.
 bool km_uses_tc(const Plan& p, bool query) {
   const KmView v = view(p, query);
-  return p.dm.engine == SPARSEPR_ENGINE_AUTO && km_tc_supported(v.C) && (long long)p.dm.H * v.N < (1LL << 31);
+  return p.dm.engine == SPARSEPR_ENGINE_AUTO && km_tc_supported(v.C) && (long long)v.H * v.N < (1LL << 31);
 }
 
 // fp64 coordinates for either engine; the split coordinates of the tensor-core k-means
@@ -673,7 +674,7 @@ sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st) { return 
 
 sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   const KmView v = view(p, query);
-  const int H = p.dm.H;
+  const int H = v.H;
   SPR_CUDA_OK(cudaMemsetAsync(v.km, 0, sizeof(int) * 4 * H, st));
   SPR_CUDA_OK(cudaMemsetAsync(v.lab, 0xFF, sizeof(int) * (size_t)H * v.N, st));  // labels = -1
   if (p.warm) {
@@ -724,8 +725,8 @@ sparsepr_status launch_finalize_groups(const Plan& p, bool query, cudaStream_t s
   sparsepr_status s = run_update(p, v, 0, true, st);
   if (s != SPARSEPR_OK) return s;
   const Buffers& b = p.b;
-  if (query) groups_kernel<<<p.dm.H, 1024, 0, st>>>(v, b.compQ, b.usedQ, b.sizeQ, b.nQ, b.objH);
-  else groups_kernel<<<p.dm.H, 1024, 0, st>>>(v, b.compK, b.usedK, b.sizeK, b.nK, b.objH);
+  if (query) groups_kernel<<<v.H, 1024, 0, st>>>(v, b.compQ, b.usedQ, b.sizeQ, b.nQ, b.objH);
+  else groups_kernel<<<v.H, 1024, 0, st>>>(v, b.compK, b.usedK, b.sizeK, b.nK, b.objH);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -736,7 +737,7 @@ sparsepr_status launch_centroids(const Plan& p, bool query, cudaStream_t st) {
   if (query)
     centroid_kernel<<<dim3(m.Cq, m.H), kCentSub * kMaxD, 0, st>>>(m, p.Q, nullptr, m.Nq, m.Cq, b.permQ, b.offQ, b.usedQ, b.nQ, b.qbar, nullptr);
   else
-    centroid_kernel<<<dim3(m.Ck, m.H), kCentSub * kMaxD, 0, st>>>(m, p.K, p.V, m.Nk, m.Ck, b.permK, b.offK, b.usedK, b.nK, b.kbar, b.vbar);
+    centroid_kernel<<<dim3(m.Ck, m.Hk), kCentSub * kMaxD, 0, st>>>(m, p.K, p.V, m.Nk, m.Ck, b.permK, b.offK, b.usedK, b.nK, b.kbar, b.vbar);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -748,7 +749,7 @@ sparsepr_status launch_save_state(const Plan& p, void* state, cudaStream_t st) {
 }
 
 sparsepr_status launch_query_metric(const Plan& p, cudaStream_t st) {
-  query_metric_kernel<<<p.dm.H, 1024, 0, st>>>(p.dm, p.b.kbar, p.b.nK, p.b.MQ);
+  query_metric_kernel<<<p.dm.Hk, 1024, 0, st>>>(p.dm, p.b.kbar, p.b.nK, p.b.MQ);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

@@ -36,6 +36,7 @@ struct Dims {
   int max_iter, engine;
   unsigned long long seed;
   int estimator;       // sparsepr_estimator
+  int G, Hk;           // query heads per K/V head; K/V heads (H / G)
   int nchK, nchQ;      // counting-sort chunks per head
   int nsplit;          // partial blocks of the exact probe attention
   double beta;         // per-query key budget (rho - M/N_q) * N_k

@@ -21,11 +21,14 @@ constexpr int kLinThreads = 1024;
 
 // ---------------------------------------------------------------------------------
 // M_K = (1/M_s') sum_s q_s^T q_s over rows floor(s*N_q/M_s) (all rows if M_s >= N_q).
+// One block per K/V head.  With G query heads per K/V head (GQA, paper App. C) the rows
+// are those of the G heads concatenated in head order, G*M_s of them: sample s is row
+// c = floor(s*N_q/M_s) of the concatenation (the same index as floor(s*G*N_q/(G*M_s))),
+// i.e. row c mod N_q of query head G*hk + c / N_q.
 __global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const void* Q, double* MK) {
   extern __shared__ float rows[];   // [64][d]
   const int h = blockIdx.x, d = m.d;
-  const int Ms = m.Ms < m.Nq ? m.Ms : m.Nq;
-  const long long qbase = (long long)h * m.Nq * d;
+  const int Ms = m.G * (m.Ms < m.Nq ? m.Ms : m.Nq);
   double acc[16];
   for (int k = 0; k < 16; ++k) acc[k] = 0.0;
   const int entries = d * d;
@@ -34,8 +37,9 @@ __global__ void __launch_bounds__(kLinThreads) key_metric_kernel(Dims m, const v
     __syncthreads();
     for (int e = threadIdx.x; e < ns * d; e += blockDim.x) {
       const int s = s0 + e / d, j = e % d;
-      const long long row = (m.Ms >= m.Nq) ? s : ((long long)s * m.Nq) / m.Ms;
-      rows[e] = load_as_float(Q, qbase + row * d + j, m.dtype);
+      const long long c = (m.Ms >= m.Nq) ? s : ((long long)s * m.Nq) / m.Ms;
+      const long long qh = (long long)h * m.G + c / m.Nq;
+      rows[e] = load_as_float(Q, (qh * m.Nq + c % m.Nq) * d + j, m.dtype);
     }
     __syncthreads();
     for (int k = 0; k < 16; ++k) {
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(kLinThreads) fit_smem_kernel(Dims m, Buffers b
 
 sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st) {
   const size_t smem = 64 * p.dm.d * sizeof(float);
-  key_metric_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.Q, p.b.MK);
+  key_metric_kernel<<<p.dm.Hk, kLinThreads, smem, st>>>(p.dm, p.Q, p.b.MK);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -661,10 +665,11 @@ sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st) 
   const size_t smem = (size_t)p.dm.d * p.dm.d * sizeof(double);
   SPR_CUDA_OK(cudaFuncSetAttribute(eigen_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int* only = p.warm ? p.b.warmCold + (query ? p.dm.H : 0) : nullptr;
+  // both metrics belong to the K/V head (M_Q is built from its groups' centroids)
   if (query)
-    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MQ, p.dm.rQ, p.b.lamQ, p.b.FQ64, p.b.FQ, p.b.err, kErrEigQ, only);
+    eigen_factor_kernel<<<p.dm.Hk, kLinThreads, smem, st>>>(p.dm, p.b.MQ, p.dm.rQ, p.b.lamQ, p.b.FQ64, p.b.FQ, p.b.err, kErrEigQ, only);
   else
-    eigen_factor_kernel<<<p.dm.H, kLinThreads, smem, st>>>(p.dm, p.b.MK, p.dm.rK, p.b.lamK, p.b.FK64, p.b.FK, p.b.err, kErrEigK, only);
+    eigen_factor_kernel<<<p.dm.Hk, kLinThreads, smem, st>>>(p.dm, p.b.MK, p.dm.rK, p.b.lamK, p.b.FK64, p.b.FK, p.b.err, kErrEigK, only);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }
@@ -680,7 +685,7 @@ sparsepr_status launch_warm_factor(const Plan& p, bool query, cudaStream_t st) {
   SPR_CUDA_OK(cudaFuncSetAttribute(subspace_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int* cold = p.b.warmCold + (query ? m.H : 0);
   SPR_CUDA_OK(cudaMemsetAsync(cold, 0, sizeof(int) * m.H, st));
-  subspace_factor_kernel<<<m.H, kLinThreads, smem, st>>>(
+  subspace_factor_kernel<<<m.Hk, kLinThreads, smem, st>>>(
       m, query ? p.b.MQ : p.b.MK, reinterpret_cast<const int*>(base),
       reinterpret_cast<const double*>(base + (query ? L.FQ : L.FK)), r,
       query ? p.b.lamQ : p.b.lamK, query ? p.b.FQ64 : p.b.FK64, query ? p.b.FQ : p.b.FK, cold, p.b.err);

@@ -96,6 +96,7 @@ extern "C" sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* pa
   if (params->d < 8 || params->d > kMaxD || params->d % 8) return SPARSEPR_ERR_SHAPE;
   if (params->engine != SPARSEPR_ENGINE_AUTO && params->engine != SPARSEPR_ENGINE_SIMT) return SPARSEPR_ERR_ARG;
   if (nrows < 1 || nrows > kMaxM) return SPARSEPR_ERR_ARG;
+  if (params->G < 0 || (params->G > 1 && params->H % params->G != 0)) return SPARSEPR_ERR_SHAPE;
   if (noalloc_rows_scratch_bytes(params->H, nrows, params->N_k, params->d) > kNoAllocScratchBytes)
     return SPARSEPR_ERR_WORKSPACE;
   void* base = nullptr;
@@ -106,6 +107,8 @@ extern "C" sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* pa
   Plan p{};
   p.dm.H = params->H; p.dm.Nq = params->N_q; p.dm.Nk = params->N_k; p.dm.d = params->d;
   p.dm.dtype = params->dtype; p.dm.engine = params->engine; p.dm.M = nrows;
+  p.dm.G = params->G > 1 ? params->G : 1;
+  p.dm.Hk = p.dm.H / p.dm.G;
   p.dm.nsplit = cdiv(params->N_k, kProbeSplit);
   p.Q = Q; p.K = K; p.V = V;
   char* c = reinterpret_cast<char*>(base);

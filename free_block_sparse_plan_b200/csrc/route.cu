@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
   const int nq = b.nQ[h];
   if (a0 >= nq) return;
   const int na = min(kScoreQ, nq - a0);
-  const int n = b.nK[h];
+  const int hk = h / m.G;                 // the K/V head of this query head
+  const int n = b.nK[hk];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   double* out0 = b.scores + ((long long)h * m.Cq + a0) * m.Ck;
   if (n == 1) {
@@ -46,9 +47,9 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
   double* zz = kv + kScoreK * ld;         // [kScoreQ][n] logits, then exp(l - max)
   double* zr = zz + kScoreQ * n;          // [kScoreQ][n] exp(l - second max), 0 at the top
   const double tau = 1.0 / sqrt((double)d);
-  const double* kb = b.kbar + (long long)h * m.Ck * d;
-  const double* vb = b.vbar + (long long)h * m.Ck * d;
-  const int* sz = b.sizeK + (long long)h * m.Ck;
+  const double* kb = b.kbar + (long long)hk * m.Ck * d;
+  const double* vb = b.vbar + (long long)hk * m.Ck * d;
+  const int* sz = b.sizeK + (long long)hk * m.Ck;
   for (int e = tid; e < kScoreQ * d; e += blockDim.x) {
     const int a = e / d, j = e % d;
     qa[a * ld + j] = a < na ? b.qbar[((long long)h * m.Cq + a0 + a) * d + j] : 0.0;
@@ -171,7 +172,8 @@ __global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
     if (threadIdx.x == 0) b.cellCnt[(long long)h * m.Cq + a] = 0;
     return;
   }
-  const int n = b.nK[h];
+  const int hk = h / m.G;        // the K/V head of this query head
+  const int n = b.nK[hk];
   int P2 = 1;
   while (P2 < n) P2 <<= 1;
   const double* S = b.scores + ((long long)h * m.Cq + a) * m.Ck;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
       __syncthreads();
     }
   }
-  const int* sz = b.sizeK + (long long)h * m.Ck;
+  const int* sz = b.sizeK + (long long)hk * m.Ck;
   const int t = threadIdx.x;
   const int mine = t < n ? sz[id[t]] : 0;
   int tot;
@@ -384,9 +386,9 @@ sparsepr_status launch_permute(const Plan& p, cudaStream_t st) {
   const int blocks = 148 * 8;
   gather_kernel<<<blocks, 256, 0, st>>>(p.Q, p.b.Qp, p.b.permQ, p.b.invQ, m.H, m.Nq, chunks);
   SPR_LAUNCH_OK();
-  gather_kernel<<<blocks, 256, 0, st>>>(p.K, p.b.Kp, p.b.permK, nullptr, m.H, m.Nk, chunks);
+  gather_kernel<<<blocks, 256, 0, st>>>(p.K, p.b.Kp, p.b.permK, nullptr, m.Hk, m.Nk, chunks);
   SPR_LAUNCH_OK();
-  gather_kernel<<<blocks, 256, 0, st>>>(p.V, p.b.Vp, p.b.permK, nullptr, m.H, m.Nk, chunks);
+  gather_kernel<<<blocks, 256, 0, st>>>(p.V, p.b.Vp, p.b.permK, nullptr, m.Hk, m.Nk, chunks);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

@@ -84,7 +84,8 @@ typedef enum {
 /*
  * Problem and hyper-parameters of one call (paper S2, S4; values of the review page's
  * hyper-parameter table: r_K=48, r_Q=64, M=64, r=16, lambda=0.1).
- *   H                 heads (each head is an independent problem)
+ *   H                 query heads (each head is an independent problem, but for the K/V
+ *                     partition it shares with the other heads of its group when G > 1)
  *   N_q, N_k          query and key/value tokens per head
  *   d                 head dimension (multiple of 8, <= 128)
  *   dtype             sparsepr_dtype of Q, K, V and Out
@@ -99,6 +100,17 @@ typedef enum {
  *   engine            sparsepr_engine
  *   seed              seed of the SplitMix64 stream that draws the k-means initial rows
  *   estimator         sparsepr_estimator (0, the method's weighted ridge, unless comparing)
+ *   G                 query heads per K/V head (grouped-query attention; 0 or 1 = none).
+ *                     H must be a multiple of G; K and V are then [H/G, N_k, d], query head
+ *                     h reads K/V head h/G.  Paper App. C: the shared key response metric
+ *                     of a K/V head is built from its G query heads' rows, concatenated in
+ *                     head order, of which G*M_s evenly spaced rows are taken; the K/V
+ *                     groups, their centroids, the query metric and F_Q are shared by the
+ *                     G heads, and everything from the query coordinates on is per query
+ *                     head.  Exports of the K/V side (LABELS_K, PERM_K, GROUPS_K, SIZES_K,
+ *                     FACTOR_K, EIG_K, METRIC_K, PHI_K, KBAR, METRIC_Q, FACTOR_Q, EIG_Q)
+ *                     then have H/G rows; KMEANS_ITERS and OBJECTIVE keep H rows, the key
+ *                     column of row h being that of K/V head h/G.  Warm starts take G <= 1.
  */
 typedef struct {
   int32_t H, N_q, N_k, d;
@@ -110,7 +122,7 @@ typedef struct {
   int32_t engine;
   uint64_t seed;
   int32_t estimator;
-  int32_t reserved;          /* must be 0 */
+  int32_t G;
 } sparsepr_params;
 
 typedef struct sparsepr_plan_s* sparsepr_plan_t;
@@ -142,7 +154,7 @@ sparsepr_status sparsepr_plan(const sparsepr_params* params, const void* Q, cons
                               void* stream, sparsepr_plan_t* out);
 
 /*
- * As sparsepr_plan, but the k-means labels are given: labQ [H,N_q] and labK [H,N_k] are
+ * As sparsepr_plan, but the k-means labels are given: labQ [H,N_q] and labK [H/G,N_k] are
  * device int32 arrays with values in [0,C_q) and [0,C_k).  Every later step (groups,
  * centroids, query coordinates, routing, permutation, probes) is computed from them
  * exactly as sparsepr_plan computes it from its own k-means labels.  For testing the

@@ -267,6 +267,60 @@ def test_warm_state_that_was_never_saved_starts_cold_and_is_flagged():
     assert torch.equal(out, out_c)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_gqa_shared_key_partition_matches_oracle(name):
+    # App. C GQA: G query heads share each K/V head; the key metric comes from their
+    # concatenated rows, the K/V groups and F_Q are shared, the rest is per query head
+    w = (W.TINY.with_(H=2, G=2) if name == "tiny" else W.MID.with_(H=4, G=2))
+    P = O.Params.from_dict(w.params())
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    assert K.shape[0] == w.H_kv
+    rows = None if w.N <= 4096 else (np.arange(2048) * w.N) // 2048
+    groups = [W.make_kv_group(w, hk) for hk in range(w.H_kv)]
+    parts = [O.partition(groups[h // w.G][0][h % w.G], groups[h // w.G][1], groups[h // w.G][2], P, h,
+                         Qgroup=groups[h // w.G][0], kv_head=h // w.G) for h in range(w.H)]
+    # free running: labels, objectives, iterations
+    plan, out, _ = gpu_call(w, inputs=(Q, K, V))
+    assert plan.check() == 0
+    labK, labQ = plan.export("LABELS_K"), plan.export("LABELS_Q")
+    MK = plan.export("METRIC_K")
+    obj, iters = plan.export("OBJECTIVE"), plan.export("KMEANS_ITERS")
+    for h, part in enumerate(parts):
+        hk = h // w.G
+        assert rel(MK[hk], part.M_K) < 1e-12
+        assert np.mean(labK[hk] == part.km_K.labels) >= 0.999
+        assert np.mean(labQ[h] == part.km_Q.labels) >= 0.999
+        assert abs(obj[h][0] - part.km_K.objective) <= 1e-4 * part.km_K.objective
+        assert abs(obj[h][1] - part.km_Q.objective) <= 1e-4 * part.km_Q.objective
+        if np.array_equal(labK[hk], part.km_K.labels) and np.array_equal(labQ[h], part.km_Q.labels):
+            assert tuple(iters[h]) == (part.km_K.iterations, part.km_Q.iterations)
+    # oracle labels injected: bit-exact indexing and the output
+    labQi = torch.tensor(np.stack([p_.km_Q.labels for p_ in parts]), dtype=torch.int32, device="cuda")
+    labKi = torch.tensor(np.stack([parts[hk * w.G].km_K.labels for hk in range(w.H_kv)]),
+                         dtype=torch.int32, device="cuda")
+    plan, out, _ = gpu_call(w, inputs=(Q, K, V), labels=(labQi, labKi))
+    assert plan.check() == 0
+    for h, part in enumerate(parts):
+        g = groups[h // w.G]
+        res = O.sparsepr_call(g[0][h % w.G], g[1], g[2], P, head=h, rows=rows, part=part)
+        check_injected_head_gqa(plan, out[h].double().cpu().numpy(), res, h, w)
+
+
+def check_injected_head_gqa(plan, out_h, res, h, w):
+    """check_injected_head with the K/V-side exports read at the K/V head h / G."""
+    hk = h // w.G
+    gq, gk = res.part.gq, res.part.gk
+    assert np.array_equal(plan.export("PERM_Q")[h], res.permQ)
+    assert np.array_equal(plan.export("PERM_K")[hk], res.permK)
+    assert plan.export("GROUPS_Q")[h] == gq.sizes.size and plan.export("GROUPS_K")[hk] == gk.sizes.size
+    cc, ci = plan.export("CELL_COUNT")[h], plan.export("CELL_IDS")[h]
+    for a, sel in enumerate(res.sel):
+        assert cc[a] == sel.size and np.array_equal(ci[a][:sel.size], sel), a
+    assert int(plan.export("PAIRS")[h]) == res.pairs_route
+    assert tie_ambiguous_probes(res, plan.export("PROBES")[h])
+    assert rel(out_h[res.rows], res.out) < TOL[w.dtype]
+
+
 def test_tiny_simt_engine_equals_auto():
     w = W.TINY
     _, out_a, inputs = gpu_call(w)

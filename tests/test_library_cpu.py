@@ -68,6 +68,7 @@ def test_workspace_size_positive_and_monotone():
     ("lam", -0.5, N.SPARSEPR_ERR_ARG), ("lam", float("nan"), N.SPARSEPR_ERR_ARG),
     ("target_density", 1.5, N.SPARSEPR_ERR_ARG), ("target_density", 0.01, N.SPARSEPR_ERR_ARG),
     ("kmeans_max_iter", 0, N.SPARSEPR_ERR_ARG), ("engine", 3, N.SPARSEPR_ERR_ARG),
+    ("G", -1, N.SPARSEPR_ERR_SHAPE), ("G", 5, N.SPARSEPR_ERR_SHAPE),
 ])
 def test_invalid_parameters_rejected_on_host(field, value, status):
     p = _params()
@@ -98,3 +99,16 @@ def test_calls_out_of_order_or_null_are_rejected():
     assert L.sparsepr_probe_fit(None, None) == N.SPARSEPR_ERR_ARG
     assert L.sparsepr_correct(None, 256, None) == N.SPARSEPR_ERR_ARG
     L.sparsepr_destroy(None)
+
+
+def test_gqa_group_sizes_and_warm_start_restriction():
+    # H = 4 query heads: groups of 1, 2 and 4 are valid; a warm start takes G <= 1
+    for g in (0, 1, 2, 4):
+        p = _params()
+        p.H, p.G = 4, g
+        assert N.sparsepr_workspace_size(p) > 0
+    p = _params()
+    p.H, p.G = 4, 2
+    h = ctypes.c_void_p()
+    st = N.lib().sparsepr_plan_warm(ctypes.byref(p), 256, 256, 256, 256, 256, 1 << 40, None, ctypes.byref(h))
+    assert st == N.SPARSEPR_ERR_ARG and not h.value
