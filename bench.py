@@ -147,6 +147,13 @@ def cpu_oracle_sample(w, head=0):
             "seconds_per_head": dt}
 
 
+def workload_config(w):
+    """The `config` object both arms report for workload w."""
+    return {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "C_q": w.C_q, "C_k": w.C_k,
+            "M": w.M, "r": w.r, "target_density": w.rho, "heads_per_gpu": w.H,
+            "l2": "flushed between timed calls (256 MiB write)"}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -174,7 +181,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * sum(times) / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "sample": "one head per step"},
+        "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"one head of {w.H} per step (heads 0..), full fp64 call"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -377,9 +384,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "C_q": w.C_q, "C_k": w.C_k,
-                   "M": w.M, "r": w.r, "target_density": w.rho, "heads_per_gpu": w.H,
-                   "l2": "flushed between timed calls (256 MiB write)"},
+        "config": workload_config(w),
         "ms_per_call": ms,
         "stages_ms": {"plan": float(np.median(stage[:, 0])), "attend": attend_ms,
                       "probe_fit": float(np.median(stage[:, 2])),
