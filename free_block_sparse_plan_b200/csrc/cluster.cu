@@ -688,7 +688,7 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
     km_init_kernel<<<H, 256, 0, st>>>(v, p.dm.seed);
   }
   SPR_LAUNCH_OK();
-  // tensor-core scores with exact rescoring (labels identical to the fp32 full scan) when
+  // tensor-core scores with exact rescoring (labels identical to the fp64 full scan) when
   // there are enough centres to fill the tiles; the full scan otherwise or on request
   const bool tc = km_uses_tc(p, query);
   const Buffers& b = p.b;

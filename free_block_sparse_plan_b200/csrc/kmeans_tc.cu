@@ -1,4 +1,4 @@
-// k-means assignment on the tensor cores, with labels identical to the fp32 full scan.
+// k-means assignment on the tensor cores, with labels identical to the fp64 full scan.
 //
 // Scores a_c = ||c||^2 - 2 x.c (argmin a_c = argmin ||x - c||^2) come from three bf16
 // products per k-step, x_hi c_hi + x_hi c_lo + x_lo c_hi, with x = x_hi + x_lo + e,
@@ -26,13 +26,17 @@
 // three 256-centre chunks) stay in shared memory; point tiles stream through a ring of
 // X slots.  Both arrive by TMA (2-D tiled copies, 128-byte swizzle).
 //   warps 0-3 / 4-7  epilogue of the tiles of even / odd local index (thread = TMEM lane):
-//                    scores from TMEM, running four smallest, decision or queue entry;
+//                    scores from TMEM, running best, its centre and the runner-up,
+//                    decision or queue entry;
 //   warp 8           TMA producer (one thread);
 //   warp 9           MMA issuer (one thread) and TMEM owner: M=128, N=chunk width, K=16,
 //                    both operands K-major, into two 256-column accumulators that
 //                    alternate job by job (job = one tile against one centre chunk).
 // Every accumulator has one "full" mbarrier per epilogue group, so each waiter sees the
 // phases of its barrier one by one (a parity wait cannot tell phase k from k - 2).
+// Warm plans also keep distance bounds (km_filter_kernel below): the kernel then runs over
+// the compacted rows of the points whose label can still change (template flag B);
+// cold plans assign every point of the heads that have not converged.
 #include <cudaTypedefs.h>
 
 #include <cmath>
