@@ -46,6 +46,10 @@ Readings where the pages are silent (each is listed in the design doc):
       the K/V partition, its centroids, the query metric and F_Q are shared by the G
       heads; query coordinates, query k-means (init stream of the query head), routing,
       probes and fit stay per query head
+  S25 the semantic (reference) partition runs the same k-means on the raw key and query
+      rows; probe distances are then taken on raw query rows
+  S26 O1 support densities are fractions of the keys: tau_i = |D_i(alpha)| / N_k and the
+      pooled gamma = |union of the D_i| / N_k
   W2  warm k-means starts label c at the previous call's original-space centroid of
       label c mapped into the current coordinates (phi_K linear, phi_Q with its RMS
       step); a label that was empty in the previous call has no centroid and takes the
@@ -502,13 +506,15 @@ class Params:
     kmeans_max_iter: int = 25
     seed: int = 0
     estimator: str = "ridge"
+    partition: str = "response"     # "response" (RCP) or "semantic" (the reference partition)
 
     @classmethod
     def from_dict(cls, p: Dict) -> "Params":
         return cls(d=p["d"], M_s=p["M_s"], r_K=p["r_K"], r_Q=p["r_Q"], C_q=p["C_q"],
                    C_k=p["C_k"], M=p["M"], r=p["r"], lam=p["lam"],
                    rho=p["target_density"], kmeans_max_iter=p["kmeans_max_iter"],
-                   seed=p["seed"], estimator=ESTIMATORS[int(p.get("estimator", 0))])
+                   seed=p["seed"], estimator=ESTIMATORS[int(p.get("estimator", 0))],
+                   partition=p.get("partition", "response"))
 
 
 @dataclass
@@ -610,6 +616,74 @@ def partition(Q, K, V, p: Params, head: int, warm: Optional[WarmState] = None,
                      lam_Q, phiQ, km_Q, gq, qbar)
 
 
+def partition_semantic(Q, K, V, p: Params, head: int) -> Partition:
+    """The reference (semantic) partition of [P] S3 and of its ablations: k-means applied
+    separately to the raw key rows and to the raw query rows, each value following its
+    key.  Reading S25: the same Lloyd steps, init streams and stop rule as the response
+    coordinates' k-means, on the stored rows themselves (no metric, no RMS step); the
+    coordinate maps are the identity, so probe distances (S16) are taken on raw query rows.
+    """
+    N_q, N_k, d = Q.shape[0], K.shape[0], Q.shape[1]
+    km_K = kmeans(K, kmeans_init_indices(p.seed, head, 0, p.C_k, N_k), p.kmeans_max_iter)
+    gk = compact_groups(km_K.labels, p.C_k)
+    kbar = group_means(K, gk)
+    vbar = group_means(V, gk)
+    km_Q = kmeans(Q, kmeans_init_indices(p.seed, head, 1, p.C_q, N_q), p.kmeans_max_iter)
+    gq = compact_groups(km_Q.labels, p.C_q)
+    qbar = group_means(Q, gq)
+    eye = np.eye(d)
+    none = np.zeros((0,))
+    return Partition(none, none, eye, np.ones(d), K, km_K, gk, kbar, vbar,
+                     centred_key_centroids(kbar), none, eye, np.ones(d), Q, km_Q, gq, qbar)
+
+
+def support_size(a: np.ndarray, alpha: float) -> np.ndarray:
+    """|D_i(alpha)|: the fewest highest-weight keys whose dense attention mass reaches
+    alpha, per row of the attention matrix `a` ([P] S3, O1).  Ties in weight do not change
+    the count."""
+    srt = -np.sort(-a, axis=1)
+    cum = np.cumsum(srt, axis=1)
+    return np.argmax(cum >= alpha * cum[:, -1:] * (1.0 - 1e-15), axis=1) + 1
+
+
+def support_densities(a: np.ndarray, alpha: float):
+    """O1 ([P] S3): individual support densities tau_i(alpha) = |D_i(alpha)| / N_k of
+    the rows of `a`, and the pooled density gamma(alpha) = |union_i D_i(alpha)| / N_k of
+    those rows taken together (reading S26: the equations were lost; the text defines
+    both as fractions of the keys).  D_i keeps the keys of largest weight, lowest index
+    first among equal weights."""
+    n = a.shape[1]
+    sizes = support_size(a, alpha)
+    order = np.lexsort((np.broadcast_to(np.arange(n), a.shape), -a), axis=1)
+    union = np.zeros(n, dtype=bool)
+    for i in range(a.shape[0]):
+        union[order[i, :sizes[i]]] = True
+    return sizes / n, float(union.sum()) / n
+
+
+def oracle_affine_fit(osp: np.ndarray, dense: np.ndarray, tol: float = SV_REL_TOL):
+    """O3 ([P] S3, App. D.5): least-squares affine fit R ~ 1 b + O_sp B of the residual
+    R = dense - O_sp over all given rows, in fp64: the columns of the centred sparse
+    output are scaled to unit norm (zero columns left out), singular values below `tol`
+    times the largest are dropped, the fit is the projection of the centred residual on
+    the remaining left singular vectors, and the residual mean is the intercept.  Returns
+    (explained fraction of the residual's squared norm, remaining squared error)."""
+    R = dense - osp
+    Xc = osp - osp.mean(axis=0, keepdims=True)
+    nrm = np.linalg.norm(Xc, axis=0)
+    Xs = Xc[:, nrm > 0] / nrm[nrm > 0]
+    Rc = R - R.mean(axis=0, keepdims=True)
+    if Xs.shape[1]:
+        U, sig, _ = np.linalg.svd(Xs, full_matrices=False)
+        U = U[:, sig > tol * sig[0]] if sig[0] > 0 else U[:, :0]
+        fit = U @ (U.T @ Rc)
+    else:
+        fit = np.zeros_like(Rc)
+    err = float(((Rc - fit) ** 2).sum())
+    tot = float((R * R).sum())
+    return (1.0 - err / tot if tot > 0 else 0.0), err
+
+
 @dataclass
 class CallResult:
     part: Partition
@@ -646,7 +720,9 @@ def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] 
     `warm` is the previous call's state in a sequence ([P] App. C warm start).
     """
     N_q, N_k = Q.shape[0], K.shape[0]
-    part = partition(Q, K, V, p, head, warm) if part is None else part
+    if part is None:
+        part = (partition_semantic(Q, K, V, p, head) if p.partition == "semantic"
+                else partition(Q, K, V, p, head, warm))
     gq, gk = part.gq, part.gk
     S = route_scores(part.qbar, part.kbar, part.vbar, gk.sizes, p.d)
     beta = route_budget(p.rho, p.M, N_q, N_k)

@@ -691,3 +691,61 @@ def test_gqa_query_heads_share_the_key_partition_and_keep_their_own_query_groups
     assert np.array_equal(a.F_Q, b.F_Q)                    # M_Q comes from the K/V groups
     assert not np.array_equal(a.km_Q.labels, b.km_Q.labels)
     assert not np.array_equal(qs[0], qs[1])
+
+
+# ---------------------------------------------------------------- semantic partition, O1, O3
+def test_semantic_partition_clusters_raw_rows_and_full_density_is_dense():
+    Q, K, V = _clustered(31)
+    p = _small_workload_params(rho=1.0)
+    p.partition = "semantic"
+    res = O.sparsepr_call(Q, K, V, p)
+    assert np.abs(res.out - O.dense_attention(Q, K, V)).max() < 1e-12
+    # the key groups are the k-means of the raw key rows, and every value follows its key
+    km = O.kmeans(K, O.kmeans_init_indices(p.seed, 0, 0, p.C_k, K.shape[0]), p.kmeans_max_iter)
+    assert np.array_equal(res.part.km_K.labels, km.labels)
+    assert np.allclose(res.part.vbar, O.group_means(V, res.part.gk), rtol=0, atol=0)
+
+
+def test_support_size_hand_worked():
+    a = np.array([[0.5, 0.3, 0.1, 0.1],          # 0.5 + 0.3 + 0.1 >= 0.9
+                  [0.25, 0.25, 0.25, 0.25],      # ceil(0.9 * 4) = 4 keys
+                  [0.0, 1.0, 0.0, 0.0],          # one key
+                  [0.1, 0.2, 0.3, 0.4]])         # 0.4 + 0.3 + 0.2 >= 0.9
+    assert O.support_size(a, 0.9).tolist() == [3, 4, 1, 3]
+    assert O.support_size(a, 0.95).tolist() == [4, 4, 1, 4]
+    assert O.support_size(a[:1], 0.5).tolist() == [1]
+
+
+def test_pooled_support_density_is_the_union_of_the_supports():
+    n = 8
+    one_hot = np.eye(n)[[1, 5, 5]]
+    tau, gamma = O.support_densities(one_hot, 0.9)
+    assert tau.tolist() == [1 / n] * 3 and gamma == 2 / n      # keys {1, 5}
+    a = np.array([[0.6, 0.3, 0.1, 0, 0, 0, 0, 0],
+                  [0, 0, 0.1, 0.3, 0.6, 0, 0, 0]])
+    tau, gamma = O.support_densities(a, 0.85)                   # {0, 1} and {4, 3}
+    assert tau.tolist() == [2 / n, 2 / n] and gamma == 4 / n
+
+
+def test_oracle_affine_fit_recovers_a_planted_affine_residual_and_matches_lstsq():
+    rng = _rng(41)
+    n, d = 200, 6
+    osp = rng.standard_normal((n, d))
+    B = rng.standard_normal((d, d))
+    b = rng.standard_normal(d)
+    frac, err = O.oracle_affine_fit(osp, osp + b + osp @ B)
+    assert abs(frac - 1.0) < 1e-12 and err < 1e-20 * n
+    # a generic residual: the explained part is the least-squares projection on [1, O_sp]
+    R = rng.standard_normal((n, d))
+    frac, err = O.oracle_affine_fit(osp, osp + R)
+    A = np.hstack([np.ones((n, 1)), osp])
+    coef, *_ = np.linalg.lstsq(A, R, rcond=None)
+    rem = float(((R - A @ coef) ** 2).sum())
+    assert abs(err - rem) < 1e-10 * rem
+    assert abs(frac - (1.0 - rem / float((R * R).sum()))) < 1e-12
+    # a duplicated (rank-deficient) feature column changes nothing
+    frac2, err2 = O.oracle_affine_fit(np.hstack([osp, osp[:, :1]]), np.hstack([osp, osp[:, :1]]) + np.hstack([R, R[:, :1]]))
+    A2 = np.hstack([np.ones((n, 1)), osp])
+    coef2, *_ = np.linalg.lstsq(A2, np.hstack([R, R[:, :1]]), rcond=None)
+    rem2 = float(((np.hstack([R, R[:, :1]]) - A2 @ coef2) ** 2).sum())
+    assert abs(err2 - rem2) < 1e-10 * rem2
