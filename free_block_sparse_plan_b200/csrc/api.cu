@@ -57,6 +57,10 @@ sparsepr_status validate(const sparsepr_params* q) {
   if (q->engine != SPARSEPR_ENGINE_AUTO && q->engine != SPARSEPR_ENGINE_SIMT) return SPARSEPR_ERR_ARG;
   if (q->estimator < SPARSEPR_EST_RIDGE || q->estimator > SPARSEPR_EST_DIAGONAL) return SPARSEPR_ERR_ARG;
   if (q->G < 0 || (q->G > 1 && q->H % q->G != 0)) return SPARSEPR_ERR_SHAPE;
+  if (q->partition != SPARSEPR_PARTITION_RESPONSE && q->partition != SPARSEPR_PARTITION_SEMANTIC)
+    return SPARSEPR_ERR_ARG;
+  if (q->partition == SPARSEPR_PARTITION_SEMANTIC && q->d > kMaxR) return SPARSEPR_ERR_ARG;
+  if (q->reserved != 0) return SPARSEPR_ERR_ARG;
   return SPARSEPR_OK;
 }
 
@@ -69,6 +73,8 @@ Dims make_dims(const sparsepr_params* q) {
   d.estimator = q->estimator;
   d.G = q->G > 1 ? q->G : 1;
   d.Hk = d.H / d.G;
+  d.semantic = q->partition == SPARSEPR_PARTITION_SEMANTIC;
+  if (d.semantic) d.rK = d.rQ = d.d;        // coordinates are the raw channels
   d.nchK = cdiv(q->N_k, kSortChunk);
   d.nchQ = cdiv(q->N_q, kSortChunk);
   d.nsplit = cdiv(q->N_k, kProbeSplit);
@@ -209,8 +215,12 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_CUDA_OK(cudaMemsetAsync(p.b.pairs, 0, m.H * sizeof(long long), st));
   SPR_CUDA_OK(cudaMemsetAsync(p.b.kmReassigned, 0, 2 * m.H * sizeof(long long), st));
   // key side (paper S4.1, App. B.1)
-  SPR_TRY(launch_key_metric(p, st));
-  SPR_TRY(p.warm ? launch_warm_factor(p, false, st) : launch_eigen_factor(p, false, st));
+  if (m.semantic) {
+    SPR_TRY(launch_identity_factors(p, st));       // F_K = F_Q = I: raw rows as coordinates
+  } else {
+    SPR_TRY(launch_key_metric(p, st));
+    SPR_TRY(p.warm ? launch_warm_factor(p, false, st) : launch_eigen_factor(p, false, st));
+  }
   SPR_TRY(launch_project_keys(p, st));
   if (labK) {
     SPR_CUDA_OK(cudaMemcpyAsync(p.b.labK, labK, sizeof(int) * m.Hk * m.Nk,
@@ -222,8 +232,10 @@ sparsepr_status run_plan(Plan& p, const int32_t* labQ, const int32_t* labK, cuda
   SPR_TRY(launch_finalize_groups(p, false, st));
   SPR_TRY(launch_centroids(p, false, st));
   // query side (paper S4.1, App. B.2)
-  SPR_TRY(launch_query_metric(p, st));
-  SPR_TRY(p.warm ? launch_warm_factor(p, true, st) : launch_eigen_factor(p, true, st));
+  if (!m.semantic) {
+    SPR_TRY(launch_query_metric(p, st));
+    SPR_TRY(p.warm ? launch_warm_factor(p, true, st) : launch_eigen_factor(p, true, st));
+  }
   SPR_TRY(launch_project_queries(p, st));
   if (labQ) {
     SPR_CUDA_OK(cudaMemcpyAsync(p.b.labQ, labQ, sizeof(int) * m.H * m.Nq,
@@ -342,7 +354,7 @@ sparsepr_status sparsepr_plan_warm(const sparsepr_params* params, const void* Q,
                                    const void* V, const void* state, void* workspace,
                                    size_t workspace_bytes, void* stream, sparsepr_plan_t* out) {
   if (!state || (reinterpret_cast<uintptr_t>(state) & 255)) return SPARSEPR_ERR_ARG;
-  if (params && params->G > 1) return SPARSEPR_ERR_ARG;
+  if (params && (params->G > 1 || params->partition != SPARSEPR_PARTITION_RESPONSE)) return SPARSEPR_ERR_ARG;
   return plan_common(params, Q, K, V, nullptr, nullptr, state, workspace, workspace_bytes, stream, out);
 }
 

@@ -62,13 +62,13 @@ constexpr int kProjXs = kProjRows + 4;     // transposed tile row stride (floats
 template <int R, bool RMS>
 __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int N, const double* Fall, int r,
                                                       double* out, __nv_bfloat16* xhi, __nv_bfloat16* xlo,
-                                                      float* xn, int Npad) {
+                                                      float* xn, int Npad, int fdiv) {
   constexpr int CPT = R / 16;              // columns per thread
   extern __shared__ double smd[];
   const int d = m.d, h = blockIdx.y;
   double* F = smd;                         // [d][R], zero columns k >= r
   float* Xt = reinterpret_cast<float*>(smd + d * R);  // [d][kProjXs]: Xt[j][row]
-  const double* Fh = Fall + (long long)(RMS ? h / m.G : h) * d * r;   // queries: their K/V head's F_Q
+  const double* Fh = Fall + (long long)(h / fdiv) * d * r;   // queries: their K/V head's F_Q
   for (int e = threadIdx.x; e < d * R; e += blockDim.x) {
     const int j = e / R, k = e % R;
     F[e] = k < r ? Fh[j * r + k] : 0.0;
@@ -173,16 +173,21 @@ __global__ void __launch_bounds__(256) project_kernel(Dims m, const void* X, int
   }
 }
 
+// query: one block row per query head, each reading its K/V head's factor (fdiv = G);
+// keys: one per K/V head.  RMS: the query coordinates' normalisation (not in the semantic
+// partition, whose coordinates are the raw rows).
 template <bool RMS>
-sparsepr_status launch_project(const Plan& p, const void* X, int N, const double* F, int r, double* out,
-                               __nv_bfloat16* xhi, __nv_bfloat16* xlo, float* xn, int Npad, cudaStream_t st) {
+sparsepr_status launch_project(const Plan& p, bool query, const void* X, int N, const double* F, int r,
+                               double* out, __nv_bfloat16* xhi, __nv_bfloat16* xlo, float* xn, int Npad,
+                               cudaStream_t st) {
   const int d = p.dm.d;
   const int rows = xhi ? Npad : N;
-  dim3 grid(cdiv(rows, kProjRows * kProjTiles), RMS ? p.dm.H : p.dm.Hk);
+  const int fdiv = query ? p.dm.G : 1;
+  dim3 grid(cdiv(rows, kProjRows * kProjTiles), query ? p.dm.H : p.dm.Hk);
   auto run = [&](auto kern, int R) -> sparsepr_status {
     const size_t smem = (size_t)d * R * sizeof(double) + (size_t)d * kProjXs * sizeof(float);
     SPR_CUDA_OK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    kern<<<grid, 256, smem, st>>>(p.dm, X, N, F, r, out, xhi, xlo, xn, Npad);
+    kern<<<grid, 256, smem, st>>>(p.dm, X, N, F, r, out, xhi, xlo, xn, Npad, fdiv);
     SPR_LAUNCH_OK();
     return SPARSEPR_OK;
   };
@@ -664,8 +669,8 @@ sparsepr_status launch_project_side(const Plan& p, bool query, cudaStream_t st) 
   __nv_bfloat16* xlo = fuse ? b.kmXlo : nullptr;
   float* xn = fuse ? b.kmXn : nullptr;
   const int Npad = km_tc_npad(N);
-  return query ? launch_project<true>(p, X, N, F, r, out, xhi, xlo, xn, Npad, st)
-               : launch_project<false>(p, X, N, F, r, out, xhi, xlo, xn, Npad, st);
+  return query && !m.semantic ? launch_project<true>(p, true, X, N, F, r, out, xhi, xlo, xn, Npad, st)
+                              : launch_project<false>(p, query, X, N, F, r, out, xhi, xlo, xn, Npad, st);
 }
 
 sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st) { return launch_project_side(p, false, st); }

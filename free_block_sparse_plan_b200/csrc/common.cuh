@@ -37,6 +37,7 @@ struct Dims {
   unsigned long long seed;
   int estimator;       // sparsepr_estimator
   int G, Hk;           // query heads per K/V head; K/V heads (H / G)
+  int semantic;        // semantic reference partition: coordinates = raw rows (rK = rQ = d)
   int nchK, nchQ;      // counting-sort chunks per head
   int nsplit;          // partial blocks of the exact probe attention
   double beta;         // per-query key budget (rho - M/N_q) * N_k
@@ -228,6 +229,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
 sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st);
 sparsepr_status launch_eigen_factor(const Plan& p, bool query, cudaStream_t st);
 sparsepr_status launch_warm_factor(const Plan& p, bool query, cudaStream_t st);
+sparsepr_status launch_identity_factors(const Plan& p, cudaStream_t st);
 sparsepr_status launch_save_state(const Plan& p, void* state, cudaStream_t st);
 sparsepr_status launch_project_keys(const Plan& p, cudaStream_t st);
 sparsepr_status launch_project_queries(const Plan& p, cudaStream_t st);

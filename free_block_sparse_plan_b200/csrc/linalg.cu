@@ -652,7 +652,29 @@ __global__ void __launch_bounds__(kLinThreads) fit_smem_kernel(Dims m, Buffers b
   }
 }
 
+// Semantic reference partition: F_K = F_Q = I (d x d) for every K/V head, so the
+// coordinates are the raw rows; no eigenvalues.
+__global__ void identity_factor_kernel(Dims m, double* FK64, float* FK, double* FQ64, float* FQ,
+                                       double* lamK, double* lamQ) {
+  const int h = blockIdx.x, d = m.d;
+  for (int e = threadIdx.x; e < d * d; e += blockDim.x) {
+    const double v = (e / d == e % d) ? 1.0 : 0.0;
+    const long long o = (long long)h * d * d + e;
+    FK64[o] = v; FK[o] = (float)v; FQ64[o] = v; FQ[o] = (float)v;
+  }
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    lamK[(long long)h * d + k] = 0.0;
+    lamQ[(long long)h * d + k] = 0.0;
+  }
+}
+
 }  // namespace
+
+sparsepr_status launch_identity_factors(const Plan& p, cudaStream_t st) {
+  identity_factor_kernel<<<p.dm.Hk, 256, 0, st>>>(p.dm, p.b.FK64, p.b.FK, p.b.FQ64, p.b.FQ, p.b.lamK, p.b.lamQ);
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
 
 sparsepr_status launch_key_metric(const Plan& p, cudaStream_t st) {
   const size_t smem = 64 * p.dm.d * sizeof(float);

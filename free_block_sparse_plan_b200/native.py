@@ -28,6 +28,7 @@ SPARSEPR_F32 = 0
 SPARSEPR_BF16 = 1
 SPARSEPR_ENGINE_AUTO = 0
 SPARSEPR_EST_RIDGE, SPARSEPR_EST_MEAN, SPARSEPR_EST_SCALAR, SPARSEPR_EST_DIAGONAL = 0, 1, 2, 3
+SPARSEPR_PARTITION_RESPONSE, SPARSEPR_PARTITION_SEMANTIC = 0, 1
 SPARSEPR_ENGINE_SIMT = 1
 
 EXPORTS = [
@@ -55,7 +56,8 @@ class sparsepr_params(ctypes.Structure):
                 ("C_q", c_int32), ("C_k", c_int32), ("M", c_int32), ("r", c_int32),
                 ("lam", c_double), ("target_density", c_double),
                 ("kmeans_max_iter", c_int32), ("engine", c_int32), ("seed", c_uint64),
-                ("estimator", c_int32), ("G", c_int32)]
+                ("estimator", c_int32), ("G", c_int32), ("partition", c_int32),
+                ("reserved", c_int32)]
 
 
 class sparsepr_stats(ctypes.Structure):
@@ -135,20 +137,20 @@ def _check(status: int, where: str):
 
 def make_params(H, N_q, N_k, d, dtype, M_s, r_K, r_Q, C_q, C_k, M, r, lam, target_density,
                 kmeans_max_iter=25, seed=0, engine=SPARSEPR_ENGINE_AUTO, estimator=0,
-                G=1) -> sparsepr_params:
+                G=1, partition=0) -> sparsepr_params:
     if isinstance(dtype, str):
         dtype = {"f32": SPARSEPR_F32, "bf16": SPARSEPR_BF16}[dtype]
     return sparsepr_params(H=H, N_q=N_q, N_k=N_k, d=d, dtype=dtype, M_s=M_s, r_K=r_K, r_Q=r_Q,
                            C_q=C_q, C_k=C_k, M=M, r=r, lam=lam, target_density=target_density,
                            kmeans_max_iter=kmeans_max_iter, engine=engine, seed=seed,
-                           estimator=estimator, G=G)
+                           estimator=estimator, G=G, partition=partition, reserved=0)
 
 
 def params_from_dict(p: dict, engine=SPARSEPR_ENGINE_AUTO) -> sparsepr_params:
     return make_params(p["H"], p["N_q"], p["N_k"], p["d"], p["dtype"], p["M_s"], p["r_K"],
                        p["r_Q"], p["C_q"], p["C_k"], p["M"], p["r"], p["lam"],
                        p["target_density"], p["kmeans_max_iter"], p["seed"], engine,
-                       p.get("estimator", 0), p.get("G", 1))
+                       p.get("estimator", 0), p.get("G", 1), p.get("partition", 0))
 
 
 # ----------------------------------------------------------------------------------
@@ -270,6 +272,7 @@ def _stream(stream=None) -> int:
 def _export_layout(p: sparsepr_params, name: str):
     H, d = p.H, p.d
     Hk = H // max(p.G, 1)                # K/V heads
+    rK, rQ = (d, d) if p.partition == SPARSEPR_PARTITION_SEMANTIC else (p.r_K, p.r_Q)
     i32, f64, f32, i64 = np.int32, np.float64, np.float32, np.int64
     return {
         "LABELS_K": (i32, (Hk, p.N_k)), "LABELS_Q": (i32, (H, p.N_q)),
@@ -279,11 +282,11 @@ def _export_layout(p: sparsepr_params, name: str):
         "CELL_COUNT": (i32, (H, p.C_q)), "CELL_IDS": (i32, (H, p.C_q, p.C_k)),
         "PROBES": (i32, (H, p.M)), "PROBE_COUNT": (i32, (H, p.C_q)),
         "KMEANS_ITERS": (i32, (H, 2)), "OBJECTIVE": (f64, (H, 2)), "PAIRS": (i64, (H,)),
-        "FACTOR_K": (f64, (Hk, d, p.r_K)), "FACTOR_Q": (f64, (Hk, d, p.r_Q)),
-        "EIG_K": (f64, (Hk, p.r_K)), "EIG_Q": (f64, (Hk, p.r_Q)),
+        "FACTOR_K": (f64, (Hk, d, rK)), "FACTOR_Q": (f64, (Hk, d, rQ)),
+        "EIG_K": (f64, (Hk, rK)), "EIG_Q": (f64, (Hk, rQ)),
         "METRIC_K": (f64, (Hk, d, d)), "METRIC_Q": (f64, (Hk, d, d)),
-        "PHI_K": (f64, (Hk, p.N_k, p.r_K)), "PHI_Q": (f64, (H, p.N_q, p.r_Q)),
-        "CENTRES_Q": (f64, (H, p.C_q, p.r_Q)), "SCORES": (f64, (H, p.C_q, p.C_k)),
+        "PHI_K": (f64, (Hk, p.N_k, rK)), "PHI_Q": (f64, (H, p.N_q, rQ)),
+        "CENTRES_Q": (f64, (H, p.C_q, rQ)), "SCORES": (f64, (H, p.C_q, p.C_k)),
         "OSP": (f32, (H, p.N_q, d)), "ODENSE_PROBE": (f32, (H, p.M, d)),
         "FIT_MU_X": (f64, (H, d)), "FIT_MU_R": (f64, (H, d)), "FIT_S": (f64, (H, d)),
         "FIT_B": (f64, (H, d, d)), "FIT_P": (f64, (H, d, d)), "FIT_REFF": (i32, (H,)),

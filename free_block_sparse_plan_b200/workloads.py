@@ -69,6 +69,8 @@ class Workload:
     drift: float = 0.05
     # grouped-query attention: G query heads share each K/V head (H/G K/V heads)
     G: int = 1
+    # 0 response-coupled partition (the method), 1 semantic reference partition
+    partition: int = 0
 
     @property
     def H_kv(self) -> int:
@@ -88,7 +90,7 @@ class Workload:
                     M_s=self.M_s, r_K=self.r_K, r_Q=self.r_Q, C_q=self.C_q,
                     C_k=self.C_k, M=self.M, r=self.r, lam=self.lam,
                     target_density=self.rho, kmeans_max_iter=self.kmeans_max_iter,
-                    seed=self.seed, estimator=self.estimator, G=self.G)
+                    seed=self.seed, estimator=self.estimator, G=self.G, partition=self.partition)
 
 
 TINY = Workload("tiny-f32-1x1024x64", H=1, N=1024, d=64, dtype="f32",

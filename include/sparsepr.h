@@ -81,6 +81,15 @@ typedef enum {
   SPARSEPR_EST_DIAGONAL = 3   /* B = diag(b), penalty lambda |b|^2, no projection */
 } sparsepr_estimator;
 
+/* Partition of sparsepr_plan ("Partition the Support, Reconstruct the Residual", S3 and
+ * the ablation tables): the method's response-coupled partition, or the semantic
+ * reference partition, which runs the same k-means on the raw key rows and the raw query
+ * rows (no metric, no eigen factor, no RMS step; requires d <= 64). */
+typedef enum {
+  SPARSEPR_PARTITION_RESPONSE = 0,
+  SPARSEPR_PARTITION_SEMANTIC = 1
+} sparsepr_partition;
+
 /*
  * Problem and hyper-parameters of one call (paper S2, S4; values of the review page's
  * hyper-parameter table: r_K=48, r_Q=64, M=64, r=16, lambda=0.1).
@@ -111,6 +120,11 @@ typedef enum {
  *                     FACTOR_K, EIG_K, METRIC_K, PHI_K, KBAR, METRIC_Q, FACTOR_Q, EIG_Q)
  *                     then have H/G rows; KMEANS_ITERS and OBJECTIVE keep H rows, the key
  *                     column of row h being that of K/V head h/G.  Warm starts take G <= 1.
+ *   partition         sparsepr_partition (0 unless comparing).  With the semantic partition
+ *                     r_K and r_Q are ignored (the coordinates are the d raw channels),
+ *                     FACTOR_K / FACTOR_Q export the identity and METRIC_* / EIG_* are not
+ *                     computed; warm starts take the response partition.
+ *   reserved          must be 0
  */
 typedef struct {
   int32_t H, N_q, N_k, d;
@@ -123,6 +137,8 @@ typedef struct {
   uint64_t seed;
   int32_t estimator;
   int32_t G;
+  int32_t partition;
+  int32_t reserved;
 } sparsepr_params;
 
 typedef struct sparsepr_plan_s* sparsepr_plan_t;

@@ -428,6 +428,7 @@ class Fit:
 
 
 ESTIMATORS = ("ridge", "mean", "scalar", "diagonal")   # codes 0..3 of the C ABI
+PARTITIONS = ("response", "semantic")                  # codes 0..1 of the C ABI
 
 
 def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int,
@@ -514,7 +515,7 @@ class Params:
                    C_k=p["C_k"], M=p["M"], r=p["r"], lam=p["lam"],
                    rho=p["target_density"], kmeans_max_iter=p["kmeans_max_iter"],
                    seed=p["seed"], estimator=ESTIMATORS[int(p.get("estimator", 0))],
-                   partition=p.get("partition", "response"))
+                   partition=PARTITIONS[int(p.get("partition", 0))])
 
 
 @dataclass
@@ -616,7 +617,7 @@ def partition(Q, K, V, p: Params, head: int, warm: Optional[WarmState] = None,
                      lam_Q, phiQ, km_Q, gq, qbar)
 
 
-def partition_semantic(Q, K, V, p: Params, head: int) -> Partition:
+def partition_semantic(Q, K, V, p: Params, head: int, kv_head: Optional[int] = None) -> Partition:
     """The reference (semantic) partition of [P] S3 and of its ablations: k-means applied
     separately to the raw key rows and to the raw query rows, each value following its
     key.  Reading S25: the same Lloyd steps, init streams and stop rule as the response
@@ -624,7 +625,8 @@ def partition_semantic(Q, K, V, p: Params, head: int) -> Partition:
     coordinate maps are the identity, so probe distances (S16) are taken on raw query rows.
     """
     N_q, N_k, d = Q.shape[0], K.shape[0], Q.shape[1]
-    km_K = kmeans(K, kmeans_init_indices(p.seed, head, 0, p.C_k, N_k), p.kmeans_max_iter)
+    kv = head if kv_head is None else kv_head            # GQA: the K/V head's init stream
+    km_K = kmeans(K, kmeans_init_indices(p.seed, kv, 0, p.C_k, N_k), p.kmeans_max_iter)
     gk = compact_groups(km_K.labels, p.C_k)
     kbar = group_means(K, gk)
     vbar = group_means(V, gk)

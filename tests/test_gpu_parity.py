@@ -321,6 +321,35 @@ def check_injected_head_gqa(plan, out_h, res, h, w):
     assert rel(out_h[res.rows], res.out) < TOL[w.dtype]
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_semantic_partition_matches_oracle(name):
+    # the reference partition of the paper's S3 and ablations: k-means on raw rows
+    w = (W.TINY if name == "tiny" else W.MID.with_(H=2)).with_(partition=1)
+    P = O.Params.from_dict(w.params())
+    assert P.partition == "semantic"
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    rows = None if w.N <= 4096 else (np.arange(2048) * w.N) // 2048
+    heads = [W.make_head(w, h) for h in range(w.H)]
+    parts = [O.partition_semantic(*heads[h], P, h) for h in range(w.H)]
+    plan, out, _ = gpu_call(w, inputs=(Q, K, V))
+    assert plan.check() == 0
+    labK, labQ = plan.export("LABELS_K"), plan.export("LABELS_Q")
+    obj = plan.export("OBJECTIVE")
+    for h, part in enumerate(parts):
+        assert np.mean(labK[h] == part.km_K.labels) >= 0.999
+        assert np.mean(labQ[h] == part.km_Q.labels) >= 0.999
+        assert abs(obj[h][0] - part.km_K.objective) <= 1e-4 * part.km_K.objective
+        assert abs(obj[h][1] - part.km_Q.objective) <= 1e-4 * part.km_Q.objective
+    assert np.array_equal(plan.export("PHI_Q")[0], heads[0][0])      # raw rows, no RMS step
+    labQi = torch.tensor(np.stack([p_.km_Q.labels for p_ in parts]), dtype=torch.int32, device="cuda")
+    labKi = torch.tensor(np.stack([p_.km_K.labels for p_ in parts]), dtype=torch.int32, device="cuda")
+    plan, out, _ = gpu_call(w, inputs=(Q, K, V), labels=(labQi, labKi))
+    assert plan.check() == 0
+    for h, part in enumerate(parts):
+        res = O.sparsepr_call(*heads[h], P, head=h, rows=rows, part=part)
+        check_injected_head(plan, out[h].double().cpu().numpy(), res, h, w)
+
+
 def test_tiny_simt_engine_equals_auto():
     w = W.TINY
     _, out_a, inputs = gpu_call(w)

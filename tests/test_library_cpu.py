@@ -33,8 +33,10 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_struct_layout_matches_header():
-    assert ctypes.sizeof(N.sparsepr_params) == 88
+    assert ctypes.sizeof(N.sparsepr_params) == 96
     assert N.sparsepr_params.estimator.offset == 80
+    assert N.sparsepr_params.G.offset == 84
+    assert N.sparsepr_params.partition.offset == 88
     assert N.sparsepr_params.lam.offset == 48
     assert N.sparsepr_params.seed.offset == 72
 
@@ -69,6 +71,7 @@ def test_workspace_size_positive_and_monotone():
     ("target_density", 1.5, N.SPARSEPR_ERR_ARG), ("target_density", 0.01, N.SPARSEPR_ERR_ARG),
     ("kmeans_max_iter", 0, N.SPARSEPR_ERR_ARG), ("engine", 3, N.SPARSEPR_ERR_ARG),
     ("G", -1, N.SPARSEPR_ERR_SHAPE), ("G", 5, N.SPARSEPR_ERR_SHAPE),
+    ("partition", 2, N.SPARSEPR_ERR_ARG), ("reserved", 1, N.SPARSEPR_ERR_ARG),
 ])
 def test_invalid_parameters_rejected_on_host(field, value, status):
     p = _params()
@@ -109,6 +112,19 @@ def test_gqa_group_sizes_and_warm_start_restriction():
         assert N.sparsepr_workspace_size(p) > 0
     p = _params()
     p.H, p.G = 4, 2
+    h = ctypes.c_void_p()
+    st = N.lib().sparsepr_plan_warm(ctypes.byref(p), 256, 256, 256, 256, 256, 1 << 40, None, ctypes.byref(h))
+    assert st == N.SPARSEPR_ERR_ARG and not h.value
+
+
+def test_semantic_partition_limits():
+    # the raw channels are the coordinates: d <= 64; warm starts take the response partition
+    p = _params(partition=1)
+    assert N.sparsepr_workspace_size(p) > 0
+    q = N.params_from_dict(dict(W.WAN.params(), partition=1))
+    with pytest.raises(N.SparsePRError) as ei:
+        N.sparsepr_workspace_size(q)
+    assert ei.value.status == N.SPARSEPR_ERR_ARG
     h = ctypes.c_void_p()
     st = N.lib().sparsepr_plan_warm(ctypes.byref(p), 256, 256, 256, 256, 256, 1 << 40, None, ctypes.byref(h))
     assert st == N.SPARSEPR_ERR_ARG and not h.value
