@@ -128,3 +128,24 @@ def test_semantic_partition_limits():
     h = ctypes.c_void_p()
     st = N.lib().sparsepr_plan_warm(ctypes.byref(p), 256, 256, 256, 256, 256, 1 << 40, None, ctypes.byref(h))
     assert st == N.SPARSEPR_ERR_ARG and not h.value
+
+
+def test_bench_traffic_record_matches_kernel_source_by_hash(tmp_path, monkeypatch):
+    # the recorded DRAM traffic is used only while the kernel source is the one captured,
+    # scaled by heads, and only for the captured workload family and shape
+    import hashlib
+    import json
+    import bench
+    src = b"// kernel source\n"
+    (tmp_path / "free_block_sparse_plan_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "free_block_sparse_plan_b200" / "csrc" / "k.cu").write_bytes(src)
+    rec = {"k.cu": [{"family": "mid", "N": 16384, "d": 64, "H": 12, "bytes_per_launch": 1200,
+                     "sha256": hashlib.sha256(src).hexdigest()}]}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("k.cu", W.MID) == 1200.0
+    assert bench.measured_traffic("k.cu", W.MID.with_(H=6)) == 600.0
+    assert bench.measured_traffic("k.cu", W.WAN) is None
+    (tmp_path / "free_block_sparse_plan_b200" / "csrc" / "k.cu").write_bytes(src + b"//")
+    assert bench.measured_traffic("k.cu", W.MID) is None
