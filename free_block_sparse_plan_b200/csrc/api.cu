@@ -360,6 +360,7 @@ sparsepr_status sparsepr_plan_warm(const sparsepr_params* params, const void* Q,
 
 sparsepr_status sparsepr_save_state(sparsepr_plan_t plan, void* state, void* stream) {
   if (!plan || !state || (reinterpret_cast<uintptr_t>(state) & 255)) return SPARSEPR_ERR_ARG;
+  if (plan->p.dm.G > 1 || plan->p.dm.semantic) return SPARSEPR_ERR_ARG;   // as sparsepr_plan_warm
   if (plan->p.stage < 1) return SPARSEPR_ERR_STATE;
   return launch_save_state(plan->p, state, reinterpret_cast<cudaStream_t>(stream));
 }

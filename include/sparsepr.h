@@ -205,7 +205,8 @@ sparsepr_status sparsepr_plan_from_labels(const sparsepr_params* params, const v
  * sparsepr_check).  The state is read by work enqueued on `stream`; saving the new
  * plan's state into the same buffer later on the same stream is allowed.  After a warm
  * plan, the EIG_K / EIG_Q exports are zero for the heads updated this way.
- * Errors: SPARSEPR_ERR_ARG for a null or misaligned state; otherwise as sparsepr_plan.
+ * Errors: SPARSEPR_ERR_ARG for a null or misaligned state, or for parameters with G > 1 or
+ * the semantic partition (both calls); otherwise as sparsepr_plan.
  */
 sparsepr_status sparsepr_state_size(const sparsepr_params* params, size_t* bytes);
 sparsepr_status sparsepr_save_state(sparsepr_plan_t plan, void* state, void* stream);
