@@ -149,6 +149,23 @@ def cpu_oracle_sample(w, min_seconds=10.0):
                       f"value = executed-pair FLOPs of those heads / time"}
 
 
+def tile_pairs(sizes_q, n_q, cell_cnt, cell_ids, sizes_k, G=1, tile=128):
+    """Query-key pairs the tensor-core attention engine processes and the routed pairs
+    among them: every query group runs in 128-row tiles against its selected keys in
+    128-key tiles, so a group of s rows with n selected keys costs 128 ceil(s/128) x
+    128 ceil(n/128) pairs and routes s n of them.  Arrays as the plan exports them."""
+    import numpy as np
+    proc = routed = 0
+    for h in range(sizes_q.shape[0]):
+        sk = sizes_k[h // G].astype(np.int64)
+        for a in range(int(n_q[h])):
+            s = int(sizes_q[h][a])
+            n = int(sk[cell_ids[h][a][:int(cell_cnt[h][a])]].sum())
+            proc += tile * (-(-s // tile)) * tile * (-(-n // tile))
+            routed += s * n
+    return proc, routed
+
+
 def workload_config(w):
     """The `config` object both arms report for workload w."""
     return {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "C_q": w.C_q, "C_k": w.C_k,
@@ -264,6 +281,15 @@ def main():
     plan = call()
     st = plan.stats()
     torch.cuda.synchronize()
+    padding = None
+    try:                                   # host-side accounting from the plan's exports
+        ex = {k: plan.export(k) for k in ("SIZES_Q", "GROUPS_Q", "CELL_COUNT", "CELL_IDS", "SIZES_K")}
+        proc, routed = tile_pairs(ex["SIZES_Q"], ex["GROUPS_Q"], ex["CELL_COUNT"], ex["CELL_IDS"],
+                                  ex["SIZES_K"], wr.G)
+        padding = {"processed_pairs": proc, "routed_pairs": routed,
+                   "fraction": 1.0 - routed / proc if proc else 0.0}
+    except Exception as e:                 # the accounting never stops the measurement
+        padding = {"unavailable": str(e)[:200]}
 
     def barrier():
         if world > 1:
@@ -407,6 +433,10 @@ def main():
         line["e2e"] = e2e
     if warm:
         line["warm_start"] = warm
+    if padding and "processed_pairs" in padding and world == 1:
+        # the attend kernel's rate over the pairs it processes (padding included)
+        padding["attend_tflops_processed"] = 4.0 * w.d * padding["processed_pairs"] / (attend_ms * 1e-3) / 1e12
+    line["attention_tiles"] = padding
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w)
     if world > 1:

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from conftest import ROOT
@@ -149,3 +150,21 @@ def test_bench_traffic_record_matches_kernel_source_by_hash(tmp_path, monkeypatc
     assert bench.measured_traffic("k.cu", W.WAN) is None
     (tmp_path / "free_block_sparse_plan_b200" / "csrc" / "k.cu").write_bytes(src + b"//")
     assert bench.measured_traffic("k.cu", W.MID) is None
+
+
+def test_bench_tile_pair_accounting():
+    import bench
+    sizes_q = np.array([[148, 20, 0]])             # two query groups
+    n_q = np.array([2])
+    cell_cnt = np.array([[2, 1, 0]])
+    cell_ids = np.array([[[0, 2, 0], [1, 0, 0], [0, 0, 0]]])
+    sizes_k = np.array([[100, 300, 60]])
+    proc, routed = bench.tile_pairs(sizes_q, n_q, cell_cnt, cell_ids, sizes_k)
+    # group 0: 148 rows -> 256, keys 100 + 60 = 160 -> 256; group 1: 20 -> 128, 300 -> 384
+    assert proc == 256 * 256 + 128 * 384
+    assert routed == 148 * 160 + 20 * 300
+    # GQA: query head h reads the key sizes of K/V head h // G
+    proc2, _ = bench.tile_pairs(np.vstack([sizes_q, sizes_q]), np.array([2, 2]),
+                                np.vstack([cell_cnt, cell_cnt]), np.vstack([cell_ids, cell_ids]),
+                                sizes_k, G=2)
+    assert proc2 == 2 * proc
