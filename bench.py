@@ -166,6 +166,21 @@ def tile_pairs(sizes_q, n_q, cell_cnt, cell_ids, sizes_k, G=1, tile=128):
     return proc, routed
 
 
+def attention_tile_accounting(plan, w, G):
+    """Processed and routed attention pairs of a finished plan (tensor-core engine only);
+    host-side, from the plan's exports, and never allowed to stop the measurement."""
+    if w.dtype != "bf16" or w.d not in (64, 128):
+        return {"unavailable": "the CUDA-core engine serves this dtype / head dimension"}
+    try:
+        ex = {k: plan.export(k) for k in ("SIZES_Q", "GROUPS_Q", "CELL_COUNT", "CELL_IDS", "SIZES_K")}
+        proc, routed = tile_pairs(ex["SIZES_Q"], ex["GROUPS_Q"], ex["CELL_COUNT"], ex["CELL_IDS"],
+                                  ex["SIZES_K"], G)
+    except Exception as e:
+        return {"unavailable": str(e)[:200]}
+    return {"processed_pairs": proc, "routed_pairs": routed,
+            "fraction": 1.0 - routed / proc if proc else 0.0}
+
+
 def workload_config(w):
     """The `config` object both arms report for workload w."""
     return {"workload": w.name, "H": w.H, "N": w.N, "d": w.d, "C_q": w.C_q, "C_k": w.C_k,
@@ -281,15 +296,7 @@ def main():
     plan = call()
     st = plan.stats()
     torch.cuda.synchronize()
-    padding = None
-    try:                                   # host-side accounting from the plan's exports
-        ex = {k: plan.export(k) for k in ("SIZES_Q", "GROUPS_Q", "CELL_COUNT", "CELL_IDS", "SIZES_K")}
-        proc, routed = tile_pairs(ex["SIZES_Q"], ex["GROUPS_Q"], ex["CELL_COUNT"], ex["CELL_IDS"],
-                                  ex["SIZES_K"], wr.G)
-        padding = {"processed_pairs": proc, "routed_pairs": routed,
-                   "fraction": 1.0 - routed / proc if proc else 0.0}
-    except Exception as e:                 # the accounting never stops the measurement
-        padding = {"unavailable": str(e)[:200]}
+    padding = attention_tile_accounting(plan, w, wr.G)
 
     def barrier():
         if world > 1:
