@@ -168,3 +168,26 @@ def test_bench_tile_pair_accounting():
                                 np.vstack([cell_cnt, cell_cnt]), np.vstack([cell_ids, cell_ids]),
                                 sizes_k, G=2)
     assert proc2 == 2 * proc
+
+
+def test_bench_tile_accounting_from_plan_exports():
+    import bench
+
+    class FakePlan:
+        def export(self, name):
+            return {"SIZES_Q": np.array([[148, 20, 0]]), "GROUPS_Q": np.array([2]),
+                    "CELL_COUNT": np.array([[2, 1, 0]]),
+                    "CELL_IDS": np.array([[[0, 2, 0], [1, 0, 0], [0, 0, 0]]]),
+                    "SIZES_K": np.array([[100, 300, 60]])}[name]
+
+    acc = bench.attention_tile_accounting(FakePlan(), W.MID, 1)
+    assert acc["processed_pairs"] == 256 * 256 + 128 * 384
+    assert acc["routed_pairs"] == 148 * 160 + 20 * 300
+    assert abs(acc["fraction"] - (1 - acc["routed_pairs"] / acc["processed_pairs"])) < 1e-15
+    assert "unavailable" in bench.attention_tile_accounting(FakePlan(), W.TINY, 1)   # fp32: CUDA cores
+
+    class Broken:
+        def export(self, name):
+            raise RuntimeError("no such export")
+
+    assert "unavailable" in bench.attention_tile_accounting(Broken(), W.MID, 1)
