@@ -177,8 +177,14 @@ def attention_tile_accounting(plan, w, G):
                                   ex["SIZES_K"], G)
     except Exception as e:
         return {"unavailable": str(e)[:200]}
-    return {"processed_pairs": proc, "routed_pairs": routed,
-            "fraction": 1.0 - routed / proc if proc else 0.0}
+    out = {"processed_pairs": proc, "routed_pairs": routed,
+           "fraction": 1.0 - routed / proc if proc else 0.0}
+    try:                                   # realised (non-empty) group counts per head
+        out["groups_q"] = [int(x) for x in ex["GROUPS_Q"]]
+        out["groups_kv"] = [int(x) for x in plan.export("GROUPS_K")]
+    except Exception:
+        pass
+    return out
 
 
 def workload_config(w):

@@ -178,9 +178,10 @@ def test_bench_tile_accounting_from_plan_exports():
             return {"SIZES_Q": np.array([[148, 20, 0]]), "GROUPS_Q": np.array([2]),
                     "CELL_COUNT": np.array([[2, 1, 0]]),
                     "CELL_IDS": np.array([[[0, 2, 0], [1, 0, 0], [0, 0, 0]]]),
-                    "SIZES_K": np.array([[100, 300, 60]])}[name]
+                    "SIZES_K": np.array([[100, 300, 60]]), "GROUPS_K": np.array([3])}[name]
 
     acc = bench.attention_tile_accounting(FakePlan(), W.MID, 1)
+    assert acc["groups_q"] == [2] and acc["groups_kv"] == [3]
     assert acc["processed_pairs"] == 256 * 256 + 128 * 384
     assert acc["routed_pairs"] == 148 * 160 + 20 * 300
     assert abs(acc["fraction"] - (1 - acc["routed_pairs"] / acc["processed_pairs"])) < 1e-15
