@@ -749,3 +749,23 @@ def test_oracle_affine_fit_recovers_a_planted_affine_residual_and_matches_lstsq(
     coef2, *_ = np.linalg.lstsq(A2, np.hstack([R, R[:, :1]]), rcond=None)
     rem2 = float(((np.hstack([R, R[:, :1]]) - A2 @ coef2) ** 2).sum())
     assert abs(err2 - rem2) < 1e-10 * rem2
+
+
+def test_warm_query_centres_pass_the_rms_step():
+    # W2: a non-empty query label restarts at phi_Q(qbar) = (qbar F_Q) / rms, a point of the
+    # RMS sphere (raw qbar F_Q is not), and the partition's query k-means starts there
+    from free_block_sparse_plan_b200 import workloads as W
+    w = W.TINY
+    p = O.Params.from_dict(w.params())
+    Q, K, V = W.make_head(w, 0)
+    st = O.warm_state(O.partition(Q, K, V, p, 0), p)
+    Q1, K1, V1 = W.make_head(w.with_(step=1), 0)
+    part = O.partition(Q1, K1, V1, p, 0, st)
+    mapped = O.query_coords(st.qbar, part.F_Q)
+    used = np.flatnonzero(st.q_used)
+    assert np.allclose(np.sqrt((mapped[used] ** 2).mean(axis=1)), 1.0, rtol=1e-12)
+    raw = st.qbar[used] @ part.F_Q
+    assert not np.allclose(np.sqrt((raw ** 2).mean(axis=1)), 1.0, rtol=1e-3)
+    idx = O.kmeans_init_indices(p.seed, 0, 1, p.C_q, w.N)
+    again = O.kmeans(part.phiQ, idx, p.kmeans_max_iter, O.warm_centres(part.phiQ, idx, st.q_used, mapped))
+    assert np.array_equal(again.labels, part.km_Q.labels) and again.iterations == part.km_Q.iterations
