@@ -24,9 +24,10 @@
  *                       rows, restored to the original token order.
  *
  * Conventions (every entry point):
- *   - Q is [H, N_q, d], K and V are [H, N_k, d], contiguous row-major DEVICE memory in
- *     the dtype of sparsepr_params.dtype (fp32 or bf16).  Out is [H, N_q, d] in the same
- *     dtype.  d must be a multiple of 8 and at most 128.
+ *   - Q is [H, N_q, d], K and V are [H/G, N_k, d] (G = sparsepr_params.G, 1 unless
+ *     grouped-query attention), contiguous row-major DEVICE memory in the dtype of
+ *     sparsepr_params.dtype (fp32 or bf16).  Out is [H, N_q, d] in the same dtype.  d must
+ *     be a multiple of 8 and at most 128.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *     Every call except sparsepr_get_stats, sparsepr_export and sparsepr_check only
  *     enqueues work on it and never synchronises the host.
@@ -40,9 +41,10 @@
  *     SPARSEPR_ERR_SHAPE, SPARSEPR_ERR_DTYPE, SPARSEPR_ERR_WORKSPACE); a CUDA launch
  *     error returns SPARSEPR_ERR_CUDA; calls out of order return SPARSEPR_ERR_STATE.
  *     Inconsistencies found on the device (a metric with no positive eigenvalue,
- *     non-finite values) set a device error word that sparsepr_check and
- *     sparsepr_get_stats report as SPARSEPR_ERR_DEVICE_CHECK.  No call traps or aborts
- *     the CUDA context.
+ *     non-finite values, injected labels out of range, a warm state saved for other
+ *     dimensions, a pipeline wait that timed out) set a device error word that
+ *     sparsepr_check and sparsepr_get_stats report as SPARSEPR_ERR_DEVICE_CHECK.  No call
+ *     traps or aborts the CUDA context.
  */
 #ifndef SPARSEPR_H
 #define SPARSEPR_H
