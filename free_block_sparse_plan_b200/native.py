@@ -292,7 +292,7 @@ def _export_layout(p: sparsepr_params, name: str):
         "FIT_B": (f64, (H, d, d)), "FIT_P": (f64, (H, d, d)), "FIT_REFF": (i32, (H,)),
         "PROBE_DIST": (f64, (H, p.N_q)), "KBAR": (f64, (Hk, p.C_k, d)),
         "QBAR": (f64, (H, p.C_q, d)),
-        "KM_REASSIGNED": (i64, (H, 2)),
+        "KM_REASSIGNED": (i64, (2, H)),
     }[name]
 
 

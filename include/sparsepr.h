@@ -310,9 +310,11 @@ typedef enum {
   SPARSEPR_X_PROBE_DIST = 33, /* double [H,N_q] squared phi_Q distance to the group centre */
   SPARSEPR_X_KBAR = 34,       /* double [H,C_k,d] K/V group key centroids (compact ids) */
   SPARSEPR_X_QBAR = 35,       /* double [H,C_q,d] query group centroids (compact ids) */
-  SPARSEPR_X_KM_REASSIGNED = 36,/* int64 [H,2] points the tensor-core k-means re-assigned,
-                                   summed over its steps (keys, queries); the others kept
-                                   their label by the distance bounds */
+  SPARSEPR_X_KM_REASSIGNED = 36,/* int64 [2,H]: row 0 keys (by K/V head), row 1 queries:
+                                   points the tensor-core k-means listed for re-assignment,
+                                   summed over its steps, when it keeps distance bounds
+                                   (warm plans; zero otherwise); the others kept their
+                                   label by the bounds */
   SPARSEPR_X_COUNT = 37
 } sparsepr_export_what;
 
