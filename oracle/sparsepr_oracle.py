@@ -17,12 +17,14 @@ derivation, App. A.2 probe selection (Algorithm A.1), App. A.3 estimator statist
 App. B.1 key metric, App. B.2 query metric and RMS normalisation, App. B.3 routing,
 App. C implementation, App. D ablations.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   S1  evenly spaced sample rows are floor(s*N_q/M_s), s = 0..M_s-1 (all rows if M_s >= N_q)
   S2  M_K = (1/M_s) Q_s^T Q_s, the unique symmetric matrix with
       dk M_K dk^T = mean_s (q_s . dk)^2
   S3  eigenvalues normalised to unit mean over the retained r; negatives clamped to 0
-  S5  k-means assignment ties go to the lowest centre index
+  S5  k-means assignment: label = argmin_c sum_j (x_j - c_j)^2 in the direct form (the
+      sum over ascending j, one fused multiply-add per term), ties to the lowest
+      centre index; computed by the plain C routine in kmeans_direct.c
   S6  an empty cluster keeps its previous centre
   S7  k-means stops after max_iter assignment steps or when an assignment changes no label
   S8  k-means init: C rows drawn with replacement by SplitMix64 (counter-based)
@@ -62,7 +64,10 @@ a hand-worked value are pinned).
 """
 from __future__ import annotations
 
+import ctypes
 import math
+import os
+import subprocess
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional
 
@@ -178,10 +183,42 @@ class KMeansResult:
     history: List[float] = field(default_factory=list)  # objective after each update
 
 
+_C_SRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "kmeans_direct.c")
+_C_LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libkmeans_direct.so")
+_clib_handle = None
+
+
+def _clib():
+    """The direct-form assignment of ``kmeans_direct.c`` (plain C, OpenMP over rows),
+    compiled with gcc on first use when the shared object is missing or older than its
+    source."""
+    global _clib_handle
+    if _clib_handle is None:
+        if not os.path.exists(_C_LIB) or os.path.getmtime(_C_LIB) < os.path.getmtime(_C_SRC):
+            os.makedirs(os.path.dirname(_C_LIB), exist_ok=True)
+            tmp = f"{_C_LIB}.{os.getpid()}.tmp"
+            subprocess.run(["gcc", "-O3", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC",
+                            _C_SRC, "-o", tmp, "-lm"], check=True)
+            os.replace(tmp, _C_LIB)
+        lib = ctypes.CDLL(_C_LIB)
+        lib.oracle_assign_direct.restype = None
+        lib.oracle_assign_direct.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+        _clib_handle = lib
+    return _clib_handle
+
+
 def _assign(X: np.ndarray, centres: np.ndarray) -> np.ndarray:
-    # squared Euclidean distances; np.argmin returns the lowest index on ties (S5)
-    d2 = (X * X).sum(1)[:, None] - 2.0 * (X @ centres.T) + (centres * centres).sum(1)[None, :]
-    return np.argmin(d2, axis=1)
+    """S5: label = argmin_c sum_j (x_j - c_j)^2, the sum over ascending j with one fused
+    multiply-add per term, ties to the lowest centre index (computed in plain C)."""
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    CT = np.ascontiguousarray(np.asarray(centres, dtype=np.float64).T)
+    n, r = X.shape
+    k = CT.shape[1]
+    labels = np.empty(n, dtype=np.int64)
+    if n:
+        _clib().oracle_assign_direct(X.ctypes.data, CT.ctypes.data, n, k, r, labels.ctypes.data)
+    return labels
 
 
 def _update(X: np.ndarray, labels: np.ndarray, centres: np.ndarray) -> np.ndarray:
@@ -414,6 +451,14 @@ def select_probes(dist: np.ndarray, gq: Groups, M: int):
     probes = np.array(probes, dtype=np.int64)
     m_a = np.bincount(gq.compact[probes], minlength=n_groups)
     return probes, m_a
+
+
+def coverage_weights(gq: Groups, probes: np.ndarray, m_a: np.ndarray) -> np.ndarray:
+    """[R] step 4 ([P] App. A.3, whose formula was lost): probe p of query group a stands
+    for its group's rows, w_p = |G_a^Q| / m_a, so the weights of a group's probes sum to
+    the group's size."""
+    a_of = gq.compact[probes]
+    return gq.sizes[a_of].astype(np.float64) / m_a[a_of]
 
 
 @dataclass
@@ -736,8 +781,7 @@ def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] 
     cQ = part.km_Q.centres[gq.labels_used]
     dist = probe_distances(part.phiQ, cQ, gq)
     probes, m_a = select_probes(dist, gq, p.M)
-    a_of = gq.compact[probes]
-    w = gq.sizes[a_of].astype(np.float64) / m_a[a_of]  # [R] step 4: w_p = |G_a^Q| / m_a
+    w = coverage_weights(gq, probes, m_a)
     x_probe = sparse_attention(Q, K, V, gq, gk, sel, probes)
     dense_probe = dense_attention(Q, K, V, probes)
     fit = fit_residual(x_probe, dense_probe - x_probe, w, p.lam, p.r, p.estimator)

@@ -110,6 +110,33 @@ def test_kmeans_hand_worked():
     assert np.allclose(one.centres, g["centres_max_iter_1"], rtol=1e-15)
 
 
+def test_kmeans_assignment_is_the_exact_argmin_of_direct_distances():
+    # S5: label = argmin_c sum_j (x_j - c_j)^2 taken in the direct form.  With a large
+    # common offset the differences x_j - c_j are exact (Sterbenz) and the sums of their
+    # squares resolve the nearest centre, which exact rational arithmetic confirms; the
+    # expanded form |x|^2 - 2 x.c + |c|^2 loses it to cancellation (checked below, so the
+    # case has teeth).  Equal distances go to the lowest centre index.
+    from fractions import Fraction
+    rng = _rng(40)
+    off = float(2 ** 30)
+    X = off + rng.random((300, 5))
+    Cn = off + rng.random((7, 5))
+    lab = O._assign(X, Cn)
+    Xf = [[Fraction(v) for v in row] for row in X]
+    Cf = [[Fraction(v) for v in row] for row in Cn]
+    exact = []
+    for x in Xf:
+        d = [sum((a - b) ** 2 for a, b in zip(x, c)) for c in Cf]
+        exact.append(min(range(len(d)), key=lambda c: (d[c], c)))
+    assert lab.tolist() == exact
+    expanded = ((X * X).sum(1)[:, None] - 2.0 * X @ Cn.T + (Cn * Cn).sum(1)[None, :]).argmin(1)
+    assert (expanded != np.array(exact)).sum() > 10
+    # ties: two centres at the same distance from every point -> the lower index
+    Xt = np.array([[0.0, 0.0], [1.0, 1.0]])
+    Ct = np.array([[5.0, 5.0], [1.0, 0.0], [0.0, 1.0]])
+    assert O._assign(Xt, Ct).tolist() == [1, 1]
+
+
 def test_kmeans_matches_sklearn_lloyd():
     from sklearn.cluster import KMeans
     rng = _rng(3)
@@ -352,6 +379,41 @@ def test_probe_selection_hand_worked():
         probes, m_a = O.select_probes(np.array(g["dist"]), gq, c["M"])
         assert probes.tolist() == c["probes"]
         assert m_a.tolist() == c["m_a"]
+
+
+def test_probe_distances_selection_and_weights_hand_worked():
+    # [P] App. A.2 (distance of a row's query coordinates to its group's centre, then
+    # Algorithm A.1) and [R] step 4 (w_p = |G_a^Q| / m_a), on values worked out by hand.
+    g = _golden("probe_distance_example.json")
+    gq = O.compact_groups(np.array(g["labels"]), 2)
+    dist = O.probe_distances(np.array(g["phi"], dtype=np.float64),
+                             np.array(g["centres"], dtype=np.float64), gq)
+    assert dist.tolist() == g["dist"]
+    probes, m_a = O.select_probes(dist, gq, g["M"])
+    assert probes.tolist() == g["probes"]
+    assert m_a.tolist() == g["m_a"]
+    w = O.coverage_weights(gq, probes, m_a)
+    assert np.allclose(w, g["weights"], rtol=1e-15, atol=0)
+
+
+def test_probe_weights_of_a_group_add_up_to_its_size_in_a_full_call():
+    # Each probe stands for an equal share of its group ([R] step 4): within a group the
+    # weights are equal and they add up to the group's size, so with a probe in every
+    # group they add up to N_q.  The group-major centres the call measures distances to
+    # are the member means of the final query labels in phi_Q space.
+    Q, K, V = _clustered(31, N=300)
+    res = O.sparsepr_call(Q, K, V, _small_workload_params(M=12), head=0)
+    gq = res.part.gq
+    a_of = gq.compact[res.probes]
+    for a in np.unique(a_of):
+        wa = res.weights[a_of == a]
+        assert np.all(wa == wa[0])
+        assert abs(wa.sum() - gq.sizes[a]) <= 1e-12 * gq.sizes[a]
+    for a in range(gq.sizes.size):
+        mem = gq.compact == a
+        c = res.part.phiQ[mem].mean(axis=0)
+        d = ((res.part.phiQ[mem] - c) ** 2).sum(axis=1)
+        assert np.allclose(res.probe_dist[mem], d, rtol=1e-12, atol=1e-14)
 
 
 def test_probe_selection_many_groups_takes_nearest_of_largest():
