@@ -430,6 +430,23 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
   return launch_dense_attention(m, Q, K, V, Out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* words[2] = {nullptr, nullptr};
+  SPR_TRY(dense_error_address(&words[0]));
+  SPR_TRY(noalloc_error_address(&words[1]));
+  int v[2] = {0, 0};
+  SPR_CUDA_OK(cudaStreamSynchronize(st));
+  for (int k = 0; k < 2; ++k) {
+    SPR_CUDA_OK(cudaMemcpyAsync(&v[k], words[k], sizeof(int), cudaMemcpyDeviceToHost, st));
+    SPR_CUDA_OK(cudaMemsetAsync(words[k], 0, sizeof(int), st));
+  }
+  SPR_CUDA_OK(cudaStreamSynchronize(st));
+  const int e = v[0] | v[1];
+  if (device_error) *device_error = e;
+  return e ? SPARSEPR_ERR_DEVICE_CHECK : SPARSEPR_OK;
+}
+
 sparsepr_status sparsepr_check(sparsepr_plan_t plan, void* stream, int32_t* device_error) {
   if (!plan) return SPARSEPR_ERR_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

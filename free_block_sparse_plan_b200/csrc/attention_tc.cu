@@ -47,7 +47,8 @@ constexpr int kPolyPairs = 4;                     // of every 16 column pairs: e
 
 enum Mode { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
-// Error word of the workspace-free dense entry point.
+// Error word of sparsepr_dense_attention (no plan, no workspace): sticky until
+// sparsepr_dense_check reads and clears it.
 __device__ int g_dense_err;
 
 struct TcArgs {
@@ -551,6 +552,11 @@ sparsepr_status with_tc_d(int d, F f) {
 
 }  // namespace
 
+sparsepr_status dense_error_address(int** out) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_dense_err) == cudaSuccess ? SPARSEPR_OK
+                                                                                          : SPARSEPR_ERR_CUDA;
+}
+
 bool tc_engine_applies(int dtype, int d, int engine) {
   return engine == SPARSEPR_ENGINE_AUTO && dtype == SPARSEPR_BF16 && (d == 64 || d == 128);
 }
@@ -599,7 +605,10 @@ sparsepr_status launch_dense_attention_tc(const Dims& m, const void* Q, const vo
   a.V = reinterpret_cast<const __nv_bfloat16*>(V);
   a.out = Out;
   a.err = err;
-  if (!a.err) SPR_CUDA_OK(cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_dense_err));
+  if (!a.err) {
+    const sparsepr_status s = dense_error_address(&a.err);
+    if (s != SPARSEPR_OK) return s;
+  }
   return with_tc_d(m.d, [&](auto DD) { return launch_tc<decltype(DD)::value>(a, dim3(cdiv(m.Nq, kItemRows), m.H), st); });
 }
 

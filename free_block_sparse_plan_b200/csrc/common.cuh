@@ -281,5 +281,9 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
                              int r, int it, int* lab, int* kmstate, int* err, bool bounds, cudaStream_t st);
 sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void* K,
                                        const void* V, void* Out, cudaStream_t st);
+// Device addresses of the error words of the plan-free entry points on the current
+// device: sparsepr_dense_attention's, and the sticky word of sparsepr_dense_rows_noalloc.
+sparsepr_status dense_error_address(int** out);
+sparsepr_status noalloc_error_address(int** out);
 
 }  // namespace spr

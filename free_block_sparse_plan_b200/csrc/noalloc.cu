@@ -10,8 +10,11 @@
 //
 // The array is shared by all calls: two calls whose work overlaps on the GPU (different
 // streams, or different host threads) race on it and must be serialised by the caller.
-// Every scratch element a call reads was written earlier in the same call, so nothing
-// has to start at zero.
+// Its first 256 bytes hold two error words: the call's own (cleared by every call before
+// its first kernel, with a memset that allocates nothing) and a sticky copy that keeps
+// every bit until sparsepr_dense_check reads and clears it.  Every other scratch element
+// a call reads was written earlier in the same call.  If a pipeline wait of the attention
+// kernel timed out, that call's output rows are NaN rather than stale partials.
 #include <mutex>
 
 #include "common.cuh"
@@ -56,10 +59,14 @@ __global__ void copy_rows_kernel(const int32_t* rows, int nrows, int Nq, int* ds
 }
 
 // Merges the split-key partials of each row and writes it in the input dtype:
-// out = sum_s e^{m_s - m} O_s / sum_s e^{m_s - m} l_s.
-__global__ void combine_rows_kernel(Dims m, const float* Opart, const float* MLpart, void* Out) {
+// out = sum_s e^{m_s - m} O_s / sum_s e^{m_s - m} l_s.  `err` is the call's error word
+// (err[0]) and the sticky word (err[1]): if the attention kernel set err[0] the partials
+// are incomplete and the row is written as NaN; a non-finite result sets kErrNonFinite.
+// Every bit found is also ORed into the sticky word.
+__global__ void combine_rows_kernel(Dims m, const float* Opart, const float* MLpart, void* Out, int* err) {
   const int p = blockIdx.x, h = blockIdx.y, j = threadIdx.x;
   const long long slot0 = ((long long)h * m.M + p) * m.nsplit;
+  const int call_err = *reinterpret_cast<volatile int*>(err);
   float mx = -INFINITY;
   for (int s = 0; s < m.nsplit; ++s) mx = fmaxf(mx, MLpart[2 * (slot0 + s)]);
   float l = 0.0f, acc = 0.0f;
@@ -68,10 +75,25 @@ __global__ void combine_rows_kernel(Dims m, const float* Opart, const float* MLp
     l += w * MLpart[2 * (slot0 + s) + 1];
     if (j < m.d) acc += w * Opart[(slot0 + s) * m.d + j];
   }
-  if (j < m.d) store_from_float(Out, ((long long)h * m.M + p) * m.d + j, acc / l, m.dtype);
+  if (j < m.d) {
+    float v = acc / l;
+    int bits = call_err;
+    if (!isfinite(v)) bits |= kErrNonFinite;
+    if (call_err) v = __int_as_float(0x7fc00000);     // NaN: the partials are incomplete
+    if (bits) atomicOr(err + 1, bits);
+    store_from_float(Out, ((long long)h * m.M + p) * m.d + j, v, m.dtype);
+  }
 }
 
 }  // namespace
+
+sparsepr_status noalloc_error_address(int** out) {
+  void* base = nullptr;
+  const sparsepr_status s = scratch_address(&base);
+  if (s != SPARSEPR_OK) return s;
+  *out = reinterpret_cast<int*>(base) + 1;             // the sticky word
+  return SPARSEPR_OK;
+}
 
 size_t noalloc_rows_scratch_bytes(int H, int nrows, int Nk, int d) {
   const size_t nsplit = (size_t)cdiv(Nk, kProbeSplit);
@@ -97,6 +119,7 @@ extern "C" sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* pa
   if (params->engine != SPARSEPR_ENGINE_AUTO && params->engine != SPARSEPR_ENGINE_SIMT) return SPARSEPR_ERR_ARG;
   if (nrows < 1 || nrows > kMaxM) return SPARSEPR_ERR_ARG;
   if (params->G < 0 || (params->G > 1 && params->H % params->G != 0)) return SPARSEPR_ERR_SHAPE;
+  if (params->H > 65535) return SPARSEPR_ERR_SHAPE;      // heads are the grid's y dimension
   if (noalloc_rows_scratch_bytes(params->H, nrows, params->N_k, params->d) > kNoAllocScratchBytes)
     return SPARSEPR_ERR_WORKSPACE;
   void* base = nullptr;
@@ -120,12 +143,13 @@ extern "C" sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* pa
   c += align256((size_t)p.dm.H * nrows * p.dm.nsplit * p.dm.d * sizeof(float));
   p.b.MLpart = reinterpret_cast<float*>(c);
 
+  SPR_CUDA_OK(cudaMemsetAsync(p.b.err, 0, sizeof(int), st));   // this call's word only
   copy_rows_kernel<<<dim3(cdiv(nrows, 128), p.dm.H), 128, 0, st>>>(rows, nrows, params->N_q, p.b.probes);
   SPR_LAUNCH_OK();
   s = tc_engine_applies(p.dm.dtype, p.dm.d, p.dm.engine) ? launch_probe_attention_tc(p, st)
                                                          : launch_probe_attention_simt(p, st);
   if (s != SPARSEPR_OK) return s;
-  combine_rows_kernel<<<dim3(nrows, p.dm.H), kMaxD, 0, st>>>(p.dm, p.b.Opart, p.b.MLpart, Out);
+  combine_rows_kernel<<<dim3(nrows, p.dm.H), kMaxD, 0, st>>>(p.dm, p.b.Opart, p.b.MLpart, Out, p.b.err);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

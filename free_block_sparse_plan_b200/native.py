@@ -47,6 +47,7 @@ SYMBOLS = [
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
     "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
     "sparsepr_launch_count", "sparsepr_state_size", "sparsepr_save_state", "sparsepr_plan_warm",
+    "sparsepr_dense_check",
 ]
 
 
@@ -100,6 +101,7 @@ def lib():
             "sparsepr_dense_attention": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p,
                                                    c_void_p]),
             "sparsepr_check": (c_int32, [c_void_p, c_void_p, POINTER(c_int32)]),
+            "sparsepr_dense_check": (c_int32, [c_void_p, POINTER(c_int32)]),
             "sparsepr_get_stats": (c_int32, [c_void_p, c_void_p, POINTER(sparsepr_stats)]),
             "sparsepr_export_size": (c_int32, [c_void_p, c_int32, POINTER(c_size_t)]),
             "sparsepr_export": (c_int32, [c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
@@ -256,6 +258,16 @@ def sparsepr_dense_rows_noalloc(params, Q, K, V, rows, nrows, Out, stream):
                                              stream), "sparsepr_dense_rows_noalloc")
 
 
+def sparsepr_dense_check(stream=None) -> int:
+    """Reads and clears the error words of the plan-free entry points (dense attention and
+    the workspace-free rows); returns the word (0 = none)."""
+    e = c_int32(0)
+    st = lib().sparsepr_dense_check(stream, ctypes.byref(e))
+    if st not in (SPARSEPR_OK, SPARSEPR_ERR_DEVICE_CHECK):
+        raise SparsePRError(st, "sparsepr_dense_check")
+    return int(e.value)
+
+
 # ----------------------------------------------------------------------------------
 # Torch convenience layer (still marshalling only)
 
@@ -396,7 +408,8 @@ def dense_attention(Q, K, V, out=None, engine=SPARSEPR_ENGINE_AUTO, stream=None)
     import torch
     H, Nq, d = Q.shape
     dt = SPARSEPR_BF16 if Q.dtype == torch.bfloat16 else SPARSEPR_F32
-    p = make_params(H, Nq, K.shape[1], d, dt, 1, 1, 1, 1, 1, 1, 0, 0.0, 1.0, engine=engine)
+    G = H // K.shape[0]                  # query heads per K/V head
+    p = make_params(H, Nq, K.shape[1], d, dt, 1, 1, 1, 1, 1, 1, 0, 0.0, 1.0, engine=engine, G=G)
     if out is None:
         out = torch.empty_like(Q)
     sparsepr_dense_attention(p, _ptr(Q), _ptr(K), _ptr(V), _ptr(out), _stream(stream))

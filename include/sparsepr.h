@@ -236,8 +236,10 @@ sparsepr_status sparsepr_forward(const sparsepr_params* params, const void* Q, c
                                  size_t workspace_bytes, void* stream);
 
 /* Dense attention softmax(Q K^T / sqrt(d)) V for all rows through the same attention
- * engine (every key selected).  Only H, N_q, N_k, d, dtype and engine of params are read.
- * Needs no workspace.  Asynchronous. */
+ * engine (every key selected).  Only H, N_q, N_k, d, dtype, engine and G of params are
+ * read (K and V are [H/G, N_k, d] when G > 1).  Needs no workspace.  Asynchronous.  A
+ * pipeline wait of the tensor-core engine that timed out (its work abandoned, part of Out
+ * unwritten) sets a sticky per-device error word that sparsepr_dense_check reports. */
 sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const void* Q,
                                          const void* K, const void* V, void* Out,
                                          void* stream);
@@ -248,22 +250,35 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
  * memory around the call -- code whose device memory is owned by another allocator (a
  * framework's caching pool that has reserved the GPU) and latency-critical loops that
  * must not pay the implicit device synchronisation of cudaMalloc/cudaFree.
- *   Q [H,N_q,d], K, V [H,N_k,d]: device, params dtype; only H, N_q, N_k, d, dtype and
- *   engine of params are read.  rows: device int32 [nrows], 1 <= nrows <= 128, indices
- *   into [0,N_q) (out-of-range indices are clamped, never read outside Q).  Out: device
- *   [H,nrows,d], params dtype: softmax(q K^T / sqrt(d)) V for each requested row.
+ *   Q [H,N_q,d], K, V [H/G,N_k,d]: device, params dtype; only H, N_q, N_k, d, dtype,
+ *   engine and G of params are read (G = query heads per K/V head, 0 or 1 = none; H must
+ *   be a multiple of G and at most 65535).  rows: device int32 [nrows], 1 <= nrows <= 128,
+ *   indices into [0,N_q) (an index below 0 reads row 0 and one at or above N_q reads row
+ *   N_q-1, never outside Q).  Out: device [H,nrows,d], params dtype:
+ *   softmax(q K^T / sqrt(d)) V for each requested row.
  * Work space is a fixed 16 MiB device array inside the library, held on every GPU that
  * loads it until the process exits; a call needing more (about
  * H * nrows * ceil(N_k/4096) * (d+2) * 4 bytes) returns SPARSEPR_ERR_WORKSPACE before
  * launching anything.  The first call on a device looks up that array's address (with
  * that device current), so make it before any stream capture.  All calls share the
  * array: calls whose work overlaps on the GPU race and must be serialised by the caller.
- * Asynchronous on `stream`; calls no allocator.
+ * A call whose attention kernel timed out on a pipeline wait writes NaN rows, and a
+ * non-finite result row is reported too: both set bits of a sticky per-device word that
+ * sparsepr_dense_check reads.  Asynchronous on `stream`; calls no allocator.
  */
 sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* params, const void* Q,
                                             const void* K, const void* V,
                                             const int32_t* rows, int32_t nrows, void* Out,
                                             void* stream);
+
+/* The paper has no counterpart: error reporting of the two plan-free entry points.
+ * Synchronises `stream`, then reads and clears, on the current device, the error words of
+ * sparsepr_dense_attention and sparsepr_dense_rows_noalloc (bits as for a plan: 4 a
+ * non-finite output row, 32 a pipeline wait that timed out).  Returns SPARSEPR_OK when
+ * both were zero, else SPARSEPR_ERR_DEVICE_CHECK with their OR in *device_error (when
+ * non-NULL).  The words collect every call since the last check; work still running on
+ * other streams may set them after the read.  Allocates nothing. */
+sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error);
 
 /* Synchronises `stream` and reports the device error word: SPARSEPR_OK or
  * SPARSEPR_ERR_DEVICE_CHECK (with the word in *device_error when non-NULL). */

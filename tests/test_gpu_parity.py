@@ -62,13 +62,21 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def tie_ambiguous_probes(res: O.CallResult, gpu_probes: np.ndarray, tol=1e-5) -> bool:
-    """True if every mismatch between the GPU's and the oracle's probe list is a swap of
-    rows of one group whose oracle distances agree to `tol` relative."""
+PROBE_TIE_TOL = 1e-6      # both sides compute the probe distances in fp64
+SWAPS_EXCUSED = []        # (test id, head, positions) of every tie-ambiguous swap excused
+
+
+def tie_ambiguous_probes(res: O.CallResult, gpu_probes: np.ndarray, tol=PROBE_TIE_TOL,
+                         where="") -> bool:
+    """True if the probe lists are equal, or if every position where they differ swaps
+    two rows of one query group whose oracle distances agree to `tol` relative (the
+    radial order of Algorithm A.1 is then decided by rounding).  Each excused swap is
+    recorded in SWAPS_EXCUSED and printed."""
     if np.array_equal(gpu_probes, res.probes):
         return True
     comp = res.part.gq.compact
-    for g, o in zip(gpu_probes, res.probes):
+    swaps = []
+    for pos, (g, o) in enumerate(zip(gpu_probes, res.probes)):
         if g == o:
             continue
         if comp[g] != comp[o]:
@@ -76,6 +84,9 @@ def tie_ambiguous_probes(res: O.CallResult, gpu_probes: np.ndarray, tol=1e-5) ->
         dg, do = res.probe_dist[g], res.probe_dist[o]
         if abs(dg - do) > tol * max(abs(dg), abs(do), 1e-30):
             return False
+        swaps.append(pos)
+    SWAPS_EXCUSED.append((where, swaps))
+    print(f"tie-ambiguous probe swaps excused {where}: positions {swaps}")
     return True
 
 
@@ -95,7 +106,8 @@ def check_injected_head(plan, out_h, res: O.CallResult, h, w, exact_probes=True)
         assert np.array_equal(ex["CELL_IDS"][h][a][:sel.size], sel), a
     assert int(ex["PAIRS"][h]) == res.pairs_route
     if exact_probes:
-        assert tie_ambiguous_probes(res, ex["PROBES"][h]), (ex["PROBES"][h], res.probes)
+        assert tie_ambiguous_probes(res, ex["PROBES"][h], where=f"{w.name} head {h}"), \
+            (ex["PROBES"][h], res.probes)
         if np.array_equal(ex["PROBES"][h], res.probes):
             assert np.array_equal(ex["PROBE_COUNT"][h][:gq.sizes.size], res.m_a)
     err = rel(out_h[res.rows], res.out)
@@ -163,6 +175,19 @@ def test_tiny_injected_stagewise():
     assert rel(plan.export("FIT_MU_X")[0], res.fit.mu_x) < 1e-5
     assert rel(plan.export("FIT_S")[0], res.fit.s) < 1e-5
     assert int(plan.export("FIT_REFF")[0]) == res.fit.r_eff
+    # the ridge B and the projector P element by element: the oracle's fit ([P] S4.2,
+    # App. D.2) run on the GPU's own probe outputs, so only the fit stage is compared
+    assert np.array_equal(plan.export("PROBES")[0], res.probes)
+    x_gpu = osp_rows[res.probes]
+    R_gpu = plan.export("ODENSE_PROBE")[0].astype(np.float64) - x_gpu
+    fit = O.fit_residual(x_gpu.astype(np.float64), R_gpu, res.weights, w.lam, w.r)
+    assert rel(plan.export("FIT_MU_X")[0], fit.mu_x) < 1e-12
+    assert rel(plan.export("FIT_MU_R")[0], fit.mu_R) < 1e-12
+    assert rel(plan.export("FIT_S")[0], fit.s) < 1e-12
+    assert rel(plan.export("FIT_B")[0], fit.B) < 1e-8
+    sig = fit.sigma
+    assert sig[w.r - 1] > (1 + 1e-6) * sig[w.r]          # no singular-value tie at r
+    assert np.abs(plan.export("FIT_P")[0] - fit.P).max() < 1e-8
     check_injected_head(plan, out[0].double().cpu().numpy(), res, 0, w)
 
 
@@ -317,7 +342,7 @@ def check_injected_head_gqa(plan, out_h, res, h, w):
     for a, sel in enumerate(res.sel):
         assert cc[a] == sel.size and np.array_equal(ci[a][:sel.size], sel), a
     assert int(plan.export("PAIRS")[h]) == res.pairs_route
-    assert tie_ambiguous_probes(res, plan.export("PROBES")[h])
+    assert tie_ambiguous_probes(res, plan.export("PROBES")[h], where=f"{w.name} head {h} (GQA)")
     assert rel(out_h[res.rows], res.out) < TOL[w.dtype]
 
 
