@@ -1,7 +1,9 @@
 """Benchmark of one SparsePR attention call (plan + attend + probe_fit + correct) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid|wan|hunyuan|tiny]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan|mid|hunyuan|tiny]
+                    [--impl ours|reference] [--sweep]
+
+The default workload is the Wan-like call (40 heads x 75600 tokens x d=128, bf16, rho*=22%).
 
 A step is one whole call over all heads of the workload with inputs resident in HBM.
 The headline value is executed-pair TFLOP/s of the call, 4 d (routed + probe pairs) /
@@ -194,6 +196,98 @@ def workload_config(w):
             "l2": "flushed between timed calls (256 MiB write)"}
 
 
+def accuracy_vs_dense(plan, out, dense_out, w, nrows=2048):
+    """Context, not a gate ([Site] Table 2, [Paper] App. D.2): per-query relative L2 error
+    ||o_i - o_dense_i|| / ||o_dense_i|| of the corrected output against this library's
+    dense attention, on `nrows` evenly spaced rows per head, over the unprobed rows (probe
+    rows carry their dense rows by construction): mean and 99th percentile.  The sparse
+    output before correction is reported beside it when its export is small."""
+    import numpy as np
+    import torch
+    rows = np.unique(np.linspace(0, w.N - 1, nrows).astype(np.int64))
+    probes = plan.export("PROBES")
+    keep = np.ones((w.H, rows.size), dtype=bool)
+    for h in range(w.H):
+        keep[h] = ~np.isin(rows, probes[h])
+    ridx = torch.tensor(rows, device=out.device)
+    ref = dense_out[:, ridx].double()
+
+    def per_row(o):
+        e = (o.double() - ref).norm(dim=-1) / ref.norm(dim=-1).clamp_min(1e-300)
+        e = e.cpu().numpy()[keep]
+        return {"mean": float(e.mean()), "p99": float(np.percentile(e, 99))}
+
+    res = {"reference": "this library's dense attention (bf16 output)", "rows_per_head": int(rows.size),
+           "corrected": per_row(out[:, ridx])}
+    if w.H * w.N * w.d * 4 <= (512 << 20):
+        osp = plan.export("OSP")
+        perm = plan.export("PERM_Q")
+        orig = np.empty_like(osp)
+        for h in range(w.H):
+            orig[h][perm[h]] = osp[h]
+        res["sparse_uncorrected"] = per_row(torch.from_numpy(orig[:, rows]).to(out.device))
+    return res
+
+
+def run_sweep(args, w):
+    """The operating-point sweep on the workload's shapes and data ([Paper] App. D.2 /
+    S4.3 budgets): target density x probe budget, r and lambda fixed.  Per point: ms per
+    call (median of --steps timed calls, L2 flushed between them), realised rho_route and
+    rho_exec, executed-pair TFLOP/s, the per-query error against this library's dense
+    attention (mean / p99 over unprobed rows, 2048 rows per head), and the relative
+    Frobenius error of head 0 against the fp64 oracle on 2048 evenly spaced rows (the GPU
+    running its own k-means; the oracle's partition does not depend on rho* or M)."""
+    import numpy as np
+    import torch
+    from free_block_sparse_plan_b200 import native as N
+    from free_block_sparse_plan_b200 import workloads as W
+    from oracle import sparsepr_oracle as O
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Q, K, V = W.make_inputs_torch(w, device=dev)
+    out = torch.empty_like(Q)
+    dense_out = N.dense_attention(Q, K, V)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    rows = np.unique(np.linspace(0, w.N - 1, 2048).astype(np.int64))
+    q0, k0, v0 = W.make_head(w, 0)
+    part0 = O.partition(q0, k0, v0, O.Params.from_dict(w.params()), 0)
+    points = []
+    for pw in W.sweep_points(w):
+        params = N.params_from_dict(pw.params())
+        ws = torch.empty(N.sparsepr_workspace_size(params), dtype=torch.uint8, device=dev)
+        for _ in range(max(1, args.warmup)):
+            N.forward(params, Q, K, V, out=out, workspace=ws)
+        ms = []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            N.forward(params, Q, K, V, out=out, workspace=ws)
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        plan = N.Plan(params, Q, K, V, workspace=ws)
+        plan.attend()
+        plan.probe_fit()
+        plan.correct(out)
+        st = plan.stats()
+        acc = accuracy_vs_dense(plan, out, dense_out, pw)
+        ref = O.sparsepr_call(q0, k0, v0, O.Params.from_dict(pw.params()), head=0, rows=rows, part=part0)
+        got = out[0, torch.tensor(rows, device=dev)].double().cpu().numpy()
+        err0 = float(np.linalg.norm(got - ref.out) / np.linalg.norm(ref.out))
+        m = float(np.median(ms))
+        points.append({"rho_target": pw.rho, "M": pw.M, "ms_per_call": m,
+                       "rho_route": st["rho_route"], "rho_exec": st["rho_exec"],
+                       "oracle_rho_exec_head0": ref.rho_exec,
+                       "tflops": 4.0 * w.d * st["pairs_exec"] / (m * 1e-3) / 1e12,
+                       "err_vs_dense": acc["corrected"], "rel_err_vs_oracle_head0": err0,
+                       "device_error": st["device_error"]})
+        del plan, ws
+    print(json.dumps({"mode": "sweep", "workload": w.name, "steps": args.steps,
+                      "warmup": args.warmup, "r": w.r, "lambda": w.lam, "points": points}), flush=True)
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -201,16 +295,22 @@ def run_reference(args, w):
     times, flops = [], []
     from free_block_sparse_plan_b200 import workloads as W
     from oracle import sparsepr_oracle as O
+    # warm-up: the oracle has no cache or compiler to warm beyond loading its libraries,
+    # so the untimed steps run the small fp32 case (about 0.2 s each)
+    tiny = W.TINY
+    pt = O.Params.from_dict(tiny.params())
+    qt, kt, vt = W.make_head(tiny, 0)
+    for _ in range(args.warmup):
+        O.sparsepr_call(qt, kt, vt, pt, head=0)
     p = O.Params.from_dict(w.params())
-    for i in range(args.warmup + args.steps):
+    for i in range(args.steps):
         h = i % w.H
         q, k, v = W.make_head(w, h)
         t0 = time.perf_counter()
         res = O.sparsepr_call(q, k, v, p, head=h)
         dt = time.perf_counter() - t0
-        if i >= args.warmup:
-            times.append(dt)
-            flops.append(4.0 * w.d * res.pairs_exec)
+        times.append(dt)
+        flops.append(4.0 * w.d * res.pairs_exec)
     value = sum(flops) / sum(times) / 1e12
     try:
         cores = len(os.sched_getaffinity(0))
@@ -223,7 +323,10 @@ def run_reference(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one head of {w.H} per step (heads 0..), full fp64 call"},
+                         "sample": f"one head of {w.H} per timed step (heads 0..{min(args.steps, w.H) - 1}), "
+                                   f"full fp64 call (partition, routing, sparse attention of all "
+                                   f"{w.N} rows, probes, fit, correction); warm-up steps run the "
+                                   f"{W.TINY.name} call"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -238,12 +341,14 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--workload", default="wan")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling cases)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-warm", action="store_true", help="skip the warm-start (second call) line")
+    ap.add_argument("--sweep", action="store_true",
+                    help="operating-point sweep (target density x probe budget) on one GPU")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many calls and exit (for an external profiler; no timing)")
     args = ap.parse_args()
@@ -254,6 +359,9 @@ def main():
         w = w.with_(H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.sweep:
+        run_sweep(args, w)
         return
 
     import numpy as np
@@ -341,6 +449,15 @@ def main():
     attend_ms = float(np.median(stage[:, 1]))
     attend_tflops = 4.0 * w.d * st["pairs_route"] / (attend_ms * 1e-3) / 1e12
     dense_med = float(np.median(dense_ms))
+    dense_err = N.sparsepr_dense_check()          # a timed-out dense pipeline would show here
+    # accuracy against dense, before the e2e and warm-start legs reuse `out` and the
+    # workspace (the last timed call left its output in `out`, its plan in `ws`)
+    accuracy = None
+    if world == 1:
+        try:
+            accuracy = accuracy_vs_dense(plan, out, dense_out, w)
+        except Exception as e:                      # context only: never stops the line
+            accuracy = {"unavailable": str(e)[:200]}
 
     # end to end through the public call with host buffers: H2D inputs, call, D2H output
     e2e = None
@@ -419,7 +536,9 @@ def main():
         del Q1, K1, V1
 
     peaks, peak_kind = load_peaks()
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # the attend kernel runs for well under a second inside each call, so the burst peak
+    # (a GEMM timed alone) is its denominator, not the seconds-long sustained one
+    peak = peaks["bf16_tflops"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -431,13 +550,15 @@ def main():
                       "probe_fit": float(np.median(stage[:, 2])),
                       "correct": float(np.median(stage[:, 3]))},
         "dense_ms": dense_med, "speedup_vs_dense": dense_med / ms,
+        "dense_device_error": dense_err,
         "rho_route": st["rho_route"], "rho_exec": st["rho_exec"],
         "kmeans_iters": [st["kmeans_iters_k_max"], st["kmeans_iters_q_max"]],
         "roofline": {"kernel": "sparse attention (attend)", "bound": "tensor",
                      "achieved": attend_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attend_tflops / peak,
                      "traffic": measured_traffic("attention_tc.cu", w),
-                     "peak_source": f"{peak_kind} bf16_tflops_sustained"},
+                     "peak_source": f"{peak_kind} bf16_tflops (burst; the attend kernel runs "
+                                    f"{attend_ms:.2f} ms inside a {ms:.2f} ms call)"},
         "pct_bf16_peak_call": value / peak,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
@@ -450,6 +571,16 @@ def main():
         # the attend kernel's rate over the pairs it processes (padding included)
         padding["attend_tflops_processed"] = 4.0 * w.d * padding["processed_pairs"] / (attend_ms * 1e-3) / 1e12
     line["attention_tiles"] = padding
+    # the correction reads O_sp (fp32, group-major) and writes Out once ([Review] step 5):
+    # its algorithmic bytes over the correct stage's time, against the measured copy peak
+    corr_ms = float(np.median(stage[:, 3]))
+    corr_bytes = float(w.H) * w.N * w.d * (4 + (2 if w.dtype == "bf16" else 4))
+    line["hbm_stages"] = {"correct": {"bytes": corr_bytes, "ms": corr_ms,
+                                      "gbs": corr_bytes / (corr_ms * 1e-3) / 1e9,
+                                      "frac": corr_bytes / (corr_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                      "peak_source": f"{peak_kind} hbm_gbs"}}
+    if accuracy is not None:
+        line["accuracy_vs_dense"] = accuracy
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w)
     if world > 1:
