@@ -35,6 +35,8 @@ Readings where the pages are silent:
       ohat_a^(-b) = sum_{c != b} pi_ac vbar_c / (1 - pi_ab),
       score_ab = pi_ab * ||vbar_b - ohat_a^(-b)||_2
   S12 score ties ranked by ascending KV group id
+  S13 the calibrated budget (optional): the common integer budget beta in [1, N_k] whose
+      prefix selection brings rho_exec nearest rho* (ties to the denser selection)
   S14 group-major order keeps ascending original index inside a group
   S16 probe distance d_i is the squared distance to the group centre in phi_Q space
   S20 r = 0 means no subspace projection (P = I)
@@ -362,6 +364,38 @@ def select_cells(S: np.ndarray, size_b: np.ndarray, beta: float) -> List[np.ndar
     return sel
 
 
+def calibrated_selection(S: np.ndarray, size_a: np.ndarray, size_b: np.ndarray, rho_target: float,
+                         M: int, N_q: int, N_k: int):
+    """S13, the calibrated budget ([P] App. D.2 speaks of a budget calibrated toward the
+    target density; [Site] Table 1's realised densities fall on both sides of it).
+
+    The prefix rule of `select_cells` with a common per-query budget beta selects, for
+    every integer beta in [1, N_k], some set of cells; the realised density
+    rho_exec(beta) = (routed pairs + M N_k) / (N_q N_k) never decreases as beta grows.
+    The calibrated budget is the beta whose selection brings rho_exec nearest rho*, i.e.
+    minimises |routed pairs - T| with T = rho* N_q N_k - M N_k (in that fp64 order);
+    between a selection below T and one above at equal distance the denser is taken, and
+    among the betas giving one selection the smallest.  Returns (beta, selection).
+    """
+    T = rho_target * N_q * N_k - M * N_k
+    C_k = S.shape[1]
+    ids = np.arange(C_k)
+    betas = np.arange(1, N_k + 1, dtype=np.int64)
+    pairs = np.zeros(betas.size, dtype=np.int64)
+    for a in range(S.shape[0]):
+        order = np.lexsort((ids, -S[a]))
+        pref = np.cumsum(size_b[order]).astype(np.int64)          # pref[-1] = N_k
+        k = np.searchsorted(pref, betas, side="left")             # first prefix >= beta
+        pairs += int(size_a[a]) * pref[k]
+    dist = np.abs(pairs.astype(np.float64) - T)
+    best = dist.min()
+    cand = np.flatnonzero(dist == best)
+    pick = cand[np.argmax(pairs[cand])]                            # the denser on a tie
+    pick = np.flatnonzero(pairs == pairs[pick])[0]                 # its smallest beta
+    beta = int(betas[pick])
+    return beta, select_cells(S, size_b, float(beta))
+
+
 def executed_pairs(size_a: np.ndarray, size_b: np.ndarray, sel: List[np.ndarray]) -> int:
     """Routed query-key interactions: each selected cell costs |G_a^Q| |G_b^KV| ([P] S2)."""
     return int(sum(int(size_a[a]) * int(size_b[s].sum()) for a, s in enumerate(sel)))
@@ -380,6 +414,16 @@ def group_major_permutation(compact: np.ndarray, n_groups: int):
 
 # ----------------------------------------------------------------------------------
 # Attention ([P] S2: dense attention and renormalised hard drop)
+
+def attention_probs(q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """Dense attention weights softmax(tau q K^T) of rows q over every key ([P] S2),
+    tau = 1/sqrt(d): the matrix whose rows the O1 support densities of [P] S3 measure."""
+    tau = 1.0 / math.sqrt(q.shape[1])
+    logits = tau * (q @ K.T)
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    return p / p.sum(axis=1, keepdims=True)
+
 
 def attention_rows(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
     """softmax(tau q K^T) V for rows q, with tau = 1/sqrt(d) ([P] S4.1: the common 1/sqrt(d)
@@ -474,6 +518,7 @@ class Fit:
 
 ESTIMATORS = ("ridge", "mean", "scalar", "diagonal")   # codes 0..3 of the C ABI
 PARTITIONS = ("response", "semantic")                  # codes 0..1 of the C ABI
+BUDGETS = ("prefix", "calibrated")                     # codes 0..1 of the C ABI
 
 
 def fit_residual(x: np.ndarray, R: np.ndarray, w: np.ndarray, lam: float, r: int,
@@ -553,6 +598,7 @@ class Params:
     seed: int = 0
     estimator: str = "ridge"
     partition: str = "response"     # "response" (RCP) or "semantic" (the reference partition)
+    budget: str = "prefix"          # "prefix" (beta = rho*_route N_k) or "calibrated" (S13)
 
     @classmethod
     def from_dict(cls, p: Dict) -> "Params":
@@ -560,7 +606,8 @@ class Params:
                    C_k=p["C_k"], M=p["M"], r=p["r"], lam=p["lam"],
                    rho=p["target_density"], kmeans_max_iter=p["kmeans_max_iter"],
                    seed=p["seed"], estimator=ESTIMATORS[int(p.get("estimator", 0))],
-                   partition=PARTITIONS[int(p.get("partition", 0))])
+                   partition=PARTITIONS[int(p.get("partition", 0))],
+                   budget=BUDGETS[int(p.get("budget", 0))])
 
 
 @dataclass
@@ -772,8 +819,11 @@ def sparsepr_call(Q, K, V, p: Params, head: int = 0, rows: Optional[np.ndarray] 
                 else partition(Q, K, V, p, head, warm))
     gq, gk = part.gq, part.gk
     S = route_scores(part.qbar, part.kbar, part.vbar, gk.sizes, p.d)
-    beta = route_budget(p.rho, p.M, N_q, N_k)
-    sel = select_cells(S, gk.sizes, beta)
+    if p.budget == "calibrated":
+        beta, sel = calibrated_selection(S, gq.sizes, gk.sizes, p.rho, p.M, N_q, N_k)
+    else:
+        beta = route_budget(p.rho, p.M, N_q, N_k)
+        sel = select_cells(S, gk.sizes, beta)
     pairs = executed_pairs(gq.sizes, gk.sizes, sel)
     pairs_exec = pairs + p.M * N_k                       # [P] S4.3: probes add M/N_q
     permQ, offQ = group_major_permutation(gq.compact, gq.sizes.size)

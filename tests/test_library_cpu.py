@@ -72,7 +72,7 @@ def test_workspace_size_positive_and_monotone():
     ("target_density", 1.5, N.SPARSEPR_ERR_ARG), ("target_density", 0.01, N.SPARSEPR_ERR_ARG),
     ("kmeans_max_iter", 0, N.SPARSEPR_ERR_ARG), ("engine", 3, N.SPARSEPR_ERR_ARG),
     ("G", -1, N.SPARSEPR_ERR_SHAPE), ("G", 5, N.SPARSEPR_ERR_SHAPE),
-    ("partition", 2, N.SPARSEPR_ERR_ARG), ("reserved", 1, N.SPARSEPR_ERR_ARG),
+    ("partition", 2, N.SPARSEPR_ERR_ARG), ("budget", 2, N.SPARSEPR_ERR_ARG),
 ])
 def test_invalid_parameters_rejected_on_host(field, value, status):
     p = _params()
@@ -192,3 +192,36 @@ def test_bench_tile_accounting_from_plan_exports():
             raise RuntimeError("no such export")
 
     assert "unavailable" in bench.attention_tile_accounting(Broken(), W.MID, 1)
+
+
+def test_exp2_poly_meets_its_stated_error_bound():
+    # The attention softmax evaluates part of its exponentials as 2^x = 2^n * p(f) with a
+    # cubic p on [-1/2, 1/2] (tc_ptx.cuh, exp2_poly / exp2_poly2).  Its comment states a
+    # relative error of 2.4e-4, under bf16's 2^-9.  The coefficients are read from the
+    # source and the fp32 steps emulated (fused multiply-adds exactly rounded once).
+    import re
+    src = open(os.path.join(ROOT, "free_block_sparse_plan_b200", "csrc", "tc_ptx.cuh")).read()
+    body = src[src.index("float exp2_poly(float x)"):]
+    body = body[:body.index("}")]
+    coef = [float(c) for c in re.findall(r"([0-9.]+e[-+][0-9]+)f", body)]
+    assert len(coef) == 4
+    c3, c2, c1, c0 = (np.float32(c) for c in coef)
+    x = np.concatenate([np.linspace(-126.0, 8.0, 2_000_001), np.linspace(-1.0, 1.0, 200_001)])
+    x = np.maximum(x.astype(np.float32), np.float32(-126.0))
+    C = np.float32(12582912.0)
+    t = (x + C).astype(np.float32)
+    f = (x - (t - C)).astype(np.float32)
+
+    def fma(a, b, c):
+        return (a.astype(np.float64) * b.astype(np.float64) + np.float64(c)).astype(np.float32)
+
+    p = fma(np.full_like(f, c3), f, c2)
+    p = fma(p, f, c1)
+    p = fma(p, f, c0)
+    bits = (p.view(np.int32).astype(np.int64) + (t.view(np.int32).astype(np.int64) << 23)) & 0xFFFFFFFF
+    y = bits.astype(np.uint32).view(np.float32).astype(np.float64)
+    exact = np.exp2(x.astype(np.float64))
+    rel = np.abs(y - exact) / exact
+    normal = exact >= 2.0 ** -125          # results in the denormal range are not claimed
+    assert rel[normal].max() < 2.5e-4, rel[normal].max()
+    assert rel[normal].max() < 2.0 ** -9

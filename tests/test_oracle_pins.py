@@ -299,6 +299,52 @@ def test_select_cells_prefix_minimal_and_full_budget():
 
 
 # ---------------------------------------------------------------- permutation
+def test_calibrated_budget_hand_worked():
+    g = _golden("calibrated_budget_example.json")
+    S = np.array(g["scores"], dtype=np.float64)
+    sa, sb = np.array(g["sizes_q"]), np.array(g["sizes_k"])
+    for c in g["cases"]:
+        beta, sel = O.calibrated_selection(S, sa, sb, c["rho"], g["M"], g["N_q"], g["N_k"])
+        assert beta == c["beta"], c
+        assert [s.tolist() for s in sel] == c["sel"], c
+        assert O.executed_pairs(sa, sb, sel) == c["pairs"]
+
+
+def test_calibrated_budget_is_the_nearest_achievable_density():
+    # S13: among the selections of the prefix rule over every integer budget (found here
+    # by running select_cells at each beta), the calibrated one is nearest rho*; rho_exec
+    # never decreases in beta; the calibrated distance is at most the plain rule's.
+    rng = _rng(41)
+    for trial in range(6):
+        Cq, Ck = rng.integers(3, 9), rng.integers(3, 9)
+        sa = rng.integers(1, 7, Cq)
+        sb = rng.integers(1, 7, Ck)
+        S = rng.random((Cq, Ck))
+        S[0, 1] = S[0, 0]                                      # a score tie
+        N_q, N_k, M = int(sa.sum()), int(sb.sum()), 1
+        for rho in (0.2, 0.35, 0.5, 0.8):
+            if rho <= M / N_q:
+                continue
+            T = rho * N_q * N_k - M * N_k
+            pairs = [O.executed_pairs(sa, sb, O.select_cells(S, sb, float(b))) for b in range(1, N_k + 1)]
+            assert all(x <= y for x, y in zip(pairs, pairs[1:]))
+            beta, sel = O.calibrated_selection(S, sa, sb, rho, M, N_q, N_k)
+            got = O.executed_pairs(sa, sb, sel)
+            assert got == pairs[beta - 1]
+            assert abs(got - T) == min(abs(x - T) for x in pairs)
+            plain = O.executed_pairs(sa, sb, O.select_cells(S, sb, O.route_budget(rho, M, N_q, N_k)))
+            assert abs(got - T) <= abs(plain - T)
+
+
+def test_calibrated_budget_full_call_lands_near_the_target():
+    Q, K, V = _clustered(42, N=400)
+    p = _small_workload_params(rho=0.3, M=8)
+    plain = O.sparsepr_call(Q, K, V, p)
+    cal = O.sparsepr_call(Q, K, V, O.Params(**{**p.__dict__, "budget": "calibrated"}), part=plain.part)
+    assert abs(cal.rho_exec - p.rho) <= abs(plain.rho_exec - p.rho)
+    assert cal.pairs_exec == cal.pairs_route + p.M * Q.shape[0]
+
+
 def test_group_major_permutation():
     perm, off = O.group_major_permutation(np.array([2, 0, 1, 0, 2, 1]), 3)
     assert perm.tolist() == [1, 3, 2, 5, 0, 4]
@@ -766,6 +812,17 @@ def test_semantic_partition_clusters_raw_rows_and_full_density_is_dense():
     km = O.kmeans(K, O.kmeans_init_indices(p.seed, 0, 0, p.C_k, K.shape[0]), p.kmeans_max_iter)
     assert np.array_equal(res.part.km_K.labels, km.labels)
     assert np.allclose(res.part.vbar, O.group_means(V, res.part.gk), rtol=0, atol=0)
+
+
+def test_attention_probs_rows_sum_to_one_and_weigh_the_values():
+    # a one-hot V turns attention output into the weights themselves ([P] S2)
+    rng = _rng(43)
+    q, K = rng.standard_normal((5, 4)), rng.standard_normal((9, 4))
+    a = O.attention_probs(q, K)
+    assert np.allclose(a.sum(axis=1), 1.0, atol=1e-15)
+    assert np.allclose(a, O.attention_rows(q, K, np.eye(9)), atol=1e-15)
+    z = np.exp(q @ K.T / 2.0)
+    assert np.allclose(a, z / z.sum(axis=1, keepdims=True), atol=1e-15)
 
 
 def test_support_size_hand_worked():
