@@ -60,7 +60,7 @@ sparsepr_status validate(const sparsepr_params* q) {
   if (q->partition != SPARSEPR_PARTITION_RESPONSE && q->partition != SPARSEPR_PARTITION_SEMANTIC)
     return SPARSEPR_ERR_ARG;
   if (q->partition == SPARSEPR_PARTITION_SEMANTIC && q->d > kMaxR) return SPARSEPR_ERR_ARG;
-  if (q->reserved != 0) return SPARSEPR_ERR_ARG;
+  if (q->budget != SPARSEPR_BUDGET_PREFIX && q->budget != SPARSEPR_BUDGET_CALIBRATED) return SPARSEPR_ERR_ARG;
   return SPARSEPR_OK;
 }
 
@@ -80,6 +80,7 @@ Dims make_dims(const sparsepr_params* q) {
   d.nsplit = cdiv(q->N_k, kProbeSplit);
   // paper S4.3: the router reserves the probe cost; common per-query key budget
   d.beta = (q->target_density - (double)q->M / (double)q->N_q) * (double)q->N_k;
+  d.budget = q->budget;
   return d;
 }
 
@@ -127,6 +128,8 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->scores = c.take<double>(H * Cq * Ck);
   b->cellCnt = c.take<int>(H * Cq);
   b->cellIds = c.take<int>(H * Cq * Ck);
+  b->rankPref = m.budget == SPARSEPR_BUDGET_CALIBRATED ? c.take<int>(H * Cq * Ck) : nullptr;
+  b->betaH = c.take<double>(H);
   b->pairs = c.take<long long>(H);
   b->Qp = c.take<char>(H * Nq * d * es);
   b->Kp = c.take<char>(H * Nk * d * es);
@@ -179,6 +182,13 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
     b->kmSlo = c.take<__nv_bfloat16>(H * Np * 64);
   }
   b->warmCold = c.take<int>(2 * H);
+  {
+    const size_t Nm = Nk > Nq ? Nk : Nq, Cm = Ck > Cq ? Ck : Cq;
+    b->kmFx = c.take<unsigned long long>(H * Cm * 64 * 3);
+    b->kmFxCnt = c.take<int>(H * Cm);
+    b->kmChg = c.take<int4>(H * Nm);
+    b->kmChgCnt = c.take<int>(2);
+  }
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);
 }
@@ -301,6 +311,7 @@ ExportDesc export_desc(const Plan& p, int what) {
     case SPARSEPR_X_KBAR: return {b.kbar, Hk * m.Ck * d * D};
     case SPARSEPR_X_QBAR: return {b.qbar, H * m.Cq * d * D};
     case SPARSEPR_X_KM_REASSIGNED: return {b.kmReassigned, H * 2 * sizeof(long long)};
+    case SPARSEPR_X_BETA: return {b.betaH, H * D};
     default: return {nullptr, 0};
   }
 }
@@ -428,6 +439,24 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* params, const vo
   m.G = params->G > 1 ? params->G : 1;
   m.Hk = m.H / m.G;
   return launch_dense_attention(m, Q, K, V, Out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sparsepr_status sparsepr_affine_workspace_size(sparsepr_plan_t plan, size_t* bytes) {
+  if (!plan || !bytes) return SPARSEPR_ERR_ARG;
+  *bytes = affine_ws_doubles(plan->p.dm) * sizeof(double);
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_affine_fit(sparsepr_plan_t plan, const void* dense, void* workspace,
+                                    size_t workspace_bytes, double* explained, double* err,
+                                    void* stream) {
+  if (!plan || !dense || !explained || !err) return SPARSEPR_ERR_ARG;
+  if (plan->p.stage < 2) return SPARSEPR_ERR_STATE;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < affine_ws_doubles(plan->p.dm) * sizeof(double))
+    return SPARSEPR_ERR_WORKSPACE;
+  return launch_affine_fit(plan->p, dense, reinterpret_cast<double*>(workspace), explained, err,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error) {

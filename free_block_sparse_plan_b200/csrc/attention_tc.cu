@@ -43,7 +43,7 @@ constexpr int kTcThreads = 384;
 constexpr int kProducers = 96;                   // warps 8-10
 constexpr long long kWaitCycles = 2000000000LL;   // about one second: a hung pipeline
 constexpr float kRescaleLog2 = 8.0f;              // lazy rescale threshold (factor 256)
-constexpr int kPolyPairs = 4;                     // of every 16 column pairs: exp2 on the FMA pipe
+constexpr int kPolyPairs = 6;                     // of every 16 column pairs: exp2 on the FMA pipe
 
 enum Mode { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
@@ -369,6 +369,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tO = tmem + 256 + 128 * t + lane_off;
     const float sl2 = 1.4426950408889634f / sqrtf((float)d);
+    // a warp none of whose 32 rows is a query row of the item (a group's tail tile) only
+    // keeps the barrier phases: its rows read zero-filled Q, their results are not stored,
+    // and the issue slots and special-function throughput go to the warps that have rows
+    const bool idle = kTileRows * t + 32 * (warp & 3) >= nrows;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -378,11 +382,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       const uint32_t tS = tmem + 128 * buf + lane_off;
       if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + buf), sfp, g.err))) { ok = false; break; }
       tc::fence_after_sync();
+      if (idle) {
+        tc::fence_before_sync();
+        tc::mbar_arrive(BAR(bPFull0 + buf));
+        continue;
+      }
       const int valid = (j == nt - 1) ? last_valid : kTileKeys;
       const bool whole = valid == kTileKeys;           // uniform: no key column masked
       float mx = -INFINITY;
+      float rs = 0.0f;
       if (whole) {
-        // two 32-column loads per wait, four independent max chains
+        // two 32-column loads per wait, four independent three-operand max chains
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 4; c += 2) {
@@ -391,9 +401,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           tc::tmem_ld32(tS + 32 * c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 64; ++i) m4[i & 3] = fmaxf(m4[i & 3], v[i]);
+          for (int i = 0; i < 64; i += 2) m4[(i >> 1) & 3] = tc::fmax3(m4[(i >> 1) & 3], v[i], v[i + 1]);
         }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        mx = tc::fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
       } else {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -429,10 +439,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         l_run *= alpha;
         m_run = m_new;
       }
-      float rs = 0.0f;
       if (whole) {
-        // two 32-column loads per wait; four independent partial sums
-        float r4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        // two 32-column loads per wait; the scaling and the row sum two lanes per
+        // instruction (paired fp32), two independent pair sums
+        uint64_t r2[2] = {0ull, 0ull};                 // (0.0f, 0.0f) pairs
+        const uint64_t sc2 = tc::f2pack(sl2, sl2), nm2 = tc::f2pack(-m_run, -m_run);
 #pragma unroll
         for (int c = 0; c < 4; c += 2) {
           float v[64];
@@ -442,19 +453,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x0 = fmaf(v[2 * i], sl2, -m_run), x1 = fmaf(v[2 * i + 1], sl2, -m_run);
-            // a quarter of the exponentials on the FMA pipe, the rest on the SFU
+            float x0, x1;
+            tc::f2unpack(tc::fma2(tc::f2pack(v[2 * i], v[2 * i + 1]), sc2, nm2), x0, x1);
+            // kPolyPairs of every 16 pairs on the FMA pipe, the rest on the SFU
             const bool poly = (i & 15) >= 16 - kPolyPairs;
-            const float p0 = poly ? tc::exp2_poly(x0) : tc::ex2(x0);
-            const float p1 = poly ? tc::exp2_poly(x1) : tc::ex2(x1);
-            r4[i & 3] += p0 + p1;
+            float p0, p1;
+            if (poly) {
+              tc::exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = tc::ex2(x0);
+              p1 = tc::ex2(x1);
+            }
+            r2[i & 1] = tc::add2(r2[i & 1], tc::f2pack(p0, p1));
             pk[i] = tc::pack_bf16x2(p0, p1);
           }
           // P columns 16c..16c+31 lie inside S columns already read (chunks 0..c+1)
           tc::tmem_st16(tS + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(pk));
           tc::tmem_st16(tS + 16 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
         }
-        rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+        float s0, s1, s2, s3;
+        tc::f2unpack(r2[0], s0, s1);
+        tc::f2unpack(r2[1], s2, s3);
+        rs = (s0 + s1) + (s2 + s3);
       } else {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -477,8 +497,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       tc::fence_before_sync();
       tc::mbar_arrive(BAR(bPFull0 + buf));
     }
-    const bool oready = hasB ? wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err) : wait_bar(ms, BAR(bOReady), 0, g.err);
-    if (ok && __all_sync(0xffffffffu, oready)) {
+    const bool oready = idle || (hasB ? wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err)
+                                      : wait_bar(ms, BAR(bOReady), 0, g.err));
+    if (ok && !idle && __all_sync(0xffffffffu, oready)) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
       const int row = kTileRows * t + r;

@@ -33,6 +33,10 @@ struct KmView {         // one k-means instance (keys or queries) for all heads
   unsigned long long* dmax;   // [2][H][G] largest movement per 32-centre group (double bits)
   int N, C, r, nch, stage;
   int H;                // instances: query heads, or K/V heads for the key side
+  unsigned long long* fx;     // [H][C][64][3] exact member sums (three 40-bit limbs)
+  int* fxcnt;                 // [H][C] member counts
+  int4* chg;                  // label changes of the step {h*N + n, old, new, 0}
+  int* chgcnt;                // [2] their counts, slot it & 1
 };
 
 KmView view(const Plan& p, bool query) {
@@ -40,9 +44,9 @@ KmView view(const Plan& p, bool query) {
   const Dims& m = p.dm;
   if (query)
     return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, b.kmDelta, b.kmDmax,
-            m.Nq, m.Cq, m.rQ, m.nchQ, 1, m.H};
+            m.Nq, m.Cq, m.rQ, m.nchQ, 1, m.H, b.kmFx, b.kmFxCnt, b.kmChg, b.kmChgCnt};
   return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, b.kmDelta, b.kmDmax,
-          m.Nk, m.Ck, m.rK, m.nchK, 0, m.Hk};
+          m.Nk, m.Ck, m.rK, m.nchK, 0, m.Hk, b.kmFx, b.kmFxCnt, b.kmChg, b.kmChgCnt};
 }
 
 // ---------------------------------------------------------------------------------
@@ -320,9 +324,11 @@ __global__ void __launch_bounds__(128) km_assign_kernel(KmView v, int it) {
   }
   if (valid) {
     int* lp = v.lab + (long long)h * v.N + row;
-    if (*lp != bi) {
+    const int old = *lp;
+    if (old != bi) {
       *lp = bi;
       km[1 + (it & 1)] = 1;
+      v.chg[atomicAdd(v.chgcnt + (it & 1), 1)] = make_int4((int)((long long)h * v.N + row), old, bi, 0);
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) km[3] += 1;
@@ -492,6 +498,127 @@ __global__ void __launch_bounds__(kMeanSub * kMaxR) cs_mean_kernel(KmView v, int
     for (int q = 0; q < kMeanSub * kMaxR / 32; ++q) s += opart[q];
     v.obj[(long long)h * v.C + c] = s;
   }
+}
+
+// ---------------------------------------------------------------------------------
+// Exact incremental means.  Every coordinate is taken as round(x 2^80) = l2 2^80 +
+// l1 2^40 + l0, the limbs of |x| with the sign of x, |l1|, |l0| <= 2^40 (exact for
+// |x| >= 2^-28, the rounding of smaller ones is below 2^-81), and each limb of a centre's member sum is an int64 of its own, so
+// integer atomics in any order give the same sums bit for bit.  A step moves only the
+// points whose label changed: their limbs leave the old centre and join the new one.
+__device__ __forceinline__ void fx_split(double x, long long* l) {
+  const double a = fabs(x);
+  const double f2 = floor(a);
+  const double y1 = (a - f2) * 1099511627776.0;          // 2^40; a - floor(a) is exact for a >= 0
+  const double f1 = floor(y1);
+  const long long sg = x < 0.0 ? -1 : 1;                 // limbs of |x|, signed together
+  l[2] = sg * (long long)f2;
+  l[1] = sg * (long long)f1;
+  l[0] = sg * llrint((y1 - f1) * 1099511627776.0);
+}
+
+__device__ __forceinline__ double fx_value(const unsigned long long* s) {   // sum 2^-80
+  const __int128 t = ((__int128)(long long)s[2] << 80) + ((__int128)(long long)s[1] << 40) +
+                     (__int128)(long long)s[0];
+  const long long hi = (long long)(t >> 64);
+  const unsigned long long lo = (unsigned long long)t;
+  return ((double)hi * 18446744073709551616.0 + (double)lo) * 8.271806125530277e-25;
+}
+
+// The exact sums of every centre from scratch, one block per (centre, head): its members
+// in group-major order (the counting sort of this step), limbs summed in int64 (exact,
+// any order).  Used after the first assignment, where every point changed label and the
+// change log would cost one atomic per limb of every point.
+__global__ void __launch_bounds__(256) km_fx_full_kernel(KmView v, int it) {
+  __shared__ long long part[4][kMaxR][3];
+  const int h = blockIdx.y, c = blockIdx.x;
+  if (km_skip(v, h, it, false)) return;
+  const int k = threadIdx.x % kMaxR, sub = threadIdx.x / kMaxR;
+  const int* off = v.off + (long long)h * (v.C + 1);
+  const int m0 = off[c], m1 = off[c + 1];
+  const int* perm = v.perm + (long long)h * v.N;
+  const double* X = v.X + (long long)h * v.N * v.r;
+  long long acc[3] = {0, 0, 0};
+  if (k < v.r)
+    for (int mm = m0 + sub; mm < m1; mm += 4) {
+      long long l[3];
+      fx_split(X[(long long)perm[mm] * v.r + k], l);
+      acc[0] += l[0];
+      acc[1] += l[1];
+      acc[2] += l[2];
+    }
+  for (int j = 0; j < 3; ++j) part[sub][k][j] = acc[j];
+  __syncthreads();
+  if (sub == 0 && k < v.r) {
+    unsigned long long* dst = v.fx + (((long long)h * v.C + c) * 64 + k) * 3;
+    for (int j = 0; j < 3; ++j)
+      dst[j] = (unsigned long long)(part[0][k][j] + part[1][k][j] + part[2][k][j] + part[3][k][j]);
+  }
+  if (threadIdx.x == 0) {
+    v.fxcnt[(long long)h * v.C + c] = m1 - m0;
+    if (c == 0 && h == 0) v.chgcnt[(it + 1) & 1] = 0;     // the next step's log
+  }
+}
+
+// One warp per logged change: the point's limbs move from the old centre (none on the
+// first step) to the new one.
+__global__ void __launch_bounds__(256) km_fx_apply_kernel(KmView v, int it) {
+  const int n = v.chgcnt[it & 1];
+  const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) v.chgcnt[(it + 1) & 1] = 0;   // the next step's log
+  for (long long e = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < n;
+       e += ((long long)gridDim.x * blockDim.x) >> 5) {
+    const int4 c = v.chg[e];
+    const long long pi = c.x;
+    const int h = (int)(pi / v.N);
+    const double* x = v.X + pi * v.r;
+    unsigned long long* to = v.fx + ((long long)h * v.C + c.z) * 64 * 3;
+    unsigned long long* from = c.y >= 0 ? v.fx + ((long long)h * v.C + c.y) * 64 * 3 : nullptr;
+    for (int k = lane; k < v.r; k += 32) {
+      long long l[3];
+      fx_split(x[k], l);
+      for (int j = 0; j < 3; ++j) {
+        atomicAdd(to + 3 * k + j, (unsigned long long)l[j]);
+        if (from) atomicAdd(from + 3 * k + j, (unsigned long long)(-l[j]));
+      }
+    }
+    if (lane == 0) {
+      atomicAdd(v.fxcnt + (long long)h * v.C + c.z, 1);
+      if (c.y >= 0) atomicAdd(v.fxcnt + (long long)h * v.C + c.y, -1);
+    }
+  }
+}
+
+// Centres from the exact sums (S6: an empty centre stays), with the convergence flags and
+// the centre moves of cs_mean_kernel; one block of 64 threads per (centre, head).
+__global__ void __launch_bounds__(64) km_fx_mean_kernel(KmView v, int it) {
+  __shared__ double dd2[2];
+  const int h = blockIdx.y, c = blockIdx.x, k = threadIdx.x;
+  int* km = v.km + 4 * h;
+  if (km[0]) return;
+  if (!km[1 + (it & 1)]) {                  // converged: this assignment changed nothing
+    if (c == 0 && k == 0) km[0] = 1;
+    return;
+  }
+  if (c == 0 && k == 0) km[1 + ((it + 1) & 1)] = 0;   // reset the next step's flag
+  const int cnt = v.fxcnt[(long long)h * v.C + c];
+  double* cent = v.cent + ((long long)h * v.C + c) * v.r;
+  double t = 0.0, mean = 0.0;
+  if (k < v.r) {
+    mean = cnt > 0 ? fx_value(v.fx + (((long long)h * v.C + c) * 64 + k) * 3) / (double)cnt : cent[k];
+    t = cnt > 0 ? mean - cent[k] : 0.0;
+  }
+  double s = warp_sum(t * t);
+  if ((k & 31) == 0) dd2[k >> 5] = s;
+  __syncthreads();
+  if (k == 0) {
+    const double dl = sqrt(dd2[0] + dd2[1]) * (1.0 + 1e-12);
+    v.delta[(long long)h * v.C + c] = dl;
+    const int G = (v.C + 31) / 32;
+    atomicMax(v.dmax + ((long long)(it & 1) * gridDim.y + h) * G + c / 32,
+              (unsigned long long)__double_as_longlong(dl));
+  }
+  if (k < v.r && cnt > 0) cent[k] = mean;
 }
 
 sparsepr_status run_update(const Plan& p, const KmView& v, int it, bool force, cudaStream_t st) {
@@ -698,7 +825,12 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   const bool tc = km_uses_tc(p, query);
   const Buffers& b = p.b;
   const KmTcBuffers kb{b.kmXhi, b.kmXlo, b.kmShi, b.kmSlo, b.kmU, b.kmDelta, b.kmL, b.kmDmax, b.kmAidx,
-                       b.kmAcnt, b.kmReassigned + (query ? H : 0), b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt};
+                       b.kmAcnt, b.kmReassigned + (query ? H : 0), b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt,
+                       b.kmChg, b.kmChgCnt};
+  // exact sums start empty; every label starts at -1, so the first step logs every point
+  SPR_CUDA_OK(cudaMemsetAsync(b.kmFx, 0, sizeof(unsigned long long) * (size_t)H * v.C * 64 * 3, st));
+  SPR_CUDA_OK(cudaMemsetAsync(b.kmFxCnt, 0, sizeof(int) * (size_t)H * v.C, st));
+  SPR_CUDA_OK(cudaMemsetAsync(b.kmChgCnt, 0, sizeof(int) * 2, st));
   if (tc) {
     SPR_CUDA_OK(cudaMemsetAsync(b.kmCmaxb, 0, sizeof(int) * 2 * H, st));
     SPR_CUDA_OK(cudaMemsetAsync(b.kmQcnt, 0, sizeof(int) * 2, st));
@@ -719,8 +851,23 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
       else assign<64>(v, H, it, st);
       SPR_LAUNCH_OK();
     }
-    sparsepr_status s = run_update(p, v, it, false, st);
-    if (s != SPARSEPR_OK) return s;
+    if (it == 0) {
+      // every label changed: group the points (counting sort) and sum each centre's limbs
+      cs_hist_kernel<<<dim3(v.nch, H), kSortChunk, 0, st>>>(v, it, false);
+      SPR_LAUNCH_OK();
+      cs_scan_kernel<<<H, 1024, 0, st>>>(v, it, false);
+      SPR_LAUNCH_OK();
+      const size_t wsm = (size_t)(kSortChunk / 32) * v.C * sizeof(int);
+      SPR_CUDA_OK(cudaFuncSetAttribute(cs_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsm));
+      cs_scatter_kernel<<<dim3(v.nch, H), kSortChunk, wsm, st>>>(v, it, false);
+      SPR_LAUNCH_OK();
+      km_fx_full_kernel<<<dim3(v.C, H), 256, 0, st>>>(v, it);
+    } else {
+      km_fx_apply_kernel<<<8 * 148, 256, 0, st>>>(v, it);
+    }
+    SPR_LAUNCH_OK();
+    km_fx_mean_kernel<<<dim3(v.C, H), 64, 0, st>>>(v, it);
+    SPR_LAUNCH_OK();
   }
   return SPARSEPR_OK;
 }

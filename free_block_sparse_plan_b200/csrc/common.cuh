@@ -40,7 +40,8 @@ struct Dims {
   int semantic;        // semantic reference partition: coordinates = raw rows (rK = rQ = d)
   int nchK, nchQ;      // counting-sort chunks per head
   int nsplit;          // partial blocks of the exact probe attention
-  double beta;         // per-query key budget (rho - M/N_q) * N_k
+  double beta;         // per-query key budget (rho - M/N_q) * N_k of the prefix rule
+  int budget;          // sparsepr_budget
 };
 
 // Device buffers carved from the caller's workspace (see carve_workspace).
@@ -63,6 +64,8 @@ struct Buffers {
   double *kbar, *vbar, *qbar;  // compact centroids [H][C][d]
   double *scores;            // [H][Cq][Ck]
   int *cellCnt, *cellIds;    // [H][Cq], [H][Cq][Ck]
+  int *rankPref;             // calibrated budget: key counts of each score-ranked prefix [H][Cq][Ck]
+  double *betaH;             // budget each head's routing used [H]
   long long *pairs;          // [H]
   void *Qp, *Kp, *Vp;        // group-major copies [H][N][d]
   double *dist;              // [H][Nq]
@@ -95,6 +98,10 @@ struct Buffers {
   __nv_bfloat16 *kmShi, *kmSlo;  // their split coordinates, compacted [H][Npad][64]
   int *kmQcnt;               // queue lengths [2]
   int *warmCold;             // heads whose warm factor update fell back to the eigensolve [2][H]
+  unsigned long long *kmFx;  // exact member sums of each centre, three 40-bit limbs [H][Cmax][64][3]
+  int *kmFxCnt;              // member counts [H][Cmax]
+  int4 *kmChg;               // label changes of the current step {h*N + n, old, new, -} [H*Nmax]
+  int *kmChgCnt;             // their counts [2], slot it & 1
   int *err;                  // device error word
 };
 
@@ -276,6 +283,8 @@ struct KmTcBuffers {
   int* cmaxb;
   int4* queue;
   int* qcnt;
+  int4* chg;                 // label-change log (exact incremental means)
+  int* chgcnt;
 };
 sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const double* cent, int H, int N, int C,
                              int r, int it, int* lab, int* kmstate, int* err, bool bounds, cudaStream_t st);
@@ -285,5 +294,9 @@ sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void
 // device: sparsepr_dense_attention's, and the sticky word of sparsepr_dense_rows_noalloc.
 sparsepr_status dense_error_address(int** out);
 sparsepr_status noalloc_error_address(int** out);
+// O3 affine-fit diagnostic over a plan's sparse output (diagnostics.cu).
+sparsepr_status launch_affine_fit(const Plan& p, const void* dense, double* ws, double* explained,
+                                  double* err, cudaStream_t st);
+size_t affine_ws_doubles(const Dims& m);
 
 }  // namespace spr

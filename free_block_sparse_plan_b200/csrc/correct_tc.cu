@@ -2,8 +2,10 @@
 // App. D.2):  O_hat = O_sp + c + O_sp B' on every row, in the original token order (the
 // probe rows are overwritten with their exact dense rows afterwards).
 //
-// One CTA per 128 group-major rows of one head: the fp32 O_sp rows and B'^T are copied
-// into 128-byte-swizzled K-major shared memory, delta = O_sp B' comes from
+// Persistent CTAs, one per SM, each over a contiguous range of 128-row tiles (group-major
+// rows of one head): the fp32 O_sp rows (two stages, the next tile copied while the
+// current one is processed) and B'^T (once per head) sit in 128-byte-swizzled K-major
+// shared memory, delta = O_sp B' comes from
 // tcgen05.mma kind::tf32 (M=128, N=d, K=8 per instruction) into TMEM, and thread r adds
 // its row's O_sp (from the same shared-memory tile) and c, rounds to bf16 and stores the
 // row at its original position.  tf32 keeps 10 mantissa bits of each operand, so delta
@@ -36,71 +38,102 @@ __global__ void transpose_bp_kernel(const float* Bp, int d, float* BT) {
   }
 }
 
+// Persistent: one CTA per SM takes a contiguous range of (head, 128-row tile) pairs.  B'^T
+// of the current head stays in shared memory; the O_sp tiles go through two stages, the
+// next tile's rows copied while the current one is multiplied and written out.
 template <int D>
-__global__ void __launch_bounds__(128) correct_tc_kernel(Dims m, Buffers b, const float* BT,
-                                                         __nv_bfloat16* Out) {
+__global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, const float* BT,
+                                                            __nv_bfloat16* Out, int tiles_per_head,
+                                                            long long total) {
   constexpr int NP = D / 32;                          // 128-byte panels per fp32 row
   constexpr uint32_t kAPanel = kRowsC * 128, kBPanel = D * 128;
-  constexpr uint32_t kATile = NP * kAPanel;
+  constexpr uint32_t kATile = NP * kAPanel, kBTile = NP * kBPanel;
+  constexpr int CPR = D / 4;                          // 16-byte chunks per fp32 row
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t base = (raw + 1023u) & ~1023u;       // B'^T, then stage 0, then stage 1
   uint8_t* gbase = smem_raw + (base - raw);
-  unsigned long long* bar = reinterpret_cast<unsigned long long*>(gbase + kATile + NP * kBPanel);
+  unsigned long long* bar = reinterpret_cast<unsigned long long*>(gbase + kBTile + 2 * kATile);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const long long p0 = (long long)blockIdx.x * kRowsC;
+  const long long t0 = total * blockIdx.x / gridDim.x, t1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (t0 >= t1) return;
 
   if (tid == 0) tc::mbar_init(tc::smem_u32(bar), 1);
   if (warp == 0) {
     tc::tmem_alloc(tc::smem_u32(tslot), D);
     tc::tmem_relinquish();
   }
-  constexpr int CPR = D / 4;                          // 16-byte chunks per fp32 row
-  const float* Oh = b.Osp + (long long)h * m.Nq * D;
-  for (int e = tid; e < kRowsC * CPR; e += 128) {
-    const int row = e / CPR, c = e % CPR;
-    const bool ok = p0 + row < m.Nq;
-    const uint32_t dst = base + (c >> 3) * kAPanel + tc::sw128_offset(row, c & 7);
-    tc::cp_async16(dst, ok ? (const void*)(Oh + (p0 + row) * D + c * 4) : (const void*)Oh, ok ? 16u : 0u);
-  }
-  const float* Bh = BT + (long long)h * D * D;
-  for (int e = tid; e < D * CPR; e += 128) {
-    const int row = e / CPR, c = e % CPR;
-    const uint32_t dst = base + kATile + (c >> 3) * kBPanel + tc::sw128_offset(row, c & 7);
-    tc::cp_async16(dst, Bh + (long long)row * D + c * 4, 16u);
-  }
+  // rows of tile t into stage s (rows past N_q read as zeros and are not stored)
+  auto load_tile = [&](long long t, int s) {
+    const int h = (int)(t / tiles_per_head);
+    const long long p0 = (t % tiles_per_head) * kRowsC;
+    const float* Oh = b.Osp + (long long)h * m.Nq * D;
+    const uint32_t st0 = base + kBTile + (uint32_t)s * kATile;
+    for (int e = tid; e < kRowsC * CPR; e += 128) {
+      const int row = e / CPR, c = e % CPR;
+      const bool ok = p0 + row < m.Nq;
+      const uint32_t dst = st0 + (c >> 3) * kAPanel + tc::sw128_offset(row, c & 7);
+      tc::cp_async16(dst, ok ? (const void*)(Oh + (p0 + row) * D + c * 4) : (const void*)Oh, ok ? 16u : 0u);
+    }
+  };
+  auto load_bt = [&](int h) {
+    const float* Bh = BT + (long long)h * D * D;
+    for (int e = tid; e < D * CPR; e += 128) {
+      const int row = e / CPR, c = e % CPR;
+      tc::cp_async16(base + (c >> 3) * kBPanel + tc::sw128_offset(row, c & 7), Bh + (long long)row * D + c * 4, 16u);
+    }
+  };
+  load_tile(t0, 0);
   tc::cp_async_commit();
-  tc::cp_async_wait_all();
-  tc::fence_proxy_async();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
-
-  if (tid == 0) {
-    constexpr uint32_t idesc = tc::idesc_tf32_f32(kRowsC, D);
-#pragma unroll
-    for (int kk = 0; kk < D / 8; ++kk) {
-      const uint64_t ad = tc::sw128_desc(base + (kk >> 2) * kAPanel + (kk & 3) * 32, 16, 1024);
-      const uint64_t bd = tc::sw128_desc(base + kATile + (kk >> 2) * kBPanel + (kk & 3) * 32, 16, 1024);
-      tc::mma_ss_tf32(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+  int loaded = -1;
+  bool ok = true;
+  for (long long t = t0; t < t1; ++t) {
+    const int s = (int)((t - t0) & 1);
+    const int h = (int)(t / tiles_per_head);
+    if (h != loaded) {                                // a new head: its B'^T (the previous
+      load_bt(h);                                     // multiply has completed)
+      tc::cp_async_commit();
+      loaded = h;
     }
-    tc::mma_commit(tc::smem_u32(bar));
-  }
-  __syncwarp();
-  const bool ok = tc::mbar_wait(tc::smem_u32(bar), 0, kCWait);
-  if (!__all_sync(0xffffffffu, ok)) {
-    if ((tid & 31) == 0) atomicOr(b.err, kErrHang);
-  } else {
+    tc::cp_async_wait_all();                          // this tile's rows (and B'^T)
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
     tc::fence_after_sync();
-    const long long pos = p0 + tid;
+    const uint32_t st0 = base + kBTile + (uint32_t)s * kATile;
+    if (tid == 0) {
+      constexpr uint32_t idesc = tc::idesc_tf32_f32(kRowsC, D);
+#pragma unroll
+      for (int kk = 0; kk < D / 8; ++kk) {
+        const uint64_t ad = tc::sw128_desc(st0 + (kk >> 2) * kAPanel + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::sw128_desc(base + (kk >> 2) * kBPanel + (kk & 3) * 32, 16, 1024);
+        tc::mma_ss_tf32(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(tc::smem_u32(bar));
+    }
+    __syncwarp();
+    // the next tile's rows go to the other stage while this one is multiplied and stored
+    if (t + 1 < t1) load_tile(t + 1, s ^ 1);
+    tc::cp_async_commit();
+    const bool done = tc::mbar_wait(tc::smem_u32(bar), (uint32_t)((t - t0) & 1), kCWait);
+    if (!__all_sync(0xffffffffu, done)) {
+      if ((tid & 31) == 0) atomicOr(b.err, kErrHang);
+      ok = false;
+    }
+    if (!__syncthreads_and(ok)) break;                // every thread stops together
+    tc::fence_after_sync();
+    const long long pos = (t % tiles_per_head) * kRowsC + tid;
     const bool live = pos < m.Nq;
     const long long orow = live ? b.permQ[(long long)h * m.Nq + pos] : 0;
     uint4* dst = reinterpret_cast<uint4*>(Out + ((long long)h * m.Nq + orow) * D);
     const float* cv = b.cvec + (long long)h * D;
     const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint8_t* arow = gbase + kBTile + (uint32_t)s * kATile;
 #pragma unroll 1
     for (int q = 0; q < NP; ++q) {                    // 32 output columns per step
       float dl[32];
@@ -110,7 +143,7 @@ __global__ void __launch_bounds__(128) correct_tc_kernel(Dims m, Buffers b, cons
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const float4 o = *reinterpret_cast<const float4*>(gbase + q * kAPanel + tc::sw128_offset(tid, c));
+          const float4 o = *reinterpret_cast<const float4*>(arow + q * kAPanel + tc::sw128_offset(tid, c));
           const float4 cc = __ldg(reinterpret_cast<const float4*>(cv + 32 * q + 4 * c));
           pk[2 * c] = tc::pack_bf16x2(o.x + cc.x + dl[4 * c], o.y + cc.y + dl[4 * c + 1]);
           pk[2 * c + 1] = tc::pack_bf16x2(o.z + cc.z + dl[4 * c + 2], o.w + cc.w + dl[4 * c + 3]);
@@ -120,7 +153,12 @@ __global__ void __launch_bounds__(128) correct_tc_kernel(Dims m, Buffers b, cons
           dst[4 * q + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
+    // the accumulator and this stage are free once every thread has read them
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
   }
+  tc::cp_async_wait_all();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -134,10 +172,15 @@ sparsepr_status run_correct_tc(const Plan& p, void* Out, cudaStream_t st) {
   const Dims& m = p.dm;
   transpose_bp_kernel<<<dim3(cdiv(D, 32), cdiv(D, 32), m.H), dim3(32, 8), 0, st>>>(p.b.Bp, D, p.b.BpT);
   SPR_LAUNCH_OK();
-  const size_t smem = (size_t)kRowsC * D * 4 + (size_t)D * D * 4 + 64 + 1024;
+  const int tph = cdiv(m.Nq, kRowsC);
+  const long long total = (long long)tph * m.H;
+  int dev = 0, sms = 148;
+  SPR_CUDA_OK(cudaGetDevice(&dev));
+  SPR_CUDA_OK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int grid = (int)(total < sms ? total : sms);
+  const size_t smem = (size_t)D * D * 4 + 2 * (size_t)kRowsC * D * 4 + 64 + 1024;
   SPR_CUDA_OK(cudaFuncSetAttribute(correct_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  correct_tc_kernel<D><<<dim3(cdiv(m.Nq, kRowsC), m.H), 128, smem, st>>>(m, p.b, p.b.BpT,
-                                                                         static_cast<__nv_bfloat16*>(Out));
+  correct_tc_kernel<D><<<grid, 128, smem, st>>>(m, p.b, p.b.BpT, static_cast<__nv_bfloat16*>(Out), tph, total);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

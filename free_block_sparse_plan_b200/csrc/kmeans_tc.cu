@@ -72,6 +72,8 @@ struct KmArgs {
   int* km;                    // [H][4]
   int4* queue;                // ambiguous points: h * N + n, candidate slots, flags
   int* qcnt;                  // [2] queue lengths, slot it & 1
+  int4* chg;                  // label changes {h * N + n, old, new, 0}
+  int* chgcnt;                // [2] their counts, slot it & 1
   int qcap;
   const double* X;            // [H][N][r] fp64 features (fallback when the queue is full)
   const double* cent;         // [H][C][r] fp64 centres
@@ -263,8 +265,10 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
           tc::fence_after_sync();
           const uint32_t acc = tmem + 256 * s;
           const uint32_t ch = base + oChi + c * kCBytes, cl = base + oClo + c * kCBytes;
-#pragma unroll
-          for (int kk = 0; kk < kKP / 16; ++kk) {
+          // k-steps of 16 features up to r: the padding columns are zero in both operands
+          const int nks = (g.r + 15) >> 4;
+#pragma unroll 4
+          for (int kk = 0; kk < nks; ++kk) {
             const uint64_t xh = tc::sw128_desc(xa + kk * 32, 16, 1024);
             const uint64_t xl = tc::sw128_desc(xa + kXBytes + kk * 32, 16, 1024);
             const uint64_t chd = tc::sw128_desc(ch + kk * 32, 16, 1024);
@@ -338,6 +342,10 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
         if (s) ++nfull1; else ++nfull0;
         tc::fence_after_sync();
         const uint32_t acc = tmem + 256 * s + lane_off;
+        // four independent (smallest, runner-up, centre) chains, chain e over the columns
+        // e mod 4, so consecutive scores do not wait on one another; merged below
+        float x0[4] = {BIG, BIG, BIG, BIG}, x1[4] = {BIG, BIG, BIG, BIG};
+        int xc[4] = {0, 0, 0, 0};
 #pragma unroll 1
         for (int q = 0; q < g.Cw; q += 64) {
           const int cb = c * kChunk + q;
@@ -357,9 +365,9 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float a = fmaf(-2.0f, v[4 * i4 + e], cv[e]);
-              a1 = fminf(a1, fmaxf(a0, a));
-              c0 = a < a0 ? cb + 4 * i4 + e : c0;
-              a0 = fminf(a0, a);
+              x1[e] = fminf(x1[e], fmaxf(x0[e], a));
+              xc[e] = a < x0[e] ? cb + 4 * i4 + e : xc[e];
+              x0[e] = fminf(x0[e], a);
               if (B) gm[i4 >> 3] = fminf(gm[i4 >> 3], a);
             }
           }
@@ -370,6 +378,16 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
               if (gi < g.G) g.L[((long long)h * g.G + gi) * g.N + (pi - (long long)h * g.N)] = dist_floor(gm[s2], Eb, x2);
             }
           }
+        }
+        // merge the chains into the running values: the smallest score with the lowest
+        // centre index among equal ones (earlier chunks hold lower indices), and the
+        // second smallest of the union, min(max of the two smallests, both runners-up)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          a1 = fminf(fminf(a1, x1[e]), fmaxf(a0, x0[e]));
+          const bool take = x0[e] < a0 || (x0[e] == a0 && xc[e] < c0);
+          c0 = take ? xc[e] : c0;
+          a0 = fminf(a0, x0[e]);
         }
         // the bound, formed here so that the per-point loads above had the pass to land
         const float T = 4e-4f * xn * cm + 1e-5f * (xn + cm) * (xn + cm) + 1e-30f;
@@ -452,6 +470,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       if (old != best) {
         g.lab[pi] = best;
         g.km[4 * h + 1 + (g.it & 1)] = 1;
+        g.chg[atomicAdd(g.chgcnt + (g.it & 1), 1)] = make_int4((int)pi, old, best, 0);
       }
     }
   }
@@ -559,7 +578,8 @@ __global__ void __launch_bounds__(256) km_filter_kernel(const KmFilter f) {
 // distance by the full scan's formula, smallest distance with ties to the lowest index.
 __global__ void __launch_bounds__(256) km_rescore_kernel(const int4* queue, const int* qcnt, int qcap,
                                                          const double* X, const double* cent, int* lab,
-                                                         int* km, int N, int C, int r, int it) {
+                                                         int* km, int N, int C, int r, int it,
+                                                         int4* chg, int* chgcnt) {
   const int lane = threadIdx.x & 31;
   const int n = min(qcnt[it & 1], qcap);
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -590,8 +610,10 @@ __global__ void __launch_bounds__(256) km_rescore_kernel(const int4* queue, cons
       if (od < bd || (od == bd && oc < bc)) { bd = od; bc = oc; }
     }
     if (lane == 0 && lab[pi] != bc) {
+      const int old = lab[pi];
       lab[pi] = bc;
       km[4 * h + 1 + (it & 1)] = 1;
+      chg[atomicAdd(chgcnt + (it & 1), 1)] = make_int4((int)pi, old, bc, 0);
     }
   }
 }
@@ -702,6 +724,7 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   g.aidx = kb.aidx; g.acnt = kb.acnt + (it & 1) * H; g.U = kb.U; g.L = kb.L;
   g.xn = kb.xn; g.cn = kb.cn; g.cmaxb = kb.cmaxb; g.lab = lab; g.km = kmstate;
   g.queue = kb.queue; g.qcnt = kb.qcnt; g.qcap = (int)km_tc_queue_cap(H, N);
+  g.chg = kb.chg; g.chgcnt = kb.chgcnt;
   g.X = X; g.cent = cent; g.err = err;
   g.H = H; g.N = N; g.Npad = Npad; g.C = C; g.Cpad = Cpad; g.Cw = Cw; g.nch = nch; g.r = r; g.it = it;
   g.slots = slots;
@@ -712,7 +735,7 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   kern<<<grid, kKmThreads, smem, st>>>(g);
   SPR_LAUNCH_OK();
   km_rescore_kernel<<<4 * sm_count(), 256, 0, st>>>(kb.queue, kb.qcnt, g.qcap, X, cent, lab, kmstate, N, C, r,
-                                                    it);
+                                                    it, kb.chg, kb.chgcnt);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

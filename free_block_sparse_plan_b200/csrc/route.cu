@@ -68,9 +68,15 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
     stage(kb, k0);
     const int k = k0 + tk;
     if (ta < na && k < n) {
-      double s = 0.0;
-      for (int j = 0; j < d; ++j) s = fma(qa[ta * ld + j], kv[tk * ld + j], s);
-      zz[ta * n + k] = tau * s + log((double)sz[k]);
+      // four independent partial sums (d is a multiple of 8): a quarter of the latency
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      for (int j = 0; j < d; j += 4) {
+        s0 = fma(qa[ta * ld + j], kv[tk * ld + j], s0);
+        s1 = fma(qa[ta * ld + j + 1], kv[tk * ld + j + 1], s1);
+        s2 = fma(qa[ta * ld + j + 2], kv[tk * ld + j + 2], s2);
+        s3 = fma(qa[ta * ld + j + 3], kv[tk * ld + j + 3], s3);
+      }
+      zz[ta * n + k] = tau * ((s0 + s1) + (s2 + s3)) + log((double)sz[k]);
     }
   }
   __syncthreads();
@@ -149,11 +155,16 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
     if (ta < na && k < n) {
       const bool istop = k == sTop[ta];
       const double* ref = istop ? orr + ta * ld : qa + ta * ld;
-      double s = 0.0;
-      for (int j = 0; j < d; ++j) {
-        const double t = kv[tk * ld + j] - ref[j];
-        s = fma(t, t, s);
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+      for (int j = 0; j < d; j += 4) {
+        const double t0 = kv[tk * ld + j] - ref[j], t1 = kv[tk * ld + j + 1] - ref[j + 1];
+        const double t2 = kv[tk * ld + j + 2] - ref[j + 2], t3 = kv[tk * ld + j + 3] - ref[j + 3];
+        s0 = fma(t0, t0, s0);
+        s1 = fma(t1, t1, s1);
+        s2 = fma(t2, t2, s2);
+        s3 = fma(t3, t3, s3);
       }
+      const double s = (s0 + s1) + (s2 + s3);
       const double Z = sZ[ta], z = zz[ta * n + k];
       out0[(long long)ta * m.Ck + k] = istop ? (z / Z) * sqrt(s) : z * sqrt(s) / (Z - z);
     }
@@ -161,7 +172,10 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
 }
 
 // Prefix budget selection for one query group; selected ids written ascending.
-__global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
+// ranks_only (calibrated budget, first pass): only the key counts of the score-ranked
+// prefixes are written (rankPref); the selection pass then reads the head's budget from
+// betaH.  With the prefix rule the budget is m.beta, recorded in betaH.
+__global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b, int ranks_only) {
   __shared__ double key[kMaxC];
   __shared__ int id[kMaxC];
   __shared__ int flag[kMaxC];
@@ -206,7 +220,13 @@ __global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
   int tot;
   const int excl = block_exclusive_scan(mine, sh, &tot);
   const long long incl = (long long)excl + mine;
-  if (t < n && (double)incl >= m.beta && (t == 0 || (double)excl < m.beta)) cut = t + 1;
+  if (ranks_only) {
+    if (t < n) b.rankPref[((long long)h * m.Cq + a) * m.Ck + t] = (int)incl;
+    return;
+  }
+  const double beta = m.budget == SPARSEPR_BUDGET_CALIBRATED ? b.betaH[h] : m.beta;
+  if (m.budget != SPARSEPR_BUDGET_CALIBRATED && a == 0 && t == 0) b.betaH[h] = m.beta;
+  if (t < n && (double)incl >= beta && (t == 0 || (double)excl < beta)) cut = t + 1;
   __syncthreads();
   const int cnt = cut;
   for (int u = threadIdx.x; u < n; u += blockDim.x) flag[u] = 0;
@@ -225,6 +245,63 @@ __global__ void __launch_bounds__(1024) select_kernel(Dims m, Buffers b) {
     atomicAdd(reinterpret_cast<unsigned long long*>(b.pairs + h),
               (unsigned long long)(keys * (long long)b.sizeQ[(long long)h * m.Cq + a]));
   if (t == 0) b.cellCnt[(long long)h * m.Cq + a] = cnt;
+}
+
+// Routed pairs of head h under the common integer budget beta: every query group keeps
+// the shortest score-ranked prefix whose key count reaches beta (its last prefix holds
+// every key, N_k >= beta).  Block-wide sum, returned to every thread.
+__device__ long long pairs_at(const Dims& m, const Buffers& b, int h, int beta, long long* red) {
+  const int n = b.nK[h / m.G], nq = b.nQ[h];
+  long long acc = 0;
+  for (int a = threadIdx.x; a < nq; a += blockDim.x) {
+    const int* pref = b.rankPref + ((long long)h * m.Cq + a) * m.Ck;
+    int lo = 0, hi = n - 1;                       // first prefix with count >= beta
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (pref[mid] >= beta) hi = mid; else lo = mid + 1;
+    }
+    acc += (long long)b.sizeQ[(long long)h * m.Cq + a] * pref[lo];
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  long long s = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];   // fixed order: deterministic
+  return s;
+}
+
+// Calibrated budget (App. D.2, calibrated toward the target): routed pairs never
+// decrease in beta, so a bisection over integer beta in [1, N_k] finds the smallest beta
+// reaching T = rho* N_q N_k - M N_k; of its selection and that of beta - 1 (the last below
+// T) the one nearer T is kept, the denser on a tie, and reported by the smallest beta that
+// gives it (a second bisection when it is the one below).  One block per head.
+__global__ void __launch_bounds__(256) calibrate_kernel(Dims m, Buffers b) {
+  __shared__ long long red[8];
+  const int h = blockIdx.x;
+  const double T = m.rho * (double)m.Nq * (double)m.Nk - (double)m.M * (double)m.Nk;
+  int lo = 1, hi = m.Nk;
+  long long plo = pairs_at(m, b, h, lo, red), phi = -1;
+  int beta = 1;
+  if ((double)plo < T) {
+    phi = pairs_at(m, b, h, hi, red);             // every key: reaches T since rho* <= 1
+    while (hi - lo > 1) {                          // invariant: pairs(lo) < T <= pairs(hi)
+      const int mid = lo + (hi - lo) / 2;
+      const long long pm = pairs_at(m, b, h, mid, red);
+      if ((double)pm >= T) { hi = mid; phi = pm; } else { lo = mid; plo = pm; }
+    }
+    beta = hi;                                     // the smallest beta of its selection
+    if (T - (double)plo < (double)phi - T) {
+      // the selection below T: the smallest beta that gives it (pairs(beta) >= pairs(lo))
+      int l2 = 0, h2 = lo;                         // pairs(l2) < plo <= pairs(h2); pairs(0) := -1
+      while (h2 - l2 > 1) {
+        const int mid = l2 + (h2 - l2) / 2;
+        if (pairs_at(m, b, h, mid, red) >= plo) h2 = mid; else l2 = mid;
+      }
+      beta = h2;
+    }
+  }
+  if (threadIdx.x == 0) b.betaH[h] = (double)beta;
 }
 
 // Group-major copies of Q, K, V with 16-byte vector loads; inverse query permutation.
@@ -374,7 +451,13 @@ sparsepr_status launch_route(const Plan& p, cudaStream_t st) {
   SPR_CUDA_OK(cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem));
   score_kernel<<<dim3(cdiv(m.Cq, kScoreQ), m.H), 256, ssmem, st>>>(m, p.b);
   SPR_LAUNCH_OK();
-  select_kernel<<<dim3(m.Cq, m.H), 1024, 0, st>>>(m, p.b);
+  if (m.budget == SPARSEPR_BUDGET_CALIBRATED) {
+    select_kernel<<<dim3(m.Cq, m.H), 1024, 0, st>>>(m, p.b, 1);
+    SPR_LAUNCH_OK();
+    calibrate_kernel<<<m.H, 256, 0, st>>>(m, p.b);
+    SPR_LAUNCH_OK();
+  }
+  select_kernel<<<dim3(m.Cq, m.H), 1024, 0, st>>>(m, p.b, 0);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

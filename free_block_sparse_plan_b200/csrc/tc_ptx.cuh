@@ -226,6 +226,60 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// ---------------------------------------------------------------- paired fp32 arithmetic
+// sm_100 issues some fp32 operations on two lanes of a 64-bit register pair at once
+// (add/sub/fma .f32x2, each lane rounded exactly as the scalar instruction), and takes a
+// maximum of three operands in one instruction.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly of two values with the paired instructions: the same operations in the
+// same order per lane (bit-identical results), the exponent added by one integer
+// multiply-add per lane (the low bits of x + 1.5 * 2^23, times 2^23, are n << 23).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t C = f2pack(12582912.0f, 12582912.0f);
+  const uint64_t x = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = add2(x, C);
+  const uint64_t f = sub2(x, sub2(t, C));
+  uint64_t p = fma2(f2pack(5.306559005e-02f, 5.306559005e-02f), f, f2pack(2.421349009e-01f, 2.421349009e-01f));
+  p = fma2(p, f, f2pack(6.935124561e-01f, 6.935124561e-01f));
+  p = fma2(p, f, f2pack(9.999566473e-01f, 9.999566473e-01f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  int r0, r1;
+  asm("mad.lo.s32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_int(t0)), "r"(__float_as_int(p0)));
+  asm("mad.lo.s32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_int(t1)), "r"(__float_as_int(p1)));
+  y0 = __int_as_float(r0);
+  y1 = __int_as_float(r1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -29,6 +29,7 @@ SPARSEPR_BF16 = 1
 SPARSEPR_ENGINE_AUTO = 0
 SPARSEPR_EST_RIDGE, SPARSEPR_EST_MEAN, SPARSEPR_EST_SCALAR, SPARSEPR_EST_DIAGONAL = 0, 1, 2, 3
 SPARSEPR_PARTITION_RESPONSE, SPARSEPR_PARTITION_SEMANTIC = 0, 1
+SPARSEPR_BUDGET_PREFIX, SPARSEPR_BUDGET_CALIBRATED = 0, 1
 SPARSEPR_ENGINE_SIMT = 1
 
 EXPORTS = [
@@ -36,7 +37,7 @@ EXPORTS = [
     "CELL_COUNT", "CELL_IDS", "PROBES", "PROBE_COUNT", "KMEANS_ITERS", "OBJECTIVE", "PAIRS",
     "FACTOR_K", "FACTOR_Q", "EIG_K", "EIG_Q", "METRIC_K", "METRIC_Q", "PHI_K", "PHI_Q",
     "CENTRES_Q", "SCORES", "OSP", "ODENSE_PROBE", "FIT_MU_X", "FIT_MU_R", "FIT_S", "FIT_B",
-    "FIT_P", "FIT_REFF", "PROBE_DIST", "KBAR", "QBAR", "KM_REASSIGNED",
+    "FIT_P", "FIT_REFF", "PROBE_DIST", "KBAR", "QBAR", "KM_REASSIGNED", "BETA",
 ]
 EXPORT_ID = {name: i for i, name in enumerate(EXPORTS)}
 
@@ -47,7 +48,8 @@ SYMBOLS = [
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
     "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
     "sparsepr_launch_count", "sparsepr_state_size", "sparsepr_save_state", "sparsepr_plan_warm",
-    "sparsepr_dense_check",
+    "sparsepr_dense_check", "sparsepr_support_workspace_size", "sparsepr_support_densities",
+    "sparsepr_affine_workspace_size", "sparsepr_affine_fit",
 ]
 
 
@@ -58,7 +60,7 @@ class sparsepr_params(ctypes.Structure):
                 ("lam", c_double), ("target_density", c_double),
                 ("kmeans_max_iter", c_int32), ("engine", c_int32), ("seed", c_uint64),
                 ("estimator", c_int32), ("G", c_int32), ("partition", c_int32),
-                ("reserved", c_int32)]
+                ("budget", c_int32)]
 
 
 class sparsepr_stats(ctypes.Structure):
@@ -102,6 +104,13 @@ def lib():
                                                    c_void_p]),
             "sparsepr_check": (c_int32, [c_void_p, c_void_p, POINTER(c_int32)]),
             "sparsepr_dense_check": (c_int32, [c_void_p, POINTER(c_int32)]),
+            "sparsepr_support_workspace_size": (c_int32, [P, c_int32, c_int32, POINTER(c_size_t)]),
+            "sparsepr_support_densities": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                     c_int32, c_int32, c_double, c_void_p, c_size_t,
+                                                     c_void_p, c_void_p, c_void_p]),
+            "sparsepr_affine_workspace_size": (c_int32, [c_void_p, POINTER(c_size_t)]),
+            "sparsepr_affine_fit": (c_int32, [c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
+                                              c_void_p, c_void_p]),
             "sparsepr_get_stats": (c_int32, [c_void_p, c_void_p, POINTER(sparsepr_stats)]),
             "sparsepr_export_size": (c_int32, [c_void_p, c_int32, POINTER(c_size_t)]),
             "sparsepr_export": (c_int32, [c_void_p, c_int32, c_void_p, c_size_t, c_void_p]),
@@ -139,20 +148,21 @@ def _check(status: int, where: str):
 
 def make_params(H, N_q, N_k, d, dtype, M_s, r_K, r_Q, C_q, C_k, M, r, lam, target_density,
                 kmeans_max_iter=25, seed=0, engine=SPARSEPR_ENGINE_AUTO, estimator=0,
-                G=1, partition=0) -> sparsepr_params:
+                G=1, partition=0, budget=0) -> sparsepr_params:
     if isinstance(dtype, str):
         dtype = {"f32": SPARSEPR_F32, "bf16": SPARSEPR_BF16}[dtype]
     return sparsepr_params(H=H, N_q=N_q, N_k=N_k, d=d, dtype=dtype, M_s=M_s, r_K=r_K, r_Q=r_Q,
                            C_q=C_q, C_k=C_k, M=M, r=r, lam=lam, target_density=target_density,
                            kmeans_max_iter=kmeans_max_iter, engine=engine, seed=seed,
-                           estimator=estimator, G=G, partition=partition, reserved=0)
+                           estimator=estimator, G=G, partition=partition, budget=budget)
 
 
 def params_from_dict(p: dict, engine=SPARSEPR_ENGINE_AUTO) -> sparsepr_params:
     return make_params(p["H"], p["N_q"], p["N_k"], p["d"], p["dtype"], p["M_s"], p["r_K"],
                        p["r_Q"], p["C_q"], p["C_k"], p["M"], p["r"], p["lam"],
                        p["target_density"], p["kmeans_max_iter"], p["seed"], engine,
-                       p.get("estimator", 0), p.get("G", 1), p.get("partition", 0))
+                       p.get("estimator", 0), p.get("G", 1), p.get("partition", 0),
+                       p.get("budget", 0))
 
 
 # ----------------------------------------------------------------------------------
@@ -268,6 +278,27 @@ def sparsepr_dense_check(stream=None) -> int:
     return int(e.value)
 
 
+def support_densities(Q, K, rows, pool, npools, alpha=0.9, stream=None):
+    """O1 support sizes |D_i(alpha)| of rows [H, nrows] (device int32) and the pooled
+    union sizes of each pool [H, npools] (pool: device int32 [H, nrows]); see
+    sparsepr_support_densities."""
+    import torch
+    H, Nq, d = Q.shape
+    dt = SPARSEPR_BF16 if Q.dtype == torch.bfloat16 else SPARSEPR_F32
+    p = make_params(H, Nq, K.shape[1], d, dt, 1, 1, 1, 1, 1, 1, 0, 0.0, 1.0, G=H // K.shape[0])
+    nrows = rows.shape[1]
+    nb = c_size_t(0)
+    _check(lib().sparsepr_support_workspace_size(ctypes.byref(p), nrows, npools, ctypes.byref(nb)),
+           "sparsepr_support_workspace_size")
+    ws = torch.empty(nb.value, dtype=torch.uint8, device=Q.device)
+    sizes = torch.empty((H, nrows), dtype=torch.int32, device=Q.device)
+    pooled = torch.empty((H, npools), dtype=torch.int32, device=Q.device)
+    _check(lib().sparsepr_support_densities(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(rows), _ptr(pool),
+                                            nrows, npools, alpha, _ptr(ws), nb.value, _ptr(sizes),
+                                            _ptr(pooled), _stream(stream)), "sparsepr_support_densities")
+    return sizes, pooled
+
+
 # ----------------------------------------------------------------------------------
 # Torch convenience layer (still marshalling only)
 
@@ -304,7 +335,7 @@ def _export_layout(p: sparsepr_params, name: str):
         "FIT_B": (f64, (H, d, d)), "FIT_P": (f64, (H, d, d)), "FIT_REFF": (i32, (H,)),
         "PROBE_DIST": (f64, (H, p.N_q)), "KBAR": (f64, (Hk, p.C_k, d)),
         "QBAR": (f64, (H, p.C_q, d)),
-        "KM_REASSIGNED": (i64, (2, H)),
+        "KM_REASSIGNED": (i64, (2, H)), "BETA": (f64, (H,)),
     }[name]
 
 
@@ -364,6 +395,21 @@ class Plan:
 
     def check(self, stream=None) -> int:
         return sparsepr_check(self.handle, _stream(stream))
+
+    def affine_fit(self, dense, stream=None):
+        """O3 affine fit of the residual dense - O_sp (dense: [H, N_q, d] device tensor in
+        original order); returns (explained fraction [H], remaining squared error [H])."""
+        import torch
+        nb = c_size_t(0)
+        _check(lib().sparsepr_affine_workspace_size(self.handle, ctypes.byref(nb)),
+               "sparsepr_affine_workspace_size")
+        ws = torch.empty(nb.value, dtype=torch.uint8, device=dense.device)
+        H = self.params.H
+        expl = torch.empty(H, dtype=torch.float64, device=dense.device)
+        err = torch.empty(H, dtype=torch.float64, device=dense.device)
+        _check(lib().sparsepr_affine_fit(self.handle, _ptr(dense), _ptr(ws), nb.value, _ptr(expl),
+                                         _ptr(err), _stream(stream)), "sparsepr_affine_fit")
+        return expl, err
 
     def export(self, name: str, stream=None) -> np.ndarray:
         dtype, shape = _export_layout(self.params, name)

@@ -71,6 +71,8 @@ class Workload:
     G: int = 1
     # 0 response-coupled partition (the method), 1 semantic reference partition
     partition: int = 0
+    # 0 plain prefix budget, 1 budget calibrated toward the target density
+    budget: int = 0
 
     @property
     def H_kv(self) -> int:
@@ -90,7 +92,8 @@ class Workload:
                     M_s=self.M_s, r_K=self.r_K, r_Q=self.r_Q, C_q=self.C_q,
                     C_k=self.C_k, M=self.M, r=self.r, lam=self.lam,
                     target_density=self.rho, kmeans_max_iter=self.kmeans_max_iter,
-                    seed=self.seed, estimator=self.estimator, G=self.G, partition=self.partition)
+                    seed=self.seed, estimator=self.estimator, G=self.G, partition=self.partition,
+                    budget=self.budget)
 
 
 TINY = Workload("tiny-f32-1x1024x64", H=1, N=1024, d=64, dtype="f32",

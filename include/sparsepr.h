@@ -92,6 +92,21 @@ typedef enum {
   SPARSEPR_PARTITION_SEMANTIC = 1
 } sparsepr_partition;
 
+/* Routing budget of sparsepr_plan ("Partition the Support, Reconstruct the Residual",
+ * S4.3 and App. B.3: every query group keeps the shortest score-ranked prefix of K/V
+ * groups whose key count reaches a common budget beta).
+ *   PREFIX      beta = (target_density - M/N_q) N_k: the realised rho_exec is at or above
+ *               the target.
+ *   CALIBRATED  App. D.2 calibrates the budget toward the target: per head, the integer
+ *               beta in [1, N_k] whose selection brings rho_exec nearest the target (of two
+ *               selections equally near, the denser; of the betas giving one selection,
+ *               the smallest), found by bisection on beta (rho_exec never decreases in
+ *               beta).  The realised density may then fall on either side of the target. */
+typedef enum {
+  SPARSEPR_BUDGET_PREFIX = 0,
+  SPARSEPR_BUDGET_CALIBRATED = 1
+} sparsepr_budget;
+
 /*
  * Problem and hyper-parameters of one call (paper S2, S4; values of the review page's
  * hyper-parameter table: r_K=48, r_Q=64, M=64, r=16, lambda=0.1).
@@ -126,7 +141,7 @@ typedef enum {
  *                     r_K and r_Q are ignored (the coordinates are the d raw channels),
  *                     FACTOR_K / FACTOR_Q export the identity and METRIC_* / EIG_* are not
  *                     computed; warm starts take the response partition.
- *   reserved          must be 0
+ *   budget            sparsepr_budget (0, the plain prefix rule, unless calibrating)
  */
 typedef struct {
   int32_t H, N_q, N_k, d;
@@ -140,7 +155,7 @@ typedef struct {
   int32_t estimator;
   int32_t G;
   int32_t partition;
-  int32_t reserved;
+  int32_t budget;
 } sparsepr_params;
 
 typedef struct sparsepr_plan_s* sparsepr_plan_t;
@@ -280,6 +295,49 @@ sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* params, const
  * other streams may set them after the read.  Allocates nothing. */
 sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error);
 
+/*
+ * Diagnostics of "Partition the Support, Reconstruct the Residual" S3 (observations O1,
+ * O3), in fp64.  They measure a partition; they are not part of the attention call.
+ *
+ * O1 support densities.  For query row i of head h, D_i(alpha) is the smallest set of
+ * keys whose dense attention weights softmax(q_i K^T / sqrt(d)) reach the fraction alpha
+ * of the row's mass: keys by decreasing weight, the lowest index first among equal
+ * weights, the mass compared with alpha (1 - 1e-15) times the row's total.  rows [H][nrows]
+ * (device int32, indices into [0, N_q), clamped) picks each head's rows, pool [H][nrows]
+ * (device int32 in [0, npools); a row outside marks nothing) assigns them to pools.
+ * Outputs (device int32): sizes [H][nrows] = |D_i(alpha)| (tau_i = sizes / N_k) and
+ * pooled [H][npools] = |union of the D_i of the pool's rows| (gamma = pooled / N_k).
+ * Only H, N_q, N_k, d, dtype and G of params are read (K is [H/G, N_k, d]).  workspace:
+ * device, 256-byte aligned, sparsepr_support_workspace_size bytes (about
+ * 8 H nrows N_k).  SPARSEPR_ERR_ARG for 0 < alpha <= 1 violated, nrows < 1 or
+ * npools outside [1, nrows].  Asynchronous.
+ */
+sparsepr_status sparsepr_support_workspace_size(const sparsepr_params* params, int32_t nrows,
+                                                int32_t npools, size_t* bytes);
+sparsepr_status sparsepr_support_densities(const sparsepr_params* params, const void* Q,
+                                           const void* K, const int32_t* rows,
+                                           const int32_t* pool, int32_t nrows, int32_t npools,
+                                           double alpha, void* workspace, size_t workspace_bytes,
+                                           int32_t* sizes, int32_t* pooled, void* stream);
+
+/*
+ * O3 oracle affine fit (S3 O3, App. D.5), per head over all N_q rows: the least-squares
+ * fit R ~ 1 b + O_sp B of the hard-drop residual R = dense - O_sp, with the centred sparse
+ * output's non-zero columns scaled to unit norm and directions whose singular value is
+ * at most 1e-10 times the largest left out.  The directions come from the
+ * eigendecomposition of the scaled Gram matrix, so only singular values above about
+ * 1e-8 of the largest are resolved (an ill-conditioned O_sp fits its leading directions
+ * only).  plan: after sparsepr_attend (its sparse output is used).  dense: device
+ * [H,N_q,d] in params dtype, the exact attention output in original order (for example
+ * from sparsepr_dense_attention).  Outputs (device fp64 [H]): explained = 1 - err / |R|^2
+ * and err = the remaining squared error.  workspace: device, 256-byte aligned,
+ * sparsepr_affine_workspace_size bytes.  Asynchronous.
+ */
+sparsepr_status sparsepr_affine_workspace_size(sparsepr_plan_t plan, size_t* bytes);
+sparsepr_status sparsepr_affine_fit(sparsepr_plan_t plan, const void* dense, void* workspace,
+                                    size_t workspace_bytes, double* explained, double* err,
+                                    void* stream);
+
 /* Synchronises `stream` and reports the device error word: SPARSEPR_OK or
  * SPARSEPR_ERR_DEVICE_CHECK (with the word in *device_error when non-NULL). */
 sparsepr_status sparsepr_check(sparsepr_plan_t plan, void* stream, int32_t* device_error);
@@ -330,7 +388,8 @@ typedef enum {
                                    summed over its steps, when it keeps distance bounds
                                    (warm plans; zero otherwise); the others kept their
                                    label by the bounds */
-  SPARSEPR_X_COUNT = 37
+  SPARSEPR_X_BETA = 37,       /* double [H]    per-query key budget beta the routing used */
+  SPARSEPR_X_COUNT = 38
 } sparsepr_export_what;
 
 /* Size in bytes of an exported array for this plan. Host only. */

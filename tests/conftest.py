@@ -10,3 +10,15 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200) and the built library")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Lists every probe-list swap the GPU parity tests excused as a distance tie (both
+    sides compute the distances in fp64; a swap is excused only at a 1e-6 relative tie)."""
+    mod = sys.modules.get("test_gpu_parity")
+    if mod is None or not getattr(mod, "RAN", None):
+        return
+    swaps = mod.SWAPS_EXCUSED
+    terminalreporter.write_line(f"probe-list swaps excused as distance ties: {len(swaps)}")
+    for where, positions in swaps:
+        terminalreporter.write_line(f"  {where}: positions {positions}")

@@ -26,12 +26,16 @@ TOL = {"f32": 1e-5, "bf16": 1e-2}
 _oracle_cache = {}
 
 
+RAN = []                  # set once the module's GPU tests start (for the summary)
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     import __graft_entry__
     __graft_entry__.build()
+    RAN.append(True)
 
 
 def oracle_head(w: W.Workload, h: int, rows=None):
@@ -459,6 +463,8 @@ def test_hunyuan_full_size_sampled_heads():
 
 
 def test_operating_point_sweep_head0():
+    # every (rho*, M) point of the operating-point sweep on the Wan-like head 0, oracle
+    # labels injected (the partition does not depend on rho* or M)
     base = W.WAN
     q, k, v, _ = oracle_head(base, 0, rows=np.arange(4))
     part = _oracle_cache[(base, 0)][3]
@@ -467,7 +473,9 @@ def test_operating_point_sweep_head0():
     labQ = torch.tensor(part.km_Q.labels[None], dtype=torch.int32, device="cuda")
     labK = torch.tensor(part.km_K.labels[None], dtype=torch.int32, device="cuda")
     rows = np.unique(np.linspace(0, base.N - 1, 1024).astype(np.int64))
-    for rho, M in [(0.12, 64), (0.17, 64), (0.26, 64), (0.35, 64), (0.22, 32), (0.22, 128)]:
+    points = [(rho, M) for rho in W.SWEEP_RHO for M in W.SWEEP_M]
+    assert len(points) == 15
+    for rho, M in points:
         w = base.with_(H=1, rho=rho, M=M)
         p = O.Params.from_dict(w.params())
         res = O.sparsepr_call(q, k, v, p, head=0, rows=rows, part=part)
@@ -475,6 +483,100 @@ def test_operating_point_sweep_head0():
         check_injected_head(plan, out[0].float().cpu().numpy(), res, 0, w)
         st = plan.stats()
         assert abs(st["rho_exec"] - res.rho_exec) < 1e-15
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_calibrated_budget_matches_oracle(name):
+    # App. D.2's budget calibrated toward the target (reading S13): the per-head budget,
+    # the selected cells and the routed pairs bit-exact with oracle labels injected, the
+    # output within tolerance, and the realised density no farther from the target than
+    # the plain prefix rule's.
+    base = W.TINY if name == "tiny" else W.MID.with_(H=3)
+    w = base.with_(budget=1)
+    inputs = W.make_inputs_torch(w, device="cuda")
+    ref = [oracle_head(w, h)[3] for h in range(w.H)]
+    labQ = torch.tensor(np.stack([r.part.km_Q.labels for r in ref]), dtype=torch.int32, device="cuda")
+    labK = torch.tensor(np.stack([r.part.km_K.labels for r in ref]), dtype=torch.int32, device="cuda")
+    plan, out, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK))
+    assert plan.check() == 0
+    beta = plan.export("BETA")
+    out_np = out.double().cpu().numpy()
+    for h, r in enumerate(ref):
+        assert beta[h] == r.beta, (h, beta[h], r.beta)
+        check_injected_head(plan, out_np[h], r, h, w)
+    plain, _, _ = gpu_call(base, inputs=inputs, labels=(labQ, labK))
+    assert np.all(plain.export("BETA") == (base.rho - base.M / base.N) * base.N)
+    pairs_cal, pairs_plain = plan.export("PAIRS"), plain.export("PAIRS")
+    for h in range(w.H):
+        T = w.rho * w.N * w.N - w.M * w.N
+        assert abs(pairs_cal[h] - T) <= abs(pairs_plain[h] - T)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_support_densities_match_oracle(name):
+    # O1 ([P] S3): |D_i(0.9)| of sampled rows and the pooled union per query group,
+    # against the oracle on fp64 weights of the same stored values.  Sizes are exact
+    # unless the oracle's sorted running sum sits within 1e-12 of the mass target at the
+    # boundary (a rounding tie); pooled sizes are compared where every size matched.
+    w = W.TINY if name == "tiny" else W.MID.with_(H=2)
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    nrows = 256 if name == "tiny" else 64
+    idx = np.unique(np.linspace(0, w.N - 1, nrows).astype(np.int64))
+    rows_h, pool_h, refs = [], [], []
+    for h in range(w.H):
+        _, _, _, res = oracle_head(w, h, rows=np.arange(4))
+        comp = res.part.gq.compact[idx]
+        uniq, pool = np.unique(comp, return_inverse=True)
+        rows_h.append(idx)
+        pool_h.append(pool)
+        refs.append((uniq.size, pool))
+    npools = max(u for u, _ in refs)
+    rows = torch.tensor(np.stack(rows_h), dtype=torch.int32, device="cuda")
+    pool = torch.tensor(np.stack(pool_h), dtype=torch.int32, device="cuda")
+    sizes, pooled = N.support_densities(Q, K, rows, pool, npools, 0.9)
+    sizes, pooled = sizes.cpu().numpy(), pooled.cpu().numpy()
+    for h in range(w.H):
+        q, k, _ = W.make_head(w, h)
+        a = O.attention_probs(q[idx], k)
+        ref = O.support_size(a, 0.9)
+        exact = np.array_equal(sizes[h], ref)
+        if not exact:
+            srt = -np.sort(-a, axis=1)
+            cum = np.cumsum(srt, axis=1)
+            for i in np.flatnonzero(sizes[h] != ref):
+                assert abs(int(sizes[h][i]) - int(ref[i])) == 1, (h, i)
+                k0 = min(sizes[h][i], ref[i]) - 1
+                gap = abs(cum[i, k0] - 0.9 * cum[i, -1] * (1 - 1e-15)) / cum[i, -1]
+                assert gap < 1e-12, (h, i, gap)
+        else:
+            npool_h, pid = refs[h]
+            for c in range(npool_h):
+                sel = pid == c
+                _, gamma = O.support_densities(a[sel], 0.9)
+                assert pooled[h][c] == round(gamma * w.N), (h, c)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_affine_fit_matches_oracle(name):
+    # O3 ([P] S3, App. D.5): the affine fit of R = dense - O_sp on O_sp over all rows, on
+    # the GPU's own sparse and dense outputs, against the oracle's SVD-based fit.
+    w = W.TINY if name == "tiny" else W.MID.with_(H=2)
+    Q, K, V = W.make_inputs_torch(w, device="cuda")
+    plan = N.Plan(N.params_from_dict(w.params()), Q, K, V)
+    plan.attend()
+    dense = N.dense_attention(Q, K, V)
+    expl, err = plan.affine_fit(dense)
+    expl, err = expl.cpu().numpy(), err.cpu().numpy()
+    assert plan.check() == 0
+    osp = plan.export("OSP")
+    perm = plan.export("PERM_Q")
+    dn = dense.double().cpu().numpy()
+    for h in range(w.H):
+        orig = np.empty_like(osp[h], dtype=np.float64)
+        orig[perm[h]] = osp[h]
+        e_ref, err_ref = O.oracle_affine_fit(orig, dn[h])
+        assert abs(expl[h] - e_ref) < 1e-9, (h, expl[h], e_ref)
+        assert abs(err[h] - err_ref) <= 1e-6 * err_ref + 1e-300, (h, err[h], err_ref)
 
 
 # ---------------------------------------------------------------------------------- edges
