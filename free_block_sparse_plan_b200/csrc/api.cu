@@ -186,8 +186,7 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
     const size_t Nm = Nk > Nq ? Nk : Nq, Cm = Ck > Cq ? Ck : Cq;
     b->kmFx = c.take<unsigned long long>(H * Cm * 64 * 3);
     b->kmFxCnt = c.take<int>(H * Cm);
-    b->kmChg = c.take<int4>(H * Nm);
-    b->kmChgCnt = c.take<int>(2);
+    b->kmChg = c.take<unsigned long long>(H * Nm);
   }
   b->err = c.take<int>(64);
   return (c.off + 255) & ~size_t(255);

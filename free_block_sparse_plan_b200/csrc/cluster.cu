@@ -35,8 +35,7 @@ struct KmView {         // one k-means instance (keys or queries) for all heads
   int H;                // instances: query heads, or K/V heads for the key side
   unsigned long long* fx;     // [H][C][64][3] exact member sums (three 40-bit limbs)
   int* fxcnt;                 // [H][C] member counts
-  int4* chg;                  // label changes of the step {h*N + n, old, new, 0}
-  int* chgcnt;                // [2] their counts, slot it & 1
+  unsigned long long* chg;    // [H][N] last label change of each point (chg_entry)
 };
 
 KmView view(const Plan& p, bool query) {
@@ -44,9 +43,9 @@ KmView view(const Plan& p, bool query) {
   const Dims& m = p.dm;
   if (query)
     return {b.phiQ, b.centQ, b.labQ, b.histQ, b.permQ, b.offQ, b.kmQ, b.objQ, b.kmDelta, b.kmDmax,
-            m.Nq, m.Cq, m.rQ, m.nchQ, 1, m.H, b.kmFx, b.kmFxCnt, b.kmChg, b.kmChgCnt};
+            m.Nq, m.Cq, m.rQ, m.nchQ, 1, m.H, b.kmFx, b.kmFxCnt, b.kmChg};
   return {b.phiK, b.centK, b.labK, b.histK, b.permK, b.offK, b.kmK, b.objK, b.kmDelta, b.kmDmax,
-          m.Nk, m.Ck, m.rK, m.nchK, 0, m.Hk, b.kmFx, b.kmFxCnt, b.kmChg, b.kmChgCnt};
+          m.Nk, m.Ck, m.rK, m.nchK, 0, m.Hk, b.kmFx, b.kmFxCnt, b.kmChg};
 }
 
 // ---------------------------------------------------------------------------------
@@ -328,7 +327,7 @@ __global__ void __launch_bounds__(128) km_assign_kernel(KmView v, int it) {
     if (old != bi) {
       *lp = bi;
       km[1 + (it & 1)] = 1;
-      v.chg[atomicAdd(v.chgcnt + (it & 1), 1)] = make_int4((int)((long long)h * v.N + row), old, bi, 0);
+      v.chg[(long long)h * v.N + row] = chg_entry(old, bi, it);
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) km[3] += 1;
@@ -556,35 +555,42 @@ __global__ void __launch_bounds__(256) km_fx_full_kernel(KmView v, int it) {
   }
   if (threadIdx.x == 0) {
     v.fxcnt[(long long)h * v.C + c] = m1 - m0;
-    if (c == 0 && h == 0) v.chgcnt[(it + 1) & 1] = 0;     // the next step's log
   }
 }
 
-// One warp per logged change: the point's limbs move from the old centre (none on the
-// first step) to the new one.
+// Each warp scans 32 points at a time for changes stamped with this step; for every such
+// point the whole warp moves its limbs from the old centre to the new one.
 __global__ void __launch_bounds__(256) km_fx_apply_kernel(KmView v, int it) {
-  const int n = v.chgcnt[it & 1];
   const int lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && threadIdx.x == 0) v.chgcnt[(it + 1) & 1] = 0;   // the next step's log
-  for (long long e = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; e < n;
-       e += ((long long)gridDim.x * blockDim.x) >> 5) {
-    const int4 c = v.chg[e];
-    const long long pi = c.x;
-    const int h = (int)(pi / v.N);
-    const double* x = v.X + pi * v.r;
-    unsigned long long* to = v.fx + ((long long)h * v.C + c.z) * 64 * 3;
-    unsigned long long* from = c.y >= 0 ? v.fx + ((long long)h * v.C + c.y) * 64 * 3 : nullptr;
-    for (int k = lane; k < v.r; k += 32) {
-      long long l[3];
-      fx_split(x[k], l);
-      for (int j = 0; j < 3; ++j) {
-        atomicAdd(to + 3 * k + j, (unsigned long long)l[j]);
-        if (from) atomicAdd(from + 3 * k + j, (unsigned long long)(-l[j]));
+  const long long HN = (long long)v.H * v.N;
+  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long base = w0 * 32; base < HN; base += nw * 32) {
+    const long long i = base + lane;
+    const unsigned long long e = i < HN ? v.chg[i] : ~0ull;
+    unsigned todo = __ballot_sync(0xffffffffu, (int)(e >> 32) == it);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const unsigned long long ee = __shfl_sync(0xffffffffu, e, src);
+      const long long pi = base + src;
+      const int h = (int)(pi / v.N);
+      const int cnew = (int)(ee & 0xFFFF), cold = (int)((ee >> 16) & 0xFFFF);
+      const double* x = v.X + pi * v.r;
+      unsigned long long* to = v.fx + ((long long)h * v.C + cnew) * 64 * 3;
+      unsigned long long* from = cold != 0xFFFF ? v.fx + ((long long)h * v.C + cold) * 64 * 3 : nullptr;
+      for (int k = lane; k < v.r; k += 32) {
+        long long l[3];
+        fx_split(x[k], l);
+        for (int j = 0; j < 3; ++j) {
+          atomicAdd(to + 3 * k + j, (unsigned long long)l[j]);
+          if (from) atomicAdd(from + 3 * k + j, (unsigned long long)(-l[j]));
+        }
       }
-    }
-    if (lane == 0) {
-      atomicAdd(v.fxcnt + (long long)h * v.C + c.z, 1);
-      if (c.y >= 0) atomicAdd(v.fxcnt + (long long)h * v.C + c.y, -1);
+      if (lane == 0) {
+        atomicAdd(v.fxcnt + (long long)h * v.C + cnew, 1);
+        if (from) atomicAdd(v.fxcnt + (long long)h * v.C + cold, -1);
+      }
     }
   }
 }
@@ -826,11 +832,12 @@ sparsepr_status launch_kmeans(const Plan& p, bool query, cudaStream_t st) {
   const Buffers& b = p.b;
   const KmTcBuffers kb{b.kmXhi, b.kmXlo, b.kmShi, b.kmSlo, b.kmU, b.kmDelta, b.kmL, b.kmDmax, b.kmAidx,
                        b.kmAcnt, b.kmReassigned + (query ? H : 0), b.kmXn, b.kmChi, b.kmClo, b.kmCn, b.kmCmaxb, b.kmQueue, b.kmQcnt,
-                       b.kmChg, b.kmChgCnt};
+                       b.kmChg};
   // exact sums start empty; every label starts at -1, so the first step logs every point
   SPR_CUDA_OK(cudaMemsetAsync(b.kmFx, 0, sizeof(unsigned long long) * (size_t)H * v.C * 64 * 3, st));
   SPR_CUDA_OK(cudaMemsetAsync(b.kmFxCnt, 0, sizeof(int) * (size_t)H * v.C, st));
-  SPR_CUDA_OK(cudaMemsetAsync(b.kmChgCnt, 0, sizeof(int) * 2, st));
+  // no point has a stamped change yet (stamp -1)
+  SPR_CUDA_OK(cudaMemsetAsync(b.kmChg, 0xFF, sizeof(unsigned long long) * (size_t)H * v.N, st));
   if (tc) {
     SPR_CUDA_OK(cudaMemsetAsync(b.kmCmaxb, 0, sizeof(int) * 2 * H, st));
     SPR_CUDA_OK(cudaMemsetAsync(b.kmQcnt, 0, sizeof(int) * 2, st));

@@ -100,8 +100,7 @@ struct Buffers {
   int *warmCold;             // heads whose warm factor update fell back to the eigensolve [2][H]
   unsigned long long *kmFx;  // exact member sums of each centre, three 40-bit limbs [H][Cmax][64][3]
   int *kmFxCnt;              // member counts [H][Cmax]
-  int4 *kmChg;               // label changes of the current step {h*N + n, old, new, -} [H*Nmax]
-  int *kmChgCnt;             // their counts [2], slot it & 1
+  unsigned long long *kmChg; // last label change of each point: new | old << 16 | step << 32 [H*Nmax]
   int *err;                  // device error word
 };
 
@@ -160,6 +159,14 @@ inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // ---------------------------------------------------------------------------------
 // Device utilities
+
+// A point's label change at k-means step `it`: new | old << 16 | it << 32 (old = 0xFFFF
+// for none); the exact-sum update applies the entries stamped with its own step, so the
+// array needs no clearing between steps.
+__device__ __forceinline__ unsigned long long chg_entry(int old, int now, int it) {
+  return (unsigned long long)(now & 0xFFFF) | ((unsigned long long)(old & 0xFFFF) << 16) |
+         ((unsigned long long)(unsigned)it << 32);
+}
 __device__ __forceinline__ float load_as_float(const void* p, long long i, int dtype) {
   if (dtype == SPARSEPR_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
   return reinterpret_cast<const float*>(p)[i];
@@ -283,8 +290,7 @@ struct KmTcBuffers {
   int* cmaxb;
   int4* queue;
   int* qcnt;
-  int4* chg;                 // label-change log (exact incremental means)
-  int* chgcnt;
+  unsigned long long* chg;   // label change of each point at this step (exact incremental means)
 };
 sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const double* cent, int H, int N, int C,
                              int r, int it, int* lab, int* kmstate, int* err, bool bounds, cudaStream_t st);

@@ -39,8 +39,10 @@ __global__ void transpose_bp_kernel(const float* Bp, int d, float* BT) {
 }
 
 // Persistent: one CTA per SM takes a contiguous range of (head, 128-row tile) pairs.  B'^T
-// of the current head stays in shared memory; the O_sp tiles go through two stages, the
-// next tile's rows copied while the current one is multiplied and written out.
+// of the current head stays in shared memory; the O_sp tiles go through two stages, and
+// the copy of tile t+2 starts as soon as tile t has been written out, so that one copy is
+// always in flight while a tile is multiplied and written (about 64 KB per SM, which the
+// HBM latency needs to reach the copy bandwidth).
 template <int D>
 __global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, const float* BT,
                                                             __nv_bfloat16* Out, int tiles_per_head,
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, c
   };
   load_tile(t0, 0);
   tc::cp_async_commit();
+  if (t0 + 1 < t1) load_tile(t0 + 1, 1);
+  tc::cp_async_commit();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -95,12 +99,14 @@ __global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, c
   for (long long t = t0; t < t1; ++t) {
     const int s = (int)((t - t0) & 1);
     const int h = (int)(t / tiles_per_head);
-    if (h != loaded) {                                // a new head: its B'^T (the previous
-      load_bt(h);                                     // multiply has completed)
+    if (h != loaded) {                                // a new head's B'^T: no multiply is
+      load_bt(h);                                     // running (the last one was waited for)
       tc::cp_async_commit();
+      tc::cp_async_wait_all();
       loaded = h;
+    } else {
+      tc::cp_async_wait_group1();                     // tile t arrived (t + 1 may be in flight)
     }
-    tc::cp_async_wait_all();                          // this tile's rows (and B'^T)
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -117,9 +123,6 @@ __global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, c
       tc::mma_commit(tc::smem_u32(bar));
     }
     __syncwarp();
-    // the next tile's rows go to the other stage while this one is multiplied and stored
-    if (t + 1 < t1) load_tile(t + 1, s ^ 1);
-    tc::cp_async_commit();
     const bool done = tc::mbar_wait(tc::smem_u32(bar), (uint32_t)((t - t0) & 1), kCWait);
     if (!__all_sync(0xffffffffu, done)) {
       if ((tid & 31) == 0) atomicOr(b.err, kErrHang);
@@ -153,10 +156,13 @@ __global__ void __launch_bounds__(128, 1) correct_tc_kernel(Dims m, Buffers b, c
           dst[4 * q + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
-    // the accumulator and this stage are free once every thread has read them
+    // the accumulator and stage s are free once every thread has read them: tile t+2's
+    // copy goes there at once
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    if (t + 2 < t1) load_tile(t + 2, s);
+    tc::cp_async_commit();
   }
   tc::cp_async_wait_all();
   tc::fence_before_sync();

@@ -72,8 +72,7 @@ struct KmArgs {
   int* km;                    // [H][4]
   int4* queue;                // ambiguous points: h * N + n, candidate slots, flags
   int* qcnt;                  // [2] queue lengths, slot it & 1
-  int4* chg;                  // label changes {h * N + n, old, new, 0}
-  int* chgcnt;                // [2] their counts, slot it & 1
+  unsigned long long* chg;    // [H][N] last label change of each point (chg_entry)
   int qcap;
   const double* X;            // [H][N][r] fp64 features (fallback when the queue is full)
   const double* cent;         // [H][C][r] fp64 centres
@@ -470,7 +469,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) km_assign_tc_kernel(const __gri
       if (old != best) {
         g.lab[pi] = best;
         g.km[4 * h + 1 + (g.it & 1)] = 1;
-        g.chg[atomicAdd(g.chgcnt + (g.it & 1), 1)] = make_int4((int)pi, old, best, 0);
+        g.chg[pi] = chg_entry(old, best, g.it);
       }
     }
   }
@@ -579,7 +578,7 @@ __global__ void __launch_bounds__(256) km_filter_kernel(const KmFilter f) {
 __global__ void __launch_bounds__(256) km_rescore_kernel(const int4* queue, const int* qcnt, int qcap,
                                                          const double* X, const double* cent, int* lab,
                                                          int* km, int N, int C, int r, int it,
-                                                         int4* chg, int* chgcnt) {
+                                                         unsigned long long* chg) {
   const int lane = threadIdx.x & 31;
   const int n = min(qcnt[it & 1], qcap);
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -613,7 +612,7 @@ __global__ void __launch_bounds__(256) km_rescore_kernel(const int4* queue, cons
       const int old = lab[pi];
       lab[pi] = bc;
       km[4 * h + 1 + (it & 1)] = 1;
-      chg[atomicAdd(chgcnt + (it & 1), 1)] = make_int4((int)pi, old, bc, 0);
+      chg[pi] = chg_entry(old, bc, it);
     }
   }
 }
@@ -724,7 +723,7 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   g.aidx = kb.aidx; g.acnt = kb.acnt + (it & 1) * H; g.U = kb.U; g.L = kb.L;
   g.xn = kb.xn; g.cn = kb.cn; g.cmaxb = kb.cmaxb; g.lab = lab; g.km = kmstate;
   g.queue = kb.queue; g.qcnt = kb.qcnt; g.qcap = (int)km_tc_queue_cap(H, N);
-  g.chg = kb.chg; g.chgcnt = kb.chgcnt;
+  g.chg = kb.chg;
   g.X = X; g.cent = cent; g.err = err;
   g.H = H; g.N = N; g.Npad = Npad; g.C = C; g.Cpad = Cpad; g.Cw = Cw; g.nch = nch; g.r = r; g.it = it;
   g.slots = slots;
@@ -735,7 +734,7 @@ sparsepr_status km_tc_assign(const KmTcBuffers& kb, const double* X, const doubl
   kern<<<grid, kKmThreads, smem, st>>>(g);
   SPR_LAUNCH_OK();
   km_rescore_kernel<<<4 * sm_count(), 256, 0, st>>>(kb.queue, kb.qcnt, g.qcap, X, cent, lab, kmstate, N, C, r,
-                                                    it, kb.chg, kb.chgcnt);
+                                                    it, kb.chg);
   SPR_LAUNCH_OK();
   return SPARSEPR_OK;
 }

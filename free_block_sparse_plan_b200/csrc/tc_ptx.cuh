@@ -63,6 +63,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 // Arrive on an mbarrier once every cp.async this thread issued so far has completed; the
 // barrier's expected count includes this arrival (no pending-count increment).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
