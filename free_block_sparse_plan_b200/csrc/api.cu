@@ -109,6 +109,7 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->invQ = c.take<int>(H * Nq);
   b->offK = c.take<int>(H * (Ck + 1));
   b->offQ = c.take<int>(H * (Cq + 1));
+  b->poffK = c.take<int>(H * (Ck + 1));
   b->kmK = c.take<int>(H * 4);
   b->kmQ = c.take<int>(H * 4);
   b->objK = c.take<double>(H * Ck);
@@ -132,8 +133,12 @@ size_t carve(const Dims& m, char* base, Buffers* b) {
   b->betaH = c.take<double>(H);
   b->pairs = c.take<long long>(H);
   b->Qp = c.take<char>(H * Nq * d * es);
-  b->Kp = c.take<char>(H * Nk * d * es);
-  b->Vp = c.take<char>(H * Nk * d * es);
+  {
+    const size_t plain = H * Nk * d * es;
+    const size_t tiled = tc_engine_applies(m.dtype, m.d, m.engine) ? (size_t)m.Hk * kv_tiled_rows(m.Nk, m.Ck) * d * 2 : 0;
+    b->Kp = c.take<char>(plain > tiled ? plain : tiled);
+    b->Vp = c.take<char>(plain > tiled ? plain : tiled);
+  }
   b->dist = c.take<double>(H * Nq);
   b->probeTop = c.take<int>(H * Cq * M);
   b->probes = c.take<int>(H * M);

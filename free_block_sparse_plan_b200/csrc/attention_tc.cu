@@ -13,9 +13,14 @@
 //              reads its S row from TMEM, online softmax in base 2 with lazy rescaling
 //              (O is rescaled only when the row max grows by more than 2^8), writes P as
 //              bf16 pairs into the TMEM columns of S already read, epilogue;
-//   warps 8-10 producers: 16-byte cp.async gathers of the Q tiles and of each K/V tile
-//              (arbitrary key rows, so the selected groups need not be contiguous) into
-//              128-byte-swizzled shared memory, two stages shared by both query tiles;
+//   warps 8-10 producers: 16-byte cp.async gathers of the Q tiles; one thread copies the
+//              K/V tiles with TMA (2-D tiled boxes, 128-byte swizzle) into the stages (two
+//              at d = 128, four at d = 64) shared by both query tiles.  Dense and probe
+//              keys are consecutive rows (64-row boxes).  Sparse keys are the concatenated
+//              row ranges of the selected K/V groups, each range starting at a multiple of
+//              four key positions (its last up-to-three positions are padding): a range is
+//              copied in boxes of 64, 16 and 4 rows, and the padding columns of S are set to
+//              -inf by the softmax warps before they read the tile;
 //   warp 11    one thread issues tcgen05.mma: S_t = Q_t K_j^T (both operands in shared
 //              memory) and O_t += P_t V_j (P read from TMEM, V MN-major), and commits to
 //              mbarriers.  The warp owns the TMEM allocation: S_A, S_B (128 columns each),
@@ -32,6 +37,7 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace spr {
 namespace {
@@ -52,6 +58,9 @@ enum Mode { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 __device__ int g_dense_err;
 
 struct TcArgs {
+  // dense and probe modes: K and V as [H_k][N_k][d] bf16 in boxes of 64 columns x 64 rows
+  // (128-byte swizzle; rows past N_k read as zeros)
+  CUtensorMap tm_k, tm_v;
   int mode;
   Dims m;
   const __nv_bfloat16* Q;
@@ -76,15 +85,16 @@ struct Layout {
   static constexpr uint32_t oK0 = 2 * kTile;
   static constexpr uint32_t oV0 = (2 + S) * kTile;
   static constexpr uint32_t oMisc = (2 + 2 * S) * kTile;
-  static constexpr uint32_t kBytes = oMisc + 14 * 1024;
+  static constexpr uint32_t kBytes = oMisc + 17 * 1024;
 };
 
 struct Misc {
   unsigned long long bars[24];
   long long qrow[kItemRows];
-  long long krow[2][kTileKeys];
-  int csum[kMaxC + 1];
-  int cbase[kMaxC];
+  int csum[kMaxC + 1];        // sparse: key position of each selected range (multiples of 8)
+  int cbase[kMaxC];           // its first row in the tensor-core K/V layout of the head
+  int clen[kMaxC];            // its true length (the rest up to the next position is padding)
+  uint32_t kvmask[4][4];      // per stage: key columns that are padding
   uint32_t tmem_base;
   int abort_flag;
   int sh[32];
@@ -112,7 +122,7 @@ __device__ __forceinline__ bool wait_bar(Misc* ms, uint32_t bar, uint32_t parity
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
+__global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __grid_constant__ TcArgs g) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
@@ -143,15 +153,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
       int sz = 0, start = 0;
       if (i < cnt) {
         const int labk = g.b.usedK[(long long)(h / m.G) * m.Ck + ids[i]];
-        start = g.b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk];
-        sz = g.b.offK[(long long)(h / m.G) * (m.Ck + 1) + labk + 1] - start;
+        const long long o = (long long)(h / m.G) * (m.Ck + 1) + labk;
+        start = g.b.poffK[o];
+        sz = g.b.offK[o + 1] - g.b.offK[o];
       }
       int tot;
-      const int ex = block_exclusive_scan(sz, ms->sh, &tot);
+      const int ex = block_exclusive_scan((sz + 7) & ~7, ms->sh, &tot);   // padded to 8
       const int prev = base_i == 0 ? 0 : ms->csum[base_i];
       if (i < cnt) {
         ms->csum[i] = prev + ex;
         ms->cbase[i] = start;
+        ms->clen[i] = sz;
       }
       __syncthreads();
       if (tid == 0) ms->csum[min(base_i + (int)blockDim.x, cnt)] = prev + tot;
@@ -178,7 +190,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   if (tid == 0) {
     tc::mbar_init(BAR(bQFull), kProducers);
     for (int s = 0; s < L::S; ++s) {
-      tc::mbar_init(BAR(bKVFull0 + s), kProducers);   // one cp.async completion per producer
+      tc::mbar_init(BAR(bKVFull0 + s), 1);            // the copying thread's arrive + bytes
       tc::mbar_init(BAR(bKVEmpty0 + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
   if (warp >= 8 && warp < 11) {
     // ============================================================ producers
     const int p = tid - 256;
-    const long long hq = (long long)h * m.Nq * d, hk = (long long)(h / m.G) * m.Nk * d;   // K/V head h / G
+    const long long hq = (long long)h * m.Nq * d;
     for (int row = p; row < kItemRows; row += kProducers) {
       long long qr = -1;
       if (row < nrows) {
@@ -228,46 +240,67 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
     tc::mbar_arrive(BAR(bQFull));
-    // K/V tiles: stage j % S.  Each producer's copies arrive on the stage's barrier when
-    // they complete (cp.async.mbarrier.arrive.noinc), so the producers move on to the next
-    // free stage without waiting for the data; the MMA thread fences the generic-proxy
-    // writes against its tensor-core reads after the barrier.
-    int cur0 = 0, cur1 = 0;             // cells of this thread's two keys (non-decreasing)
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % L::S, use = j / L::S;
-      // every producer thread takes the same decision (they meet at named barriers)
-      const bool got = use == 0 || wait_bar(ms, BAR(bKVEmpty0 + s), (use - 1) & 1, g.err);
-      if (!tc::named_sync_and(1, kProducers, got)) break;
+    // K/V tiles: stage j % S, copied by one thread.  Sparse mode: one bulk copy per panel
+    // of every run of rows (the tensor-core layout holds each panel's rows in the order of
+    // the shared-memory tile, runs start at multiples of 8 rows on both sides); the rest of
+    // the last tile comes from the head's zero rows.  Dense and probe modes: TMA boxes of
+    // 64 rows (rows past N_k read as zeros; past the item's keys, the softmax masks them).
+    // Every row of a stage is written, so its byte count is fixed.
+    if (p == 0) {
+      const int hk = h / m.G;                             // the K/V head
+      constexpr int NP = D / 64;
+      const long long rp = kv_tiled_rows(m.Nk, m.Ck);
+      const uint8_t* Kt = reinterpret_cast<const uint8_t*>(g.K) + (long long)hk * NP * rp * 128;
+      const uint8_t* Vt = reinterpret_cast<const uint8_t*>(g.V) + (long long)hk * NP * rp * 128;
+      const int zrow = g.mode == kModeSparse ? g.b.poffK[(long long)hk * (m.Ck + 1) + m.Ck] : 0;
+      int c = 0;                                          // sparse: current range
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % L::S, use = j / L::S;
+        if (use > 0 && !wait_bar(ms, BAR(bKVEmpty0 + s), (use - 1) & 1, g.err)) break;
+        const uint32_t bar = BAR(bKVFull0 + s);
+        const int t0 = j * kTileKeys;
+        if (g.mode == kModeSparse) {
+          // rows [src, src + len) of the layout into tile rows [dst, dst + len)
+          auto copy_run = [&](long long src, int dst, int len) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int kk = p + q * kProducers;
-        if (kk >= kTileKeys) break;
-        const long long v = (long long)j * kTileKeys + kk;
-        long long kr = -1;
-        if (v < nkeys) {
-          if (g.mode == kModeSparse) {
-            int c = q ? cur1 : cur0;
-            while (ms->csum[c + 1] <= v) ++c;     // csum[cnt] = nkeys > v ends the walk
-            if (q) cur1 = c; else cur0 = c;
-            kr = hk + ((long long)ms->cbase[c] + (v - ms->csum[c])) * d;
-          } else if (g.mode == kModeDense) {
-            kr = hk + v * d;
-          } else {
-            kr = hk + ((long long)split * kProbeSplit + v) * d;
+            for (int pnl = 0; pnl < NP; ++pnl) {
+              const uint32_t o = pnl * L::kPanel + (uint32_t)dst * 128u;
+              const long long so = ((long long)pnl * rp + src) * 128;
+              tc::bulk_g2s(sK(s) + o, Kt + so, (uint32_t)len * 128u, bar);
+              tc::bulk_g2s(sV(s) + o, Vt + so, (uint32_t)len * 128u, bar);
+            }
+          };
+          while (c < cnt && ms->csum[c + 1] <= t0) ++c;
+          // the padding columns of this tile, published before the stage's barrier
+          // (whose arrive releases them to the softmax warps)
+          uint32_t* mask = ms->kvmask[s];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mask[q] = 0u;
+          for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
+            const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
+            for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
           }
+          tc::mbar_expect_tx(bar, 2u * L::kTile);
+          int pos = t0;                                   // next tile position to fill
+          for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
+            const int lo = max(ms->csum[cc], t0), hi = min(ms->csum[cc + 1], t0 + kTileKeys);
+            copy_run(ms->cbase[cc] + (lo - ms->csum[cc]), lo - t0, hi - lo);
+            pos = hi;
+          }
+          if (pos < t0 + kTileKeys) copy_run(zrow, pos - t0, t0 + kTileKeys - pos);
+        } else {
+          tc::mbar_expect_tx(bar, 2u * L::kTile);
+          const int first = (g.mode == kModeProbe ? split * kProbeSplit : 0) + t0;
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int pnl = 0; pnl < NP; ++pnl) {
+              const uint32_t o = pnl * L::kPanel + (uint32_t)half * 64u * 128u;
+              tc::tma_load_3d(sK(s) + o, &g.tm_k, 64 * pnl, first + 64 * half, hk, bar);
+              tc::tma_load_3d(sV(s) + o, &g.tm_v, 64 * pnl, first + 64 * half, hk, bar);
+            }
         }
-        ms->krow[j & 1][kk] = kr;
       }
-      tc::named_sync(1, kProducers);
-      for (int e = p; e < kTileKeys * CPR; e += kProducers) {
-        const int row = e / CPR, c = e % CPR;
-        const long long off = ms->krow[j & 1][row];
-        const uint32_t o = (c >> 3) * L::kPanel + tc::sw128_offset(row, c & 7);
-        const bool ok = off >= 0;
-        tc::cp_async16(sK(s) + o, ok ? (const void*)(g.K + off + c * 8) : (const void*)g.K, ok ? 16u : 0u);
-        tc::cp_async16(sV(s) + o, ok ? (const void*)(g.V + off + c * 8) : (const void*)g.V, ok ? 16u : 0u);
-      }
-      tc::cp_async_arrive_noinc(BAR(bKVFull0 + s));
     }
     tc::cp_async_wait_all();
   } else if (warp == 11) {
@@ -386,6 +419,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(TcArgs g) {
         tc::fence_before_sync();
         tc::mbar_arrive(BAR(bPFull0 + buf));
         continue;
+      }
+      if (g.mode == kModeSparse) {
+        // padding columns of the tile (their rows belong to no selected range): -inf in S.
+        // The stage's barrier phase of tile j has completed (S(j) was computed from it);
+        // waiting on it acquires the producer's mask words.
+        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bKVFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
+        const int s = j % L::S;
+        bool any = false;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t mw = ms->kvmask[s][q];
+          any |= mw != 0u;
+          while (mw) {                                    // uniform across the warp
+            const int col = 32 * q + __ffs(mw) - 1;
+            mw &= mw - 1;
+            tc::tmem_st1(tS + col, __float_as_uint(-INFINITY));
+          }
+        }
+        if (any) tc::tmem_wait_st();
       }
       const int valid = (j == nt - 1) ? last_valid : kTileKeys;
       const bool whole = valid == kTileKeys;           // uniform: no key column masked
@@ -556,8 +608,29 @@ __global__ void __launch_bounds__(1024) build_work_kernel(Dims m, Buffers b, int
   if (threadIdx.x == 0) nwork[h] = tot;
 }
 
+// K or V of shape [H_k][N_k][d] bf16 (row-major, 16-byte aligned) in boxes of 64 columns
+// x box_rows rows; rows past N_k read as zeros.
+sparsepr_status make_kv_map(CUtensorMap* map, const void* ptr, const Dims& m, int box_rows) {
+  auto fn = tmap_encoder();
+  if (!fn) return SPARSEPR_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)m.d, (cuuint64_t)m.Nk, (cuuint64_t)m.Hk};
+  const cuuint64_t strides[2] = {(cuuint64_t)m.d * 2, (cuuint64_t)m.Nk * m.d * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+             ? SPARSEPR_OK
+             : SPARSEPR_ERR_ARG;
+}
+
 template <int D>
-sparsepr_status launch_tc(const TcArgs& args, dim3 grid, cudaStream_t st) {
+sparsepr_status launch_tc(TcArgs args, dim3 grid, cudaStream_t st) {
+  if (args.mode != kModeSparse) {
+    sparsepr_status s = make_kv_map(&args.tm_k, args.K, args.m, 64);
+    if (s == SPARSEPR_OK) s = make_kv_map(&args.tm_v, args.V, args.m, 64);
+    if (s != SPARSEPR_OK) return s;
+  }
   const size_t smem = Layout<D>::kBytes + 1024;
   SPR_CUDA_OK(cudaFuncSetAttribute(attention_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   attention_tc_kernel<D><<<grid, kTcThreads, smem, st>>>(args);

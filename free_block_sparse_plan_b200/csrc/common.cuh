@@ -54,6 +54,7 @@ struct Buffers {
   int *histK, *histQ;
   int *permK, *permQ, *invQ;
   int *offK, *offQ;          // raw-label offsets [H][C+1]
+  int *poffK;                // tensor-core K/V layout: padded raw-label row offsets [H_k][C_k+1]
   int *kmK, *kmQ;            // per-head k-means state [H][4]: done, changed, iters, -
   double *objK, *objQ;       // per-cluster objective partials [H][C]
   double *objH;              // [H][2] final objectives
@@ -67,7 +68,8 @@ struct Buffers {
   int *rankPref;             // calibrated budget: key counts of each score-ranked prefix [H][Cq][Ck]
   double *betaH;             // budget each head's routing used [H]
   long long *pairs;          // [H]
-  void *Qp, *Kp, *Vp;        // group-major copies [H][N][d]
+  void *Qp, *Kp, *Vp;        // group-major copies [H][N][d]; K/V in the tensor-core layout
+                             // (kv_tiled_rows) when that engine runs
   double *dist;              // [H][Nq]
   int *probeTop;             // [H][Cq][M]
   int *probes, *probeA, *mA; // [H][M], [H][M], [H][Cq]
@@ -156,6 +158,12 @@ void count_launch();
   } while (0)
 
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Rows per K/V head of the tensor-core K/V layout: every group's rows padded to a multiple
+// of 8 (at most 7 rows per group), then 128 zero rows.  The layout holds per K/V head the
+// 64-column panels one after the other ([panel][row][64] bf16, 128-byte rows), with the
+// 16-byte chunks of panel row p stored in the order chunk ^ (p & 7).
+__host__ __device__ inline long long kv_tiled_rows(int Nk, int Ck) { return (long long)Nk + 7LL * Ck + 128; }
 
 // ---------------------------------------------------------------------------------
 // Device utilities

@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace spr {
 namespace {
@@ -646,23 +647,9 @@ __global__ void __launch_bounds__(256) km_split_c_kernel(const double* cent, int
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // [rows][64] bf16 with 128-byte rows, copied in boxes of box_rows x 64, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, long long rows, int box_rows) {
-  auto fn = encode_fn();
+  auto fn = tmap_encoder();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kKP, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)kKP * 2};

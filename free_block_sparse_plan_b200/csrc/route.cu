@@ -321,6 +321,66 @@ __global__ void gather_kernel(const void* src, void* dst, const int* perm, int* 
   }
 }
 
+// Padded row offsets of the K/V groups in the tensor-core layout: each group's rows rounded
+// up to a multiple of 8, in raw-label order; entry C_k is where the 128 zero rows start.
+__global__ void __launch_bounds__(1024) kv_pad_offsets_kernel(Dims m, Buffers b) {
+  __shared__ int sh[32];
+  const long long o = (long long)blockIdx.x * (m.Ck + 1);
+  const int lab = threadIdx.x;
+  const int sz = lab < m.Ck ? b.offK[o + lab + 1] - b.offK[o + lab] : 0;
+  int tot;
+  const int ex = block_exclusive_scan((sz + 7) & ~7, sh, &tot);
+  if (lab < m.Ck) b.poffK[o + lab] = ex;
+  if (lab == 0) b.poffK[o + m.Ck] = tot;
+}
+
+// K and V rows into the tensor-core layout (kv_tiled_rows): group-major position `pos` of
+// K/V head hk goes to panel row poffK[label] + (pos - offK[label]), each 16-byte chunk at
+// its swizzled place.
+__global__ void kv_tiled_kernel(Dims m, Buffers b, const uint4* K, const uint4* V, uint4* Kt, uint4* Vt) {
+  const int chunks = m.d / 8, np = m.d / 64;
+  const long long rp = kv_tiled_rows(m.Nk, m.Ck);
+  const long long total = (long long)m.Hk * m.Nk * chunks;
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const long long row = t / chunks;                  // hk * N_k + pos
+    const int c = (int)(t % chunks);
+    const int hk = (int)(row / m.Nk), pos = (int)(row - (long long)hk * m.Nk);
+    const int srow = b.permK[row];
+    const int lab = b.labK[(long long)hk * m.Nk + srow];
+    const long long o = (long long)hk * (m.Ck + 1) + lab;
+    const long long prow = b.poffK[o] + (pos - b.offK[o]);
+    const long long src = ((long long)hk * m.Nk + srow) * chunks + c;
+    const long long dst = (((long long)hk * np + (c >> 3)) * rp + prow) * 8 + ((c & 7) ^ (int)(prow & 7));
+    Kt[dst] = __ldg(K + src);
+    Vt[dst] = __ldg(V + src);
+  }
+}
+
+// Zero rows of the tensor-core layout: the padding after each group (block x < C_k) and the
+// 128 rows after the last group (block x = C_k), for every panel of K/V head blockIdx.y.
+__global__ void kv_tiled_zero_kernel(Dims m, Buffers b, uint4* Kt, uint4* Vt) {
+  const int hk = blockIdx.y, lab = blockIdx.x, np = m.d / 64;
+  const long long rp = kv_tiled_rows(m.Nk, m.Ck);
+  const long long o = (long long)hk * (m.Ck + 1) + lab;
+  long long r0, r1;
+  if (lab < m.Ck) {
+    r0 = b.poffK[o] + (b.offK[o + 1] - b.offK[o]);
+    r1 = b.poffK[o + 1];
+  } else {
+    r0 = b.poffK[o];
+    r1 = r0 + 128;
+  }
+  const int n = (int)(r1 - r0) * np * 8;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int pnl = e / ((int)(r1 - r0) * 8), rem = e % ((int)(r1 - r0) * 8);
+    const long long dst = (((long long)hk * np + pnl) * rp + r0) * 8 + rem;
+    Kt[dst] = z;
+    Vt[dst] = z;
+  }
+}
+
 // Squared distance of each query's phi_Q to its group centre (fp64, ascending dims).
 __global__ void probe_dist_kernel(Dims m, Buffers b) {
   const int h = blockIdx.y;
@@ -469,6 +529,17 @@ sparsepr_status launch_permute(const Plan& p, cudaStream_t st) {
   const int blocks = 148 * 8;
   gather_kernel<<<blocks, 256, 0, st>>>(p.Q, p.b.Qp, p.b.permQ, p.b.invQ, m.H, m.Nq, chunks);
   SPR_LAUNCH_OK();
+  if (tc_engine_applies(m.dtype, m.d, m.engine)) {
+    kv_pad_offsets_kernel<<<m.Hk, 1024, 0, st>>>(m, p.b);
+    SPR_LAUNCH_OK();
+    kv_tiled_kernel<<<blocks, 256, 0, st>>>(m, p.b, static_cast<const uint4*>(p.K), static_cast<const uint4*>(p.V),
+                                            static_cast<uint4*>(p.b.Kp), static_cast<uint4*>(p.b.Vp));
+    SPR_LAUNCH_OK();
+    kv_tiled_zero_kernel<<<dim3(m.Ck + 1, m.Hk), 128, 0, st>>>(m, p.b, static_cast<uint4*>(p.b.Kp),
+                                                                static_cast<uint4*>(p.b.Vp));
+    SPR_LAUNCH_OK();
+    return SPARSEPR_OK;
+  }
   gather_kernel<<<blocks, 256, 0, st>>>(p.K, p.b.Kp, p.b.permK, nullptr, m.Hk, m.Nk, chunks);
   SPR_LAUNCH_OK();
   gather_kernel<<<blocks, 256, 0, st>>>(p.V, p.b.Vp, p.b.permK, nullptr, m.Hk, m.Nk, chunks);
