@@ -95,6 +95,8 @@ struct Misc {
   int cbase[kMaxC];           // its first row in the tensor-core K/V layout of the head
   int clen[kMaxC];            // its true length (the rest up to the next position is padding)
   uint32_t kvmask[4][4];      // per stage: key columns that are padding
+  float xm[2][kTileRows];     // alternating mode: running max and sum of each half
+  float xl[2][kTileRows];
   uint32_t tmem_base;
   int abort_flag;
   int sh[32];
@@ -183,6 +185,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
   const int nt = (int)((nkeys + kTileKeys - 1) / kTileKeys);
   const int last_valid = (int)(nkeys - (long long)(nt - 1) * kTileKeys);
   const bool hasB = nrows > kTileRows;
+  // one query tile and two or more key tiles: the even and the odd key tiles go to two
+  // softmax warp groups with their own S buffer, running max and O accumulator, merged at
+  // the end, so that one group's softmax overlaps the other's products
+  const bool alt = !hasB && nt >= 2;
 
   // ---------------------------------------------------------------- setup
   const uint32_t bars = tc::smem_u32(ms->bars);
@@ -271,16 +277,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
             }
           };
           while (c < cnt && ms->csum[c + 1] <= t0) ++c;
-          // the padding columns of this tile, published before the stage's barrier
-          // (whose arrive releases them to the softmax warps)
-          uint32_t* mask = ms->kvmask[s];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) mask[q] = 0u;
-          for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
-            const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
-            for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
-          }
-          tc::mbar_expect_tx(bar, 2u * L::kTile);
+          tc::mbar_add_tx(bar, 2u * L::kTile);
           int pos = t0;                                   // next tile position to fill
           for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
             const int lo = max(ms->csum[cc], t0), hi = min(ms->csum[cc + 1], t0 + kTileKeys);
@@ -288,6 +285,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
             pos = hi;
           }
           if (pos < t0 + kTileKeys) copy_run(zrow, pos - t0, t0 + kTileKeys - pos);
+          // the padding columns of this tile, published by the arrive (a release) that
+          // follows the copies
+          uint32_t* mask = ms->kvmask[s];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mask[q] = 0u;
+          for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
+            const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
+            for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
+          }
+          tc::mbar_arrive(bar);
         } else {
           tc::mbar_expect_tx(bar, 2u * L::kTile);
           const int first = (g.mode == kModeProbe ? split * kProbeSplit : 0) + t0;
@@ -320,12 +327,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         tc::mma_commit(BAR(bSFull0 + buf));
       };
       // O_t += P V_j with P in S buffer `buf`
-      auto issue_pv = [&](int t, int j, int buf) {
+      auto issue_pv = [&](int t, int j, int buf, bool acc) {
         const int s = j % L::S;
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk) {
           const uint64_t bd = tc::sw128_desc(sV(s) + kk * 2048, L::kPanel, 1024);
-          tc::mma_ts(tmem + 256 + 128 * t, tmem + 128 * buf + 8 * kk, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tmem + 256 + 128 * t, tmem + 128 * buf + 8 * kk, bd, idPV, (acc || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(BAR(bPvDone0 + t));
       };
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         for (int j = 0; ok && j < nt; ++j) {
           if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
-          issue_pv(0, j, 0);
+          issue_pv(0, j, 0, j > 0);
           const bool more = j + 1 < nt;
           if (more) {
             if (!kv_ready(j + 1)) { ok = false; break; }
@@ -355,9 +362,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
           }
           if (!wait_bar(ms, BAR(bPFull0 + 1), j & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
-          issue_pv(1, j, 1);
+          issue_pv(1, j, 1, j > 0);
           tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
           if (more) issue_s(1, j + 1, 1);
+        }
+      } else if (alt) {
+        // one query tile, key tile j into S buffer and O accumulator j & 1; S(j+2) follows
+        // PV(j) in the same buffer, so its completion also means O is updated
+        if (ok) {
+          tc::fence_after_sync();
+          issue_s(0, 0, 0);
+          ok = kv_ready(1);
+          if (ok) {
+            tc::fence_after_sync();
+            issue_s(0, 1, 1);
+          }
+        }
+        for (int j = 0; ok && j < nt; ++j) {
+          const int u = j & 1;
+          if (!wait_bar(ms, BAR(bPFull0 + u), (j >> 1) & 1, g.err)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_pv(u, j, u, j > 1);
+          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
+          if (j + 2 < nt) {
+            if (!kv_ready(j + 2)) { ok = false; break; }
+            tc::fence_after_sync();
+            issue_s(0, j + 2, u);
+          }
         }
       } else {
         // one query tile: S alternates between the two S buffers, so S(j+1) is ready
@@ -377,7 +408,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
           const int buf = j & 1;
           if (!wait_bar(ms, BAR(bPFull0 + buf), (j >> 1) & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
-          issue_pv(0, j, buf);
+          issue_pv(0, j, buf, j > 0);
           tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
           if (j + 2 < nt) {
             if (!kv_ready(j + 2)) { ok = false; break; }
@@ -395,22 +426,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
       }
     }
     __syncwarp();
-  } else if (warp < 8 && (warp < 4 || hasB)) {
+  } else if (warp < 8 && (warp < 4 || hasB || alt)) {
     // ============================================================ softmax / epilogue
-    const int t = warp >> 2;                            // query tile
+    const int t = warp >> 2;                            // query tile (alternating mode: half)
     const int r = tid - 128 * t;                        // its row = TMEM lane
+    const int row0 = alt ? 0 : kTileRows * t;           // the tile's first row in the item
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tO = tmem + 256 + 128 * t + lane_off;
     const float sl2 = 1.4426950408889634f / sqrtf((float)d);
     // a warp none of whose 32 rows is a query row of the item (a group's tail tile) only
     // keeps the barrier phases: its rows read zero-filled Q, their results are not stored,
     // and the issue slots and special-function throughput go to the warps that have rows
-    const bool idle = kTileRows * t + 32 * (warp & 3) >= nrows;
+    const bool idle = row0 + 32 * (warp & 3) >= nrows;
+    const bool live = row0 + r < nrows;                 // a query row of the item
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      // S buffer: the tile's own with two tiles, alternating with one
-      const int buf = hasB ? t : (j & 1);
+    for (int j = alt ? t : 0; j < nt; j += alt ? 2 : 1) {
+      // S buffer: the tile's (half's) own with two tiles or halves, alternating with one
+      const int buf = (hasB || alt) ? t : (j & 1);
       const uint32_t sfp = hasB ? (j & 1) : ((j >> 1) & 1);
       const uint32_t tS = tmem + 128 * buf + lane_off;
       if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bSFull0 + buf), sfp, g.err))) { ok = false; break; }
@@ -420,60 +453,73 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         tc::mbar_arrive(BAR(bPFull0 + buf));
         continue;
       }
+      // sparse: padding columns of the tile (rows of no selected range; their K and V rows
+      // are zero, so S = 0 there and they add nothing to O).  The stage's barrier phase of
+      // tile j has completed (S(j) was computed from it); waiting on it acquires the
+      // producer's mask words.
+      uint32_t pw[4] = {0u, 0u, 0u, 0u};
       if (g.mode == kModeSparse) {
-        // padding columns of the tile (their rows belong to no selected range): -inf in S.
-        // The stage's barrier phase of tile j has completed (S(j) was computed from it);
-        // waiting on it acquires the producer's mask words.
         if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bKVFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
-        const int s = j % L::S;
-        bool any = false;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pw[q] = ms->kvmask[j % L::S][q];
+      }
+      const bool padded = (pw[0] | pw[1] | pw[2] | pw[3]) != 0u;     // uniform
+      const int valid = (j == nt - 1) ? last_valid : kTileKeys;
+      const bool whole = valid == kTileKeys;           // uniform: no key column past the keys
+      // The padding columns' S = 0 only decides the max where no key column of a query row
+      // exceeds 0.  Then (rare) they are set to -inf and the max taken again; otherwise
+      // their exp terms, whose values are known and below the row's largest term, come off
+      // the row sum after the tile.
+      float mx;
+      bool pad_in_sum = padded;
+#pragma unroll 1
+      for (int pass = 0;; ++pass) {
+        mx = -INFINITY;
+        if (whole) {
+          // two 32-column loads per wait, four independent three-operand max chains
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 4; c += 2) {
+            float v[64];
+            tc::tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(v));
+            tc::tmem_ld32(tS + 32 * c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) m4[(i >> 1) & 3] = tc::fmax3(m4[(i >> 1) & 3], v[i], v[i + 1]);
+          }
+          mx = tc::fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tc::tmem_ld32(tS + 32 * c, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * c + i < valid) mx = fmaxf(mx, v[i]);
+          }
+        }
+        if (pass > 0 || !padded || !__any_sync(0xffffffffu, !(mx > 0.0f) && live)) break;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t mw = ms->kvmask[s][q];
-          any |= mw != 0u;
+          uint32_t mw = pw[q];
           while (mw) {                                    // uniform across the warp
             const int col = 32 * q + __ffs(mw) - 1;
             mw &= mw - 1;
             tc::tmem_st1(tS + col, __float_as_uint(-INFINITY));
           }
         }
-        if (any) tc::tmem_wait_st();
+        tc::tmem_wait_st();
+        pad_in_sum = false;
       }
-      const int valid = (j == nt - 1) ? last_valid : kTileKeys;
-      const bool whole = valid == kTileKeys;           // uniform: no key column masked
-      float mx = -INFINITY;
       float rs = 0.0f;
-      if (whole) {
-        // two 32-column loads per wait, four independent three-operand max chains
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 4; c += 2) {
-          float v[64];
-          tc::tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(v));
-          tc::tmem_ld32(tS + 32 * c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 64; i += 2) m4[(i >> 1) & 3] = tc::fmax3(m4[(i >> 1) & 3], v[i], v[i + 1]);
-        }
-        mx = tc::fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(tS + 32 * c, v);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i < valid) mx = fmaxf(mx, v[i]);
-        }
-      }
       const float m_tile = mx * sl2;
       // lazy rescale: keep the running max unless it grows by more than 2^8
       if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleLog2)) {
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = tc::ex2(m_run - m_new);     // 0 on the first tile
         // one tile: S(j) may be ready before PV(j-1) has finished updating O
-        if (!hasB && j > 0 && !__all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone0), (j - 1) & 1, g.err))) {
+        if (!hasB && !alt && j > 0 && !__all_sync(0xffffffffu, wait_bar(ms, BAR(bPvDone0), (j - 1) & 1, g.err))) {
           ok = false;
           break;
         }
@@ -545,20 +591,73 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         }
       }
       tc::tmem_wait_st();
+      if (pad_in_sum) {
+        // the padding columns' terms: exp2(0 * scale - m_run), on the special-function
+        // unit or the polynomial as their column position decided
+        constexpr uint32_t kPolyCols = ~0u << (32 - 2 * kPolyPairs);   // per 32-column word
+        int n_all = 0, n_poly = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          n_all += __popc(pw[q]);
+          n_poly += __popc(pw[q] & kPolyCols);
+        }
+        const float e_sfu = tc::ex2(-m_run);
+        if (whole) {
+          float e_poly, e_unused;
+          tc::exp2_poly2(-m_run, -m_run, e_poly, e_unused);
+          rs -= (float)(n_all - n_poly) * e_sfu + (float)n_poly * e_poly;
+        } else {
+          rs -= (float)n_all * e_sfu;
+        }
+      }
       l_run += rs;
       tc::fence_before_sync();
       tc::mbar_arrive(BAR(bPFull0 + buf));
     }
-    const bool oready = idle || (hasB ? wait_bar(ms, BAR(bPvDone0 + t), (nt - 1) & 1, g.err)
-                                      : wait_bar(ms, BAR(bOReady), 0, g.err));
-    if (ok && !idle && __all_sync(0xffffffffu, oready)) {
+    // PV commits on this tile's (half's) barrier: one per key tile it took
+    const int npv = alt ? (nt - t + 1) >> 1 : nt;
+    const bool oready = idle || ((hasB || alt) ? wait_bar(ms, BAR(bPvDone0 + t), (npv - 1) & 1, g.err)
+                                               : wait_bar(ms, BAR(bOReady), 0, g.err));
+    bool store = ok && !idle && __all_sync(0xffffffffu, oready);
+    // alternating mode: the two halves' running max and sum for every row, then each half
+    // writes half of the columns of the merged rows
+    float wA = 1.0f, wB = 0.0f;
+    int c0 = 0, c1 = D / 32;
+    if (alt) {
+      if (store) {
+        ms->xm[t][r] = m_run;
+        ms->xl[t][r] = l_run;
+      }
+      // every softmax thread of both halves arrives here exactly once
+      store = tc::named_sync_and(2, 256, store || idle) && store;
+      if (store) {
+        const float mA = ms->xm[0][r], mB = ms->xm[1][r];
+        m_run = fmaxf(mA, mB);
+        wA = tc::ex2(mA - m_run);
+        wB = tc::ex2(mB - m_run);
+        l_run = ms->xl[0][r] * wA + ms->xl[1][r] * wB;
+        c0 = t * (D / 64);
+        c1 = c0 + D / 64;
+      }
+    }
+    if (store) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
-      const int row = kTileRows * t + r;
-      for (int c = 0; c < D / 32; ++c) {
+      const int row = row0 + r;
+      const uint32_t tO0 = tmem + 256 + lane_off, tO1 = tmem + 384 + lane_off;
+      for (int c = c0; c < c1; ++c) {
         float o[32];
-        tc::tmem_ld32(tO + 32 * c, o);
-        tc::tmem_wait_ld();
+        if (alt) {
+          float o1[32];
+          tc::tmem_ld32(tO0 + 32 * c, o);
+          tc::tmem_ld32(tO1 + 32 * c, o1);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = o[i] * wA + o1[i] * wB;
+        } else {
+          tc::tmem_ld32(tO + 32 * c, o);
+          tc::tmem_wait_ld();
+        }
         if (row < nrows) {
           if (g.mode == kModeSparse) {
             float4* dst = reinterpret_cast<float4*>(g.b.Osp + ((long long)h * m.Nq + q0 + row) * d + 32 * c);
