@@ -89,7 +89,7 @@ struct Layout {
 };
 
 struct Misc {
-  unsigned long long bars[24];
+  unsigned long long bars[26];
   long long qrow[kItemRows];
   int csum[kMaxC + 1];        // sparse: key position of each selected range (multiples of 8)
   int cbase[kMaxC];           // its first row in the tensor-core K/V layout of the head
@@ -103,7 +103,8 @@ struct Misc {
 };
 
 enum Bar {
-  bQFull = 0, bKVFull0 = 1, bKVEmpty0 = 5, bSFull0 = 9, bPFull0 = 11, bPvDone0 = 13, bDrain = 15, bOReady = 16
+  bQFull = 0, bKFull0 = 1, bKEmpty0 = 5, bSFull0 = 9, bPFull0 = 11, bPvDone0 = 13, bDrain = 15, bOReady = 16,
+  bVFull0 = 17, bVEmpty0 = 21
 };
 
 // Bounded wait; the clock and the abort flag are read once every 32 polls so that
@@ -196,8 +197,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
   if (tid == 0) {
     tc::mbar_init(BAR(bQFull), kProducers);
     for (int s = 0; s < L::S; ++s) {
-      tc::mbar_init(BAR(bKVFull0 + s), 1);            // the copying thread's arrive + bytes
-      tc::mbar_init(BAR(bKVEmpty0 + s), 1);
+      tc::mbar_init(BAR(bKFull0 + s), 1);             // the copying thread's arrive + bytes
+      tc::mbar_init(BAR(bKEmpty0 + s), 1);
+      tc::mbar_init(BAR(bVFull0 + s), 1);
+      tc::mbar_init(BAR(bVEmpty0 + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(BAR(bSFull0 + s), 1);
@@ -246,38 +249,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
     tc::mbar_arrive(BAR(bQFull));
-    // K/V tiles: stage j % S, copied by one thread.  Sparse mode: one bulk copy per panel
-    // of every run of rows (the tensor-core layout holds each panel's rows in the order of
-    // the shared-memory tile, runs start at multiples of 8 rows on both sides); the rest of
-    // the last tile comes from the head's zero rows.  Dense and probe modes: TMA boxes of
-    // 64 rows (rows past N_k read as zeros; past the item's keys, the softmax masks them).
-    // Every row of a stage is written, so its byte count is fixed.
-    if (p == 0) {
+    // K and V tiles: stage j % S, K copied by one thread and V by another, each stage
+    // refilled as soon as the products reading it have finished (K after the S products,
+    // V after the PV products).  Sparse mode: one bulk copy per panel of every run of rows
+    // (the tensor-core layout holds each panel's rows in the order of the shared-memory
+    // tile, runs start at multiples of 8 rows on both sides); the rest of the last tile
+    // comes from the head's zero rows.  Dense and probe modes: TMA boxes of 64 rows (rows
+    // past N_k read as zeros; past the item's keys, the softmax masks them).  Every row of
+    // a stage is written, so its byte count is fixed.
+    if (p == 0 || p == 32) {
+      const bool isK = p == 0;
       const int hk = h / m.G;                             // the K/V head
       constexpr int NP = D / 64;
       const long long rp = kv_tiled_rows(m.Nk, m.Ck);
-      const uint8_t* Kt = reinterpret_cast<const uint8_t*>(g.K) + (long long)hk * NP * rp * 128;
-      const uint8_t* Vt = reinterpret_cast<const uint8_t*>(g.V) + (long long)hk * NP * rp * 128;
+      const uint8_t* src_base = reinterpret_cast<const uint8_t*>(isK ? g.K : g.V) + (long long)hk * NP * rp * 128;
+      const CUtensorMap* tmap = isK ? &g.tm_k : &g.tm_v;
       const int zrow = g.mode == kModeSparse ? g.b.poffK[(long long)hk * (m.Ck + 1) + m.Ck] : 0;
+      const int full0 = isK ? bKFull0 : bVFull0, empty0 = isK ? bKEmpty0 : bVEmpty0;
       int c = 0;                                          // sparse: current range
       for (int j = 0; j < nt; ++j) {
         const int s = j % L::S, use = j / L::S;
-        if (use > 0 && !wait_bar(ms, BAR(bKVEmpty0 + s), (use - 1) & 1, g.err)) break;
-        const uint32_t bar = BAR(bKVFull0 + s);
+        if (use > 0 && !wait_bar(ms, BAR(empty0 + s), (use - 1) & 1, g.err)) break;
+        const uint32_t bar = BAR(full0 + s);
+        const uint32_t tile = isK ? sK(s) : sV(s);
         const int t0 = j * kTileKeys;
         if (g.mode == kModeSparse) {
           // rows [src, src + len) of the layout into tile rows [dst, dst + len)
           auto copy_run = [&](long long src, int dst, int len) {
 #pragma unroll
-            for (int pnl = 0; pnl < NP; ++pnl) {
-              const uint32_t o = pnl * L::kPanel + (uint32_t)dst * 128u;
-              const long long so = ((long long)pnl * rp + src) * 128;
-              tc::bulk_g2s(sK(s) + o, Kt + so, (uint32_t)len * 128u, bar);
-              tc::bulk_g2s(sV(s) + o, Vt + so, (uint32_t)len * 128u, bar);
-            }
+            for (int pnl = 0; pnl < NP; ++pnl)
+              tc::bulk_g2s(tile + pnl * L::kPanel + (uint32_t)dst * 128u, src_base + ((long long)pnl * rp + src) * 128,
+                           (uint32_t)len * 128u, bar);
           };
           while (c < cnt && ms->csum[c + 1] <= t0) ++c;
-          tc::mbar_add_tx(bar, 2u * L::kTile);
+          tc::mbar_add_tx(bar, L::kTile);
           int pos = t0;                                   // next tile position to fill
           for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
             const int lo = max(ms->csum[cc], t0), hi = min(ms->csum[cc + 1], t0 + kTileKeys);
@@ -285,27 +290,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
             pos = hi;
           }
           if (pos < t0 + kTileKeys) copy_run(zrow, pos - t0, t0 + kTileKeys - pos);
-          // the padding columns of this tile, published by the arrive (a release) that
-          // follows the copies
-          uint32_t* mask = ms->kvmask[s];
+          if (isK) {
+            // the padding columns of this tile, published by the arrive (a release) that
+            // follows the copies
+            uint32_t* mask = ms->kvmask[s];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) mask[q] = 0u;
-          for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
-            const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
-            for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
+            for (int q = 0; q < 4; ++q) mask[q] = 0u;
+            for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
+              const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
+              for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
+            }
           }
           tc::mbar_arrive(bar);
         } else {
-          tc::mbar_expect_tx(bar, 2u * L::kTile);
+          tc::mbar_expect_tx(bar, L::kTile);
           const int first = (g.mode == kModeProbe ? split * kProbeSplit : 0) + t0;
 #pragma unroll
           for (int half = 0; half < 2; ++half)
 #pragma unroll
-            for (int pnl = 0; pnl < NP; ++pnl) {
-              const uint32_t o = pnl * L::kPanel + (uint32_t)half * 64u * 128u;
-              tc::tma_load_3d(sK(s) + o, &g.tm_k, 64 * pnl, first + 64 * half, hk, bar);
-              tc::tma_load_3d(sV(s) + o, &g.tm_v, 64 * pnl, first + 64 * half, hk, bar);
-            }
+            for (int pnl = 0; pnl < NP; ++pnl)
+              tc::tma_load_3d(tile + pnl * L::kPanel + (uint32_t)half * 64u * 128u, tmap, 64 * pnl, first + 64 * half, hk, bar);
         }
       }
     }
@@ -336,87 +340,71 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         }
         tc::mma_commit(BAR(bPvDone0 + t));
       };
-      // K/V stage j % S, fill j / S; the copies were made by the generic proxy
-      auto kv_ready = [&](int j) -> bool {
-        if (!wait_bar(ms, BAR(bKVFull0 + j % L::S), (j / L::S) & 1, g.err)) return false;
-        tc::fence_proxy_async();
+      // K or V stage j % S, fill j / S
+      auto k_ready = [&](int j) -> bool {
+        if (!wait_bar(ms, BAR(bKFull0 + j % L::S), (j / L::S) & 1, g.err)) return false;
+        tc::fence_after_sync();
         return true;
       };
-      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && kv_ready(0);
+      auto v_ready = [&](int j) -> bool {
+        if (!wait_bar(ms, BAR(bVFull0 + j % L::S), (j / L::S) & 1, g.err)) return false;
+        tc::fence_after_sync();
+        return true;
+      };
+      bool ok = wait_bar(ms, BAR(bQFull), 0, g.err) && k_ready(0);
       if (hasB) {
         // two query tiles: the softmax of one overlaps the products of the other
         if (ok) {
-          tc::fence_after_sync();
           issue_s(0, 0, 0);
           issue_s(1, 0, 1);
+          tc::mma_commit(BAR(bKEmpty0));
         }
         for (int j = 0; ok && j < nt; ++j) {
-          if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err)) { ok = false; break; }
-          tc::fence_after_sync();
+          if (!wait_bar(ms, BAR(bPFull0), j & 1, g.err) || !v_ready(j)) { ok = false; break; }
           issue_pv(0, j, 0, j > 0);
           const bool more = j + 1 < nt;
           if (more) {
-            if (!kv_ready(j + 1)) { ok = false; break; }
-            tc::fence_after_sync();
+            if (!k_ready(j + 1)) { ok = false; break; }
             issue_s(0, j + 1, 0);
           }
           if (!wait_bar(ms, BAR(bPFull0 + 1), j & 1, g.err)) { ok = false; break; }
           tc::fence_after_sync();
           issue_pv(1, j, 1, j > 0);
-          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
-          if (more) issue_s(1, j + 1, 1);
-        }
-      } else if (alt) {
-        // one query tile, key tile j into S buffer and O accumulator j & 1; S(j+2) follows
-        // PV(j) in the same buffer, so its completion also means O is updated
-        if (ok) {
-          tc::fence_after_sync();
-          issue_s(0, 0, 0);
-          ok = kv_ready(1);
-          if (ok) {
-            tc::fence_after_sync();
-            issue_s(0, 1, 1);
-          }
-        }
-        for (int j = 0; ok && j < nt; ++j) {
-          const int u = j & 1;
-          if (!wait_bar(ms, BAR(bPFull0 + u), (j >> 1) & 1, g.err)) { ok = false; break; }
-          tc::fence_after_sync();
-          issue_pv(u, j, u, j > 1);
-          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
-          if (j + 2 < nt) {
-            if (!kv_ready(j + 2)) { ok = false; break; }
-            tc::fence_after_sync();
-            issue_s(0, j + 2, u);
+          tc::mma_commit(BAR(bVEmpty0 + j % L::S));
+          if (more) {
+            issue_s(1, j + 1, 1);
+            tc::mma_commit(BAR(bKEmpty0 + (j + 1) % L::S));
           }
         }
       } else {
-        // one query tile: S alternates between the two S buffers, so S(j+1) is ready
-        // while the softmax of tile j runs
+        // one query tile, S alternating between the two S buffers so that S(j+1) is ready
+        // while the softmax of tile j runs.  Alternating mode: key tile j also into O
+        // accumulator j & 1, with its own softmax warp group; S(j+2) follows PV(j) in the
+        // same buffer, so its completion also means that accumulator is updated
         if (ok) {
-          tc::fence_after_sync();
           issue_s(0, 0, 0);
+          tc::mma_commit(BAR(bKEmpty0));
           if (nt > 1) {
-            ok = kv_ready(1);
+            ok = k_ready(1);
             if (ok) {
-              tc::fence_after_sync();
               issue_s(0, 1, 1);
+              tc::mma_commit(BAR(bKEmpty0 + 1 % L::S));
             }
           }
         }
         for (int j = 0; ok && j < nt; ++j) {
           const int buf = j & 1;
-          if (!wait_bar(ms, BAR(bPFull0 + buf), (j >> 1) & 1, g.err)) { ok = false; break; }
-          tc::fence_after_sync();
-          issue_pv(0, j, buf, j > 0);
-          tc::mma_commit(BAR(bKVEmpty0 + j % L::S));
+          if (!wait_bar(ms, BAR(bPFull0 + buf), (j >> 1) & 1, g.err) || !v_ready(j)) { ok = false; break; }
+          if (alt) issue_pv(buf, j, buf, j > 1);
+          else issue_pv(0, j, buf, j > 0);
+          tc::mma_commit(BAR(bVEmpty0 + j % L::S));
           if (j + 2 < nt) {
-            if (!kv_ready(j + 2)) { ok = false; break; }
-            tc::fence_after_sync();
+            if (!k_ready(j + 2)) { ok = false; break; }
             issue_s(0, j + 2, buf);
+            tc::mma_commit(BAR(bKEmpty0 + (j + 2) % L::S));
           }
         }
-        if (ok) tc::mma_commit(BAR(bOReady));
+        if (ok && !alt) tc::mma_commit(BAR(bOReady));
       }
       tc::mma_commit(BAR(bDrain));
       // bounded: completes when every MMA issued above has finished
@@ -459,7 +447,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
       // producer's mask words.
       uint32_t pw[4] = {0u, 0u, 0u, 0u};
       if (g.mode == kModeSparse) {
-        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bKVFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bKFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
 #pragma unroll
         for (int q = 0; q < 4; ++q) pw[q] = ms->kvmask[j % L::S][q];
       }
