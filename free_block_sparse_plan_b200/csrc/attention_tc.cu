@@ -290,9 +290,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
             pos = hi;
           }
           if (pos < t0 + kTileKeys) copy_run(zrow, pos - t0, t0 + kTileKeys - pos);
-          if (isK) {
-            // the padding columns of this tile, published by the arrive (a release) that
-            // follows the copies
+          if (!isK) {
+            // the padding columns of this tile, published by the V stage's arrive (a
+            // release) that follows the copies.  The V stage is refilled only after the PV
+            // products of this tile, i.e. after every softmax warp has read the words
             uint32_t* mask = ms->kvmask[s];
 #pragma unroll
             for (int q = 0; q < 4; ++q) mask[q] = 0u;
@@ -442,12 +443,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         continue;
       }
       // sparse: padding columns of the tile (rows of no selected range; their K and V rows
-      // are zero, so S = 0 there and they add nothing to O).  The stage's barrier phase of
-      // tile j has completed (S(j) was computed from it); waiting on it acquires the
-      // producer's mask words.
+      // are zero, so S = 0 there and they add nothing to O).  Waiting on the V stage's
+      // barrier phase of tile j acquires the producer's mask words; that phase cannot be
+      // followed by the next one before this warp's P of tile j is consumed.
       uint32_t pw[4] = {0u, 0u, 0u, 0u};
       if (g.mode == kModeSparse) {
-        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bKFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bVFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
 #pragma unroll
         for (int q = 0; q < 4; ++q) pw[q] = ms->kvmask[j % L::S][q];
       }
