@@ -89,12 +89,12 @@ struct Layout {
 };
 
 struct Misc {
-  unsigned long long bars[26];
+  unsigned long long bars[34];
   long long qrow[kItemRows];
   int csum[kMaxC + 1];        // sparse: key position of each selected range (multiples of 8)
   int cbase[kMaxC];           // its first row in the tensor-core K/V layout of the head
   int clen[kMaxC];            // its true length (the rest up to the next position is padding)
-  uint32_t kvmask[4][4];      // per stage: key columns that are padding
+  uint32_t kvmask[8][4];      // sparse: key columns that are padding, tile j in slot j % 2S
   float xm[2][kTileRows];     // alternating mode: running max and sum of each half
   float xl[2][kTileRows];
   uint32_t tmem_base;
@@ -102,9 +102,11 @@ struct Misc {
   int sh[32];
 };
 
+static_assert(sizeof(Misc) <= 17 * 1024, "bookkeeping exceeds its shared-memory slot");
+
 enum Bar {
   bQFull = 0, bKFull0 = 1, bKEmpty0 = 5, bSFull0 = 9, bPFull0 = 11, bPvDone0 = 13, bDrain = 15, bOReady = 16,
-  bVFull0 = 17, bVEmpty0 = 21
+  bVFull0 = 17, bVEmpty0 = 21, bMask0 = 25
 };
 
 // Bounded wait; the clock and the abort flag are read once every 32 polls so that
@@ -202,6 +204,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
       tc::mbar_init(BAR(bVFull0 + s), 1);
       tc::mbar_init(BAR(bVEmpty0 + s), 1);
     }
+    for (int q = 0; q < 2 * L::S; ++q) tc::mbar_init(BAR(bMask0 + q), 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(BAR(bSFull0 + s), 1);
       tc::mbar_init(BAR(bPFull0 + s), 128);
@@ -290,19 +293,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
             pos = hi;
           }
           if (pos < t0 + kTileKeys) copy_run(zrow, pos - t0, t0 + kTileKeys - pos);
-          if (!isK) {
-            // the padding columns of this tile, published by the V stage's arrive (a
-            // release) that follows the copies.  The V stage is refilled only after the PV
-            // products of this tile, i.e. after every softmax warp has read the words
-            uint32_t* mask = ms->kvmask[s];
+          tc::mbar_arrive(bar);
+          if (isK) {
+            // the padding columns of this tile into mask slot j % 2S, published by that
+            // slot's barrier (an arrive is a release).  The slot's previous tile, j - 2S,
+            // was read by its softmax warps before the S products of tile j - S were
+            // issued, and this thread has waited for those products to finish
+            const int slot = j % (2 * L::S);
+            uint32_t* mask = ms->kvmask[slot];
 #pragma unroll
             for (int q = 0; q < 4; ++q) mask[q] = 0u;
             for (int cc = c; cc < cnt && ms->csum[cc] < t0 + kTileKeys; ++cc) {
               const int hi = min(ms->csum[cc + 1], t0 + kTileKeys);
               for (int q = max(ms->csum[cc] + ms->clen[cc], t0); q < hi; ++q) mask[(q - t0) >> 5] |= 1u << ((q - t0) & 31);
             }
+            tc::mbar_arrive(BAR(bMask0 + slot));
           }
-          tc::mbar_arrive(bar);
         } else {
           tc::mbar_expect_tx(bar, L::kTile);
           const int first = (g.mode == kModeProbe ? split * kProbeSplit : 0) + t0;
@@ -443,14 +449,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attention_tc_kernel(const __gri
         continue;
       }
       // sparse: padding columns of the tile (rows of no selected range; their K and V rows
-      // are zero, so S = 0 there and they add nothing to O).  Waiting on the V stage's
-      // barrier phase of tile j acquires the producer's mask words; that phase cannot be
-      // followed by the next one before this warp's P of tile j is consumed.
+      // are zero, so S = 0 there and they add nothing to O).  Waiting on the mask slot's
+      // barrier phase of tile j acquires the producer's words; the slot's next phase
+      // (tile j + 2S) needs the S products of tile j + S, which follow this warp's P(j).
       uint32_t pw[4] = {0u, 0u, 0u, 0u};
       if (g.mode == kModeSparse) {
-        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bVFull0 + j % L::S), (j / L::S) & 1, g.err))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(ms, BAR(bMask0 + j % (2 * L::S)), (j / (2 * L::S)) & 1, g.err))) { ok = false; break; }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) pw[q] = ms->kvmask[j % L::S][q];
+        for (int q = 0; q < 4; ++q) pw[q] = ms->kvmask[j % (2 * L::S)][q];
       }
       const bool padded = (pw[0] | pw[1] | pw[2] | pw[3]) != 0u;     // uniform
       const int valid = (j == nt - 1) ? last_valid : kTileKeys;

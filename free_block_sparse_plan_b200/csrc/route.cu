@@ -54,18 +54,34 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
     const int a = e / d, j = e % d;
     qa[a * ld + j] = a < na ? b.qbar[((long long)h * m.Cq + a0 + a) * d + j] : 0.0;
   }
-  auto stage = [&](const double* src, int k0) {
-    __syncthreads();
-    for (int e = tid; e < kScoreK * d; e += blockDim.x) {
+  // chunks of kScoreK centroid rows go through registers into shared memory; the next
+  // chunk's loads are issued before the current chunk is used, so their latency overlaps
+  // the arithmetic
+  constexpr int kStage = kScoreK * kMaxD / 256;      // elements per thread (blockDim 256)
+  double pre[kStage];
+  auto fetch = [&](const double* src, int k0) {
+#pragma unroll
+    for (int i = 0; i < kStage; ++i) {
+      const int e = tid + 256 * i;
       const int kk = e / d, j = e % d;
-      kv[kk * ld + j] = k0 + kk < n ? src[(long long)(k0 + kk) * d + j] : 0.0;
+      pre[i] = (e < kScoreK * d && k0 + kk < n) ? src[(long long)(k0 + kk) * d + j] : 0.0;
+    }
+  };
+  auto put = [&]() {
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kStage; ++i) {
+      const int e = tid + 256 * i;
+      if (e < kScoreK * d) kv[(e / d) * ld + e % d] = pre[i];
     }
     __syncthreads();
   };
   const int ta = tid >> 5, tk = tid & 31;   // phases 1 and 4: thread = (query group, row)
   // ---- phase 1: logits l_ab = tau qbar_a . kbar_b + ln |G_b|
+  fetch(kb, 0);
   for (int k0 = 0; k0 < n; k0 += kScoreK) {
-    stage(kb, k0);
+    put();
+    if (k0 + kScoreK < n) fetch(kb, k0 + kScoreK);
     const int k = k0 + tk;
     if (ta < na && k < n) {
       // four independent partial sums (d is a multiple of 8): a quarter of the latency
@@ -119,8 +135,10 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
   double acc_h[kJ], acc_r[kJ];
 #pragma unroll
   for (int i = 0; i < kJ; ++i) acc_h[i] = acc_r[i] = 0.0;
+  fetch(vb, 0);
   for (int k0 = 0; k0 < n; k0 += kScoreK) {
-    stage(vb, k0);
+    put();
+    if (k0 + kScoreK < n) fetch(vb, k0 + kScoreK);
     if (ta < na) {
       const int kn = min(kScoreK, n - k0);
       for (int kk = 0; kk < kn; ++kk) {
@@ -149,8 +167,10 @@ __global__ void __launch_bounds__(256) score_kernel(Dims m, Buffers b) {
     }
   }
   // ---- phase 4: score_ab = pi_ab ||vbar_b - ohat_a^(-b)||
+  fetch(vb, 0);
   for (int k0 = 0; k0 < n; k0 += kScoreK) {
-    stage(vb, k0);
+    put();
+    if (k0 + kScoreK < n) fetch(vb, k0 + kScoreK);
     const int k = k0 + tk;
     if (ta < na && k < n) {
       const bool istop = k == sTop[ta];
