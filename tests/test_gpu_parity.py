@@ -580,6 +580,35 @@ def test_affine_fit_matches_oracle(name):
 
 
 # ---------------------------------------------------------------------------------- edges
+def test_negative_logits_padding_columns_masked():
+    # Every query-key logit below zero: the zero K rows that pad each K/V group to a
+    # multiple of 8 in the tensor-core layout score 0 and would decide the row max, so the
+    # kernel masks them in TMEM and takes the max again (the path other data rarely take).
+    # bf16, d = 64, oracle labels injected; output and sparse output against the oracle.
+    w = W.TINY.with_(dtype="bf16", N=2048)
+    rng = np.random.default_rng(21)
+    mu = rng.standard_normal(w.d)
+    mu *= 8.0 / np.linalg.norm(mu)                          # |mu|^2 = 64
+    k = W.round_to_bf16(mu + 0.5 * rng.standard_normal((w.N, w.d)))
+    q = W.round_to_bf16(-0.5 * mu + 0.5 * rng.standard_normal((w.N, w.d)))
+    v = W.round_to_bf16(rng.standard_normal((w.N, w.d)))
+    assert (q @ k.T).max() < 0.0
+    p = O.Params.from_dict(w.params())
+    res = O.sparsepr_call(q, k, v, p, head=0, part=O.partition(q, k, v, p, 0))
+    assert np.any(res.part.gk.sizes % 8 != 0)               # some groups are padded
+    td = W.torch_dtype(w.dtype)
+    inputs = tuple(torch.from_numpy(a[None].astype(np.float32)).to(td).cuda() for a in (q, k, v))
+    labQ = torch.tensor(res.part.km_Q.labels[None], dtype=torch.int32, device="cuda")
+    labK = torch.tensor(res.part.km_K.labels[None], dtype=torch.int32, device="cuda")
+    plan, out, _ = gpu_call(w, inputs=inputs, labels=(labQ, labK))
+    assert plan.check() == 0
+    osp = plan.export("OSP")[0]
+    rows = np.empty_like(osp)
+    rows[plan.export("PERM_Q")[0]] = osp
+    assert rel(rows[res.rows], res.osp) < 1e-2
+    check_injected_head(plan, out[0].float().cpu().numpy(), res, 0, w)
+
+
 def test_full_density_returns_dense():
     # rho* = 1 with every group larger than M: every cell is selected, residuals vanish
     # and the whole call returns dense attention (paper S2: all cells recover dense).
