@@ -480,6 +480,10 @@ sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error) {
   return e ? SPARSEPR_ERR_DEVICE_CHECK : SPARSEPR_OK;
 }
 
+sparsepr_status sparsepr_wait_selftest(void* stream) {
+  return launch_wait_selftest(reinterpret_cast<cudaStream_t>(stream));
+}
+
 sparsepr_status sparsepr_check(sparsepr_plan_t plan, void* stream, int32_t* device_error) {
   if (!plan) return SPARSEPR_ERR_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -738,7 +738,28 @@ sparsepr_status with_tc_d(int d, F f) {
   return f(std::integral_constant<int, 128>());
 }
 
+// The failure path of the pipeline waits, on a healthy GPU: one warp waits through
+// wait_bar on a fresh barrier that nothing arrives on (no copy or product is in flight),
+// gives up after kWaitCycles (about one second) and records kErrHang in the error word of
+// the plan-free entry points.
+__global__ void __launch_bounds__(32) wait_selftest_kernel() {
+  __shared__ Misc ms;
+  const uint32_t bar = tc::smem_u32(&ms.bars[0]);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(bar, 1);
+    ms.abort_flag = 0;
+  }
+  __syncthreads();
+  (void)__all_sync(0xffffffffu, wait_bar(&ms, bar, 0, &g_dense_err));
+}
+
 }  // namespace
+
+sparsepr_status launch_wait_selftest(cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>();
+  SPR_LAUNCH_OK();
+  return SPARSEPR_OK;
+}
 
 sparsepr_status dense_error_address(int** out) {
   return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_dense_err) == cudaSuccess ? SPARSEPR_OK

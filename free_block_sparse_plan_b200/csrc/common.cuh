@@ -307,6 +307,7 @@ sparsepr_status launch_dense_attention(const Dims& dm, const void* Q, const void
 // Device addresses of the error words of the plan-free entry points on the current
 // device: sparsepr_dense_attention's, and the sticky word of sparsepr_dense_rows_noalloc.
 sparsepr_status dense_error_address(int** out);
+sparsepr_status launch_wait_selftest(cudaStream_t st);
 sparsepr_status noalloc_error_address(int** out);
 // O3 affine-fit diagnostic over a plan's sparse output (diagnostics.cu).
 sparsepr_status launch_affine_fit(const Plan& p, const void* dense, double* ws, double* explained,

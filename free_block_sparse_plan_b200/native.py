@@ -48,7 +48,7 @@ SYMBOLS = [
     "sparsepr_check", "sparsepr_get_stats", "sparsepr_export_size", "sparsepr_export",
     "sparsepr_destroy", "sparsepr_status_string", "sparsepr_dense_rows_noalloc",
     "sparsepr_launch_count", "sparsepr_state_size", "sparsepr_save_state", "sparsepr_plan_warm",
-    "sparsepr_dense_check", "sparsepr_support_workspace_size", "sparsepr_support_densities",
+    "sparsepr_dense_check", "sparsepr_wait_selftest", "sparsepr_support_workspace_size", "sparsepr_support_densities",
     "sparsepr_affine_workspace_size", "sparsepr_affine_fit",
 ]
 
@@ -104,6 +104,7 @@ def lib():
                                                    c_void_p]),
             "sparsepr_check": (c_int32, [c_void_p, c_void_p, POINTER(c_int32)]),
             "sparsepr_dense_check": (c_int32, [c_void_p, POINTER(c_int32)]),
+            "sparsepr_wait_selftest": (c_int32, [c_void_p]),
             "sparsepr_support_workspace_size": (c_int32, [P, c_int32, c_int32, POINTER(c_size_t)]),
             "sparsepr_support_densities": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_void_p,
                                                      c_int32, c_int32, c_double, c_void_p, c_size_t,
@@ -276,6 +277,12 @@ def sparsepr_dense_check(stream=None) -> int:
     if st not in (SPARSEPR_OK, SPARSEPR_ERR_DEVICE_CHECK):
         raise SparsePRError(st, "sparsepr_dense_check")
     return int(e.value)
+
+
+def wait_selftest(stream=None):
+    """Launches the bounded-wait self-test (a wait nothing completes gives up after about
+    one second and sets bit 32 of the word sparsepr_dense_check reads)."""
+    _check(lib().sparsepr_wait_selftest(stream), "sparsepr_wait_selftest")
 
 
 def support_densities(Q, K, rows, pool, npools, alpha=0.9, stream=None):

@@ -295,6 +295,14 @@ sparsepr_status sparsepr_dense_rows_noalloc(const sparsepr_params* params, const
  * other streams may set them after the read.  Allocates nothing. */
 sparsepr_status sparsepr_dense_check(void* stream, int32_t* device_error);
 
+/* The paper has no counterpart: a self-test of the failure path every tensor-core kernel
+ * takes when a pipeline wait gives up.  Launches, on `stream` and the current device, one
+ * warp that waits through the engines' bounded mbarrier wait on a barrier nothing ever
+ * completes, with no copy or product in flight; after about one second (2e9 SM clocks)
+ * the wait returns and sets bit 32 of the error word that sparsepr_dense_check reads.
+ * No fault, no hang: the warp then exits.  Asynchronous; allocates nothing. */
+sparsepr_status sparsepr_wait_selftest(void* stream);
+
 /*
  * Diagnostics of "Partition the Support, Reconstruct the Residual" S3 (observations O1,
  * O3), in fp64.  They measure a partition; they are not part of the attention call.

@@ -134,3 +134,16 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     st = N.lib().sparsepr_dense_rows_noalloc(ctypes.byref(many), Q.data_ptr(), K.data_ptr(),
                                              V.data_ptr(), rows.data_ptr(), 1, out.data_ptr(), None)
     assert st == N.SPARSEPR_ERR_SHAPE
+
+
+def test_bounded_wait_gives_up_and_reports_without_fault():
+    # A pipeline wait that nothing completes (no copy or product in flight): the self-test
+    # warp waits through the engines' bounded mbarrier wait, gives up after about one
+    # second and sets the timeout bit (32) of the word sparsepr_dense_check reads and
+    # clears; the CUDA context stays usable afterwards.
+    assert N.sparsepr_dense_check() == 0
+    N.wait_selftest()
+    assert N.sparsepr_dense_check() & 32
+    assert N.sparsepr_dense_check() == 0
+    x = torch.arange(8, dtype=torch.float32, device="cuda")
+    assert float(x.sum()) == 28.0
