@@ -9,26 +9,29 @@
 //           (max, sum, numerator) for a later combine (paper S4.2, App. A.2).
 //
 // Warp roles (384 threads; twelve warps so each SM sub-partition holds three):
-//   warps 0-3, 4-7  softmax of tile A, of tile B: thread r owns query row r = TMEM lane r;
-//              reads its S row from TMEM, online softmax in base 2 with lazy rescaling
-//              (O is rescaled only when the row max grows by more than 2^8), writes P as
-//              bf16 pairs into the TMEM columns of S already read, epilogue;
-//   warps 8-10 producers: 16-byte cp.async gathers of the Q tiles; one thread copies the
-//              K/V tiles with TMA (2-D tiled boxes, 128-byte swizzle) into the stages (two
-//              at d = 128, four at d = 64) shared by both query tiles.  Dense and probe
-//              keys are consecutive rows (64-row boxes).  Sparse keys are the concatenated
-//              row ranges of the selected K/V groups, each range starting at a multiple of
-//              four key positions (its last up-to-three positions are padding): a range is
-//              copied in boxes of 64, 16 and 4 rows, and the padding columns of S are set to
-//              -inf by the softmax warps before they read the tile;
+//   warps 0-3, 4-7  softmax of tile A, of tile B (or, for an item of one query tile and
+//              several key tiles, of the even and the odd key tiles of that tile, merged
+//              at the end): thread r owns query row r = TMEM lane r; reads its S row from
+//              TMEM, online softmax in base 2 with lazy rescaling (O is rescaled only when
+//              the row max grows by more than 2^8), writes P as bf16 pairs into the TMEM
+//              columns of S already read, epilogue;
+//   warps 8-10 producers: 16-byte cp.async gathers of the Q tiles; then one thread copies
+//              K tiles and another V tiles into their stages (two at d = 128, four at
+//              d = 64).  Dense and probe keys are consecutive rows: TMA boxes of 64 rows
+//              from a 3-D tensor map.  Sparse keys are the concatenated runs of the
+//              selected K/V groups in the tensor-core K/V layout (each group padded with
+//              zero rows to a multiple of 8, panels stored in shared-memory swizzle order),
+//              one bulk copy per run and panel; the K thread also publishes each tile's
+//              padding columns in a ring of mask slots;
 //   warp 11    one thread issues tcgen05.mma: S_t = Q_t K_j^T (both operands in shared
 //              memory) and O_t += P_t V_j (P read from TMEM, V MN-major), and commits to
-//              mbarriers.  The warp owns the TMEM allocation: S_A, S_B (128 columns each),
-//              O_A, O_B (128 each).
-// Issue order per key tile: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): the softmax of one tile
-// overlaps the matrix products of the other.  tcgen05.commit arrives only when every
-// earlier tcgen05 operation of the thread is complete, so "S_t(j) ready" also certifies
-// that PV_t(j-1) has finished reading P_t and updating O_t.
+//              mbarriers (K stages are released after the S products, V stages after the
+//              PV products).  The warp owns the TMEM allocation: two S buffers and two O
+//              accumulators (128 columns each).
+// Issue order per key tile with two query tiles: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): the
+// softmax of one tile overlaps the matrix products of the other.  tcgen05.commit arrives
+// only when every earlier tcgen05 operation of the thread is complete, so "S_t(j) ready"
+// also certifies that PV_t(j-1) has finished reading P_t and updating O_t.
 //
 // Every mbarrier wait is bounded: on timeout the CTA records kErrHang, all roles stop,
 // the MMA thread drains its outstanding MMAs and the TMEM is freed before returning.
